@@ -1,0 +1,321 @@
+"""Pins of the fp64 oracle against facts fixed outside the oracle itself.
+
+Each test ties one oracle function to something independent of it: the
+exhaustive integer identity of the signed nibble split (maplevalley article,
+section 2.3), library routines (numpy integer matmul, scipy's Jensen-Shannon
+distance, torch fp64 softmax / scaled_dot_product_attention), closed forms
+derived by hand for degenerate inputs, and brute-force subset enumeration
+for the gamma-coverage rule (FAST-Prefill article, section 3.1).
+"""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+from scipy.spatial.distance import jensenshannon
+from scipy.special import softmax as sp_softmax
+
+from oracle import oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rand_problem(S, Hq, Hkv, d, b, seed, int8=False, scale=1.0):
+    g = torch.Generator().manual_seed(seed)
+    q = (torch.randn(Hq, S, d, generator=g) * scale).to(torch.bfloat16)
+    k = (torch.randn(Hkv, S, d, generator=g) * scale).to(torch.bfloat16)
+    v = torch.randn(Hkv, S, d, generator=g).to(torch.bfloat16)
+    if not int8:
+        return orc.OracleProblem(q, k, v, b), (q, k, v, None, None, None, None)
+    q8 = torch.randint(-127, 128, (Hq, S, d), generator=g, dtype=torch.int8)
+    k8 = torch.randint(-127, 128, (Hkv, S, d), generator=g, dtype=torch.int8)
+    qs = torch.rand(Hq, generator=g) * 0.05 + 0.01
+    ks = torch.rand(Hkv, generator=g) * 0.05 + 0.01
+    return (orc.OracleProblem(q, k, v, b, q8=q8, k8=k8, q_scale=qs, k_scale=ks),
+            (q, k, v, q8, k8, qs, ks))
+
+
+# ---------------------------------------------------------------- int8 arithmetic
+
+def test_nibble_identity_exhaustive():
+    """a*b == aL*bL + (aH*bL + aL*bH)*16 + aH*bH*256 for every signed int8 pair."""
+    L = orc.lib()
+    for a in range(-128, 128):
+        got = [L.orc_nibble_mul(a, bb) for bb in range(-128, 128)]
+        assert got == [a * bb for bb in range(-128, 128)], a
+
+
+def test_int_score_tile_matches_integer_matmul():
+    P, (q, k, v, q8, k8, qs, ks) = rand_problem(S=256, Hq=4, Hkv=2, d=128, b=128, seed=3, int8=True)
+    for h in (0, 3):
+        tile = P.qk_int_tile(h, 128, 64, 64, 96)
+        ref = (q8[h, 128:192].to(torch.int64) @ k8[h // 2, 64:160].to(torch.int64).T).numpy()
+        assert np.array_equal(tile.astype(np.int64), ref)
+
+
+def test_int8_logit_bound_fits_int32_and_fp64():
+    # |sum| <= 127*128*128 < 2^31 and < 2^53: the oracle's integer sums are exact.
+    assert 127 * 128 * 128 < 2 ** 31
+
+
+# ---------------------------------------------------------------- Jensen-Shannon
+
+def test_jsd_matches_scipy():
+    rng = np.random.default_rng(0)
+    for n in (2, 7, 64, 1024):
+        p = rng.random(n); p /= p.sum()
+        q = rng.random(n) ** 3; q /= q.sum()
+        ref = jensenshannon(p, q) ** 2          # natural log, squared distance = divergence
+        assert abs(orc.jsd(p, q) - ref) < 1e-12
+        assert abs(orc.jsd(p, q) - orc.jsd(q, p)) < 1e-15
+
+
+def test_jsd_special_values():
+    p = np.array([0.2, 0.3, 0.5])
+    assert orc.jsd(p, p) == 0.0
+    assert abs(orc.jsd([1.0, 0.0], [0.0, 1.0]) - math.log(2.0)) < 1e-15
+    # Worked by hand: p = (1/2, 1/2), q = (1, 0), m = (3/4, 1/4):
+    # JSD = 1/2 [1/2 ln(2/3) + 1/2 ln 2] + 1/2 ln(4/3).
+    hand = 0.5 * (0.5 * math.log(0.5 / 0.75) + 0.5 * math.log(0.5 / 0.25)) + 0.5 * math.log(1.0 / 0.75)
+    assert abs(orc.jsd([0.5, 0.5], [1.0, 0.0]) - hand) < 1e-15
+    rng = np.random.default_rng(1)
+    for _ in range(20):
+        a = rng.random(16); a /= a.sum()
+        b = rng.random(16) ** 4; b /= b.sum()
+        assert 0.0 <= orc.jsd(a, b) <= math.log(2.0) + 1e-15
+
+
+# ---------------------------------------------------------------- selection
+
+def brute_min_cover(w, r, gamma):
+    others = [c for c in range(r)]
+    for k in range(0, r + 1):
+        best = None
+        for comb in itertools.combinations(others, k):
+            cov = w[r] + sum(w[c] for c in comb)
+            if cov >= gamma:
+                best = comb if best is None else best
+                break
+        if best is not None:
+            return k + 1
+    return r + 1
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_selection_minimal_by_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    r = int(rng.integers(0, 11))
+    w = rng.random(r + 1) ** float(rng.integers(1, 6))
+    w /= w.sum()
+    for gamma in (0.3, 0.5, 0.8, 0.9, 0.95, 0.999):
+        sel, info = orc.select(w, r, gamma)
+        assert r in sel
+        assert list(sel) == sorted(set(sel.tolist()))
+        cov = w[sel].sum()
+        assert cov >= gamma - 1e-12 or len(sel) == r + 1
+        assert len(sel) == brute_min_cover(w, r, gamma)
+        # The kept non-diagonal blocks are the highest-scoring ones.
+        rest = [c for c in range(r) if c not in sel]
+        kept = [c for c in sel if c != r]
+        if kept and rest:
+            assert min(w[kept]) >= max(w[rest])
+
+
+def test_selection_gamma_one_keeps_every_causal_block():
+    w = np.full(9, 1.0 / 9)
+    sel, _ = orc.select(w, 8, 1.0)
+    assert list(sel) == list(range(9))
+
+
+def test_selection_diagonal_alone_when_it_covers():
+    w = np.array([0.05, 0.05, 0.9])
+    sel, info = orc.select(w, 2, 0.9)
+    assert list(sel) == [2] and info[0] == -1.0
+
+
+def test_selection_ties_break_by_lower_index():
+    w = np.array([0.2, 0.2, 0.2, 0.2, 0.2])
+    sel, _ = orc.select(w, 4, 0.6)
+    assert list(sel) == [0, 1, 4]
+
+
+# ---------------------------------------------------------------- block scores
+
+def test_vs_scores_hand_example():
+    ex = json.load(open(os.path.join(GOLDEN, "vs_scores_example.json")))
+    w = orc.row_scores(orc.VS, ex["r"], ex["vhat"], ex["shat"], np.zeros(4), np.zeros((len(ex["vhat"]), 4)))
+    assert np.allclose(w, ex["expected"], atol=1e-15)
+
+
+def test_qa_scores_match_scipy_softmax():
+    rng = np.random.default_rng(5)
+    kbar = rng.normal(size=(12, 16))
+    qbar = rng.normal(size=16) * 3
+    for r in (0, 5, 11):
+        w = orc.row_scores(orc.QA, r, np.zeros(12), np.zeros(12), qbar, kbar)
+        ref = sp_softmax(kbar[: r + 1] @ qbar / math.sqrt(16))
+        assert np.allclose(w, ref, rtol=1e-13, atol=1e-16)
+    pe = orc.pest(qbar, kbar)
+    assert np.allclose(pe, sp_softmax(kbar @ qbar / 4.0), rtol=1e-13)
+
+
+# ---------------------------------------------------------------- last-block statistics
+
+@pytest.mark.parametrize("S,b,d,int8", [(16, 4, 8, False), (24, 8, 16, False), (32, 8, 8, True)])
+def test_last_block_stats_against_full_attention_matrix(S, b, d, int8):
+    """vhat / shat from the full causal softmax matrix (torch fp64), pooled
+    by block columns and by torch.diagonal sums."""
+    P, (q, k, v, q8, k8, qs, ks) = rand_problem(S, 2, 1, d, b, seed=S + b, int8=int8, scale=2.0)
+    n = S // b
+    for h in range(2):
+        if int8:
+            logits = (q8[h].double() @ k8[0].double().T) * (float(qs[h]) * float(ks[0])) / math.sqrt(d)
+        else:
+            logits = (q[h].double() @ k[0].double().T) / math.sqrt(d)
+        mask = torch.ones(S, S, dtype=torch.bool).tril()
+        A = torch.softmax(logits.masked_fill(~mask, float("-inf")), dim=-1)
+        last = A[(n - 1) * b:]
+        vref = last.reshape(b, n, b).sum(dim=(0, 2)) / b
+        sref = torch.zeros(n, dtype=torch.float64)
+        for delta in range(S):
+            diag = torch.diagonal(A, offset=-delta)            # entries (p, p - delta)
+            rows = torch.arange(delta, S)
+            sref[delta // b] += diag[rows >= (n - 1) * b].sum() / b
+        vh, sh, err = P.last_block_stats(h)
+        assert err < 1e-12
+        assert np.allclose(vh, vref.numpy(), atol=1e-14)
+        assert np.allclose(sh, sref.numpy(), atol=1e-14)
+        assert abs(vh.sum() - 1) < 1e-13 and abs(sh.sum() - 1) < 1e-13
+
+
+def test_uniform_attention_closed_form():
+    """Q = 0 makes every causal row uniform: A_pj = 1/(p+1).  Then
+    vhat[c] = (1/b) sum_i |block c and [0, p_i]| / (p_i + 1) and
+    shat[o] = (1/b) sum_i |{delta in [ob, (o+1)b) : delta <= p_i}| / (p_i + 1)."""
+    S, b, d = 24, 6, 8
+    n = S // b
+    q = torch.zeros(1, S, d, dtype=torch.bfloat16)
+    g = torch.Generator().manual_seed(9)
+    k = torch.randn(1, S, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, S, d, generator=g).to(torch.bfloat16)
+    P = orc.OracleProblem(q, k, v, b)
+    vh, sh, _ = P.last_block_stats(0)
+    vf = [Fraction(0)] * n
+    sf = [Fraction(0)] * n
+    for i in range(b):
+        p = (n - 1) * b + i
+        for c in range(n):
+            vf[c] += Fraction(max(0, min(p, (c + 1) * b - 1) - c * b + 1), (p + 1) * b)
+            sf[c] += Fraction(max(0, min(p, (c + 1) * b - 1) - c * b + 1), (p + 1) * b)
+    assert np.allclose(vh, [float(x) for x in vf], atol=1e-15)
+    assert np.allclose(sh, [float(x) for x in sf], atol=1e-15)
+    out = P.build_index_head(0, 0.9, 0.1)
+    assert np.allclose(out["pest"], np.full(n, 1.0 / n), atol=1e-15)   # qbar = 0 -> uniform
+
+
+def test_single_block_is_query_aware_with_zero_divergence():
+    P, _ = rand_problem(S=16, Hq=1, Hkv=1, d=8, b=16, seed=4)
+    out = P.build_index_head(0, 0.9, 0.1)
+    assert abs(out["jsd"]) < 1e-15 and out["pattern"] == orc.QA
+    assert [list(r) for r in out["rows"]] == [[0]]
+    out = P.build_index_head(0, 0.9, -1.0)            # jsd < -1 never holds
+    assert out["pattern"] == orc.VS
+
+
+def test_block_means_match_torch():
+    P, (q, k, v, q8, k8, qs, ks) = rand_problem(S=64, Hq=2, Hkv=1, d=16, b=16, seed=2, int8=True)
+    qb = P.block_means("q", 1)
+    ref = (q8[1].double().reshape(4, 16, 16).sum(1) * float(qs[1])) / 16
+    assert np.allclose(qb, ref.numpy(), rtol=1e-15)
+    P2, (q, k, *_r) = rand_problem(S=64, Hq=2, Hkv=1, d=16, b=16, seed=2)
+    assert np.allclose(P2.block_means("k", 0), k[0].double().reshape(4, 16, 16).mean(1).numpy(), atol=1e-15)
+
+
+# ---------------------------------------------------------------- attention
+
+def sdpa_ref(q, k, v, h, g, mask=None, int8=None):
+    d = q.shape[-1]
+    if int8 is not None:
+        q8, k8, qs, ks = int8
+        logits = (q8[h].double() @ k8[h // g].double().T) * (float(qs[h]) * float(ks[h // g])) / math.sqrt(d)
+    else:
+        logits = (q[h].double() @ k[h // g].double().T) / math.sqrt(d)
+    S = q.shape[1]
+    causal = torch.ones(S, S, dtype=torch.bool).tril()
+    m = causal if mask is None else (causal & mask)
+    A = torch.softmax(logits.masked_fill(~m, float("-inf")), dim=-1)
+    return A @ v[h // g].double()
+
+
+@pytest.mark.parametrize("int8", [False, True])
+def test_gamma_one_equals_dense_causal_attention(int8):
+    S, b, d = 48, 8, 16
+    P, (q, k, v, q8, k8, qs, ks) = rand_problem(S, 4, 2, d, b, seed=11, int8=int8, scale=1.5)
+    for h in range(4):
+        idx = P.build_index_head(h, 1.0, 0.1)
+        assert all(list(r) == list(range(i + 1)) for i, r in enumerate(idx["rows"]))
+        got = np.concatenate([P.attn_rows(h, r * b, (r + 1) * b, idx["rows"][r]) for r in range(S // b)])
+        ref = sdpa_ref(q, k, v, h, 2, int8=(q8, k8, qs, ks) if int8 else None)
+        assert np.allclose(got, ref.numpy(), atol=1e-12)
+    if not int8:
+        sd = torch.nn.functional.scaled_dot_product_attention(
+            q.double()[None], k.double().repeat_interleave(2, 0)[None], v.double().repeat_interleave(2, 0)[None],
+            is_causal=True)[0]
+        got = np.concatenate([P.attn_rows(1, r * b, (r + 1) * b, list(range(r + 1))) for r in range(S // b)])
+        assert np.allclose(got, sd[1].numpy(), atol=1e-12)
+
+
+def test_sparse_attention_matches_block_masked_softmax():
+    S, b, d = 64, 8, 16
+    n = S // b
+    P, (q, k, v, *_r) = rand_problem(S, 2, 1, d, b, seed=21)
+    rng = np.random.default_rng(2)
+    for h in range(2):
+        lists = [sorted(set(rng.choice(r + 1, size=int(rng.integers(1, r + 2)), replace=False).tolist()) | {r})
+                 for r in range(n)]
+        mask = torch.zeros(S, S, dtype=torch.bool)
+        for r, blocks in enumerate(lists):
+            for c in blocks:
+                mask[r * b:(r + 1) * b, c * b:(c + 1) * b] = True
+        ref = sdpa_ref(q, k, v, h, 2, mask=mask)
+        got = np.concatenate([P.attn_rows(h, r * b, (r + 1) * b, lists[r]) for r in range(n)])
+        assert np.allclose(got, ref.numpy(), atol=1e-12)
+
+
+def test_index_invariants_on_planted_inputs():
+    from dynamic_block_sparse_last_b200 import synth
+    w = synth.Workload("t", S=1024, Hq=4, Hkv=2, b=128, seed=0, kinds=["vs", "qa", "vs", "qa"])
+    x = synth.make_inputs(w)
+    P = orc.OracleProblem(x["q"], x["k"], x["v"], w.b)
+    for h in range(4):
+        out = P.build_index_head(h, w.gamma, w.tau)
+        assert out["rowsum_err"] < 1e-12
+        assert abs(out["vhat"].sum() - 1) < 1e-12 and abs(out["shat"].sum() - 1) < 1e-12
+        assert abs(out["pest"].sum() - 1) < 1e-12
+        for r, row in enumerate(out["rows"]):
+            assert r in row
+            sc = out["scores"][r]
+            assert abs(sc.sum() - 1) < 1e-12
+            assert sc[row].sum() >= w.gamma - 1e-12
+            others = [c for c in row if c != r]
+            if others:                                  # minimal: dropping the weakest falls short
+                assert sc[row].sum() - sc[others].min() < w.gamma
+
+
+def test_golden_tiny_index_regression():
+    """Regression against the stored output of tests/golden/make_golden.py."""
+    from dynamic_block_sparse_last_b200 import synth
+    gold = json.load(open(os.path.join(GOLDEN, "tiny_index.json")))
+    w = synth.WORKLOADS["tiny"]
+    x = synth.make_inputs(w)
+    P = orc.OracleProblem(x["q"], x["k"], x["v"], w.b)
+    for h, gh in enumerate(gold["heads"]):
+        out = P.build_index_head(h, w.gamma, w.tau)
+        assert out["pattern"] == gh["pattern"]
+        assert abs(out["jsd"] - gh["jsd"]) < 1e-12
+        assert np.allclose(out["vhat"], gh["vhat"], atol=1e-14)
+        assert [list(map(int, r)) for r in out["rows"]] == gh["rows"]

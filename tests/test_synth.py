@@ -1,0 +1,60 @@
+"""The seeded input generator: determinism, rotary-embedding relative-position
+property, planted structure bookkeeping and the int8 quantisation bounds."""
+import math
+
+import torch
+
+from dynamic_block_sparse_last_b200 import synth
+
+
+def small(**kw):
+    base = dict(name="t", S=512, Hq=4, Hkv=2, seed=7)
+    base.update(kw)
+    return synth.Workload(**base)
+
+
+def test_same_seed_same_tensors():
+    a = synth.make_inputs(small())
+    b = synth.make_inputs(small())
+    c = synth.make_inputs(small(seed=8))
+    for key in ("q", "k", "v"):
+        assert torch.equal(a[key], b[key])
+        assert not torch.equal(a[key], c[key])
+        assert a[key].dtype == torch.bfloat16 and a[key].is_contiguous()
+
+
+def test_rope_dot_products_depend_on_offset_only():
+    g = torch.Generator().manual_seed(0)
+    u = torch.randn(1, 1, 128, generator=g, dtype=torch.float64)
+    w = torch.randn(1, 1, 128, generator=g, dtype=torch.float64)
+    S = 64
+    U = synth.rope_(u.expand(1, S, 128).clone().float()).double()
+    W = synth.rope_(w.expand(1, S, 128).clone().float()).double()
+    d1 = float(U[0, 40] @ W[0, 30])
+    d2 = float(U[0, 20] @ W[0, 10])
+    assert abs(d1 - d2) < 1e-3 * max(1.0, abs(d1))
+    assert abs(float(U[0, 5].norm()) - float(u.norm())) < 1e-4
+
+
+def test_head_kinds_split_groups_in_half():
+    w = synth.WORKLOADS["llama3b"]
+    kinds = w.head_kinds()
+    g = w.Hq // w.Hkv
+    assert kinds == ["vs"] * (g * w.Hkv // 2) + ["qa"] * (g * w.Hkv // 2)
+    assert synth.WORKLOADS["tiny"].head_kinds() == ["vs", "qa", "vs", "qa"]
+
+
+def test_int8_quantisation_bounds():
+    x = synth.make_inputs(small(int8=True))
+    for key, skey in (("q8", "q_scale"), ("k8", "k_scale")):
+        x8, sc = x[key], x[skey]
+        src = x[key[0]].float()
+        for h in range(x8.shape[0]):
+            assert int(x8[h].abs().max()) == 127
+            err = (x8[h].float() * sc[h] - src[h]).abs().max()
+            assert float(err) <= float(sc[h]) * 0.5 * (1 + 1e-6)
+
+
+def test_dense_equivalent_flops():
+    assert synth.dense_equiv_flops(131072, 32, 128) == 2.0 * 32 * 128 * 131072 ** 2
+    assert math.isclose(synth.dense_equiv_flops(131072, 32, 128), 1.407e14, rel_tol=1e-3)
