@@ -1,0 +1,427 @@
+// fp_sparse.cu -- host side of the C ABI declared in include/fp_sparse.h:
+// argument validation, the library-owned index workspace, TMA tensor maps
+// and the kernel launches.  Every step of the computation runs in the CUDA
+// kernels of index_kernels.cuh and attn_kernel.cuh; there is no host
+// fallback.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "attn_kernel.cuh"
+#include "fp_sparse.h"
+#include "index_kernels.cuh"
+
+using namespace fpk;
+
+// One sticky error word per device (module-scope device variable).
+static __device__ int g_fp_dev_error;
+
+struct fp_index {
+  int S, Hq, Hkv, d, b, n, nch, g;
+  int device;
+  int built;
+  int qk_dtype;
+  int R2, chunks_per_part;
+  void *slab;
+  size_t slab_bytes;
+  float *pm, *plo, *phi;   // [Hq][nch][b]
+  float *partM, *partL;    // [Hq][R2][b]
+  float *LOc, *HIc;        // [Hq][nch]
+  float *ksum;             // [Hkv][nch][128]
+  float *kbar;             // [Hkv][n][128]
+  float *qbar;             // [Hq][n][128]
+  float *vhat, *shat, *pest;  // [Hq][n]
+  float *jsd;              // [Hq]
+  int *pattern;            // [Hq]
+  int *counts;             // [Hq][n]
+  int *cols;               // [Hq][n(n+1)/2]
+};
+
+namespace {
+
+std::mutex g_mu;
+int *g_err_ptr[128] = {nullptr};
+
+int *device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fp_dev_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<int *>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a [rows][128] tensor: boxes of 128 rows x 128 bytes
+// (64 bf16 or 128 int8 columns), 128-byte swizzle.
+bool make_map(CUtensorMap *m, const void *ptr, bool i8, uint64_t rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(128 * (i8 ? 1 : 2))};
+  const cuuint32_t box[2] = {i8 ? 128u : 64u, 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool shape_ok(int S, int Hq, int Hkv, int d, int b) {
+  if (d != 128) return false;
+  if (b != 128 && b != 256) return false;
+  if (S <= 0 || S % b != 0 || S / b > kSelMaxN) return false;
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return false;
+  if ((int64_t)Hq * S > (int64_t)INT32_MAX || (int64_t)Hkv * S > (int64_t)INT32_MAX) return false;
+  return true;
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <typename T>
+T *carve(char *&cur, size_t count) {
+  T *p = reinterpret_cast<T *>(cur);
+  cur += ((count * sizeof(T) + 255) / 256) * 256;
+  return p;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? FP_OK : FP_ERR_CUDA; }
+
+template <bool I8>
+int set_smem_attrs() {
+  static bool done[128] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 128 && done[dev]) return FP_OK;
+  if (cudaFuncSetAttribute(k_score_last<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           ScoreCfg<I8>::kSmem) != cudaSuccess)
+    return FP_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_sparse_attn<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           AttnCfg<I8>::kSmem) != cudaSuccess)
+    return FP_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (kSelRows * kSelMaxN + kSelRows * 128 + 32 * 129) * 4) != cudaSuccess)
+    return FP_ERR_CUDA;
+  if (dev >= 0 && dev < 128) done[dev] = true;
+  return FP_OK;
+}
+
+template <bool I8>
+int build_index_impl(const void *q, const void *k, float gamma, float tau, const float *q_scale,
+                     const float *k_scale, fp_index *I, cudaStream_t st) {
+  int rc = set_smem_attrs<I8>();
+  if (rc) return rc;
+  int *err = device_error_word();
+  if (!err) return FP_ERR_CUDA;
+  CUtensorMap tq, tk;
+  if (!make_map(&tq, q, I8, (uint64_t)I->Hq * I->S) || !make_map(&tk, k, I8, (uint64_t)I->Hkv * I->S))
+    return FP_ERR_CUDA;
+  const int tiles_per_group = I->g * (I->b / 128);
+  const int tgroups = (tiles_per_group + 3) / 4;
+  int R = sm_count() / (tgroups * I->Hkv);
+  if (R < 1) R = 1;
+  if (R > I->nch) R = I->nch;
+  int cpc = (I->nch + R - 1) / R;
+  R = (I->nch + cpc - 1) / cpc;
+  ScoreParams sp;
+  sp.S = I->S; sp.Hq = I->Hq; sp.Hkv = I->Hkv; sp.b = I->b; sp.n = I->n; sp.nch = I->nch; sp.g = I->g;
+  sp.tiles_per_group = tiles_per_group;
+  sp.chunks_per_cta = cpc;
+  sp.scale2 = kLog2e / sqrtf((float)I->d);
+  sp.q_scale = q_scale;
+  sp.k_scale = k_scale;
+  sp.pm = I->pm; sp.plo = I->plo; sp.phi = I->phi; sp.ksum = I->ksum;
+  sp.err = err;
+  k_score_last<I8><<<dim3(R, tgroups, I->Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
+  if ((rc = launch_status())) return rc;
+
+  k_row_stats<<<dim3(I->Hq, I->R2), I->b, 0, st>>>(I->pm, I->plo, I->phi, I->nch, I->b,
+                                                   I->chunks_per_part, I->partM, I->partL);
+  if ((rc = launch_status())) return rc;
+  const size_t red_bytes = (size_t)(I->b / 32) * I->chunks_per_part * 2 * sizeof(float);
+  k_block_mass<<<dim3(I->Hq, I->R2), I->b, red_bytes, st>>>(I->pm, I->plo, I->phi, I->partM, I->partL,
+                                                            I->nch, I->b, I->chunks_per_part, I->LOc,
+                                                            I->HIc);
+  if ((rc = launch_status())) return rc;
+  k_kbar<<<dim3(I->n, I->Hkv), 128, 0, st>>>(I->ksum, I->nch, I->b, I->n, I->kbar);
+  if ((rc = launch_status())) return rc;
+  const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
+  k_pattern<I8><<<I->Hq, 1024, 0, st>>>(q, q_scale, I->LOc, I->HIc, I->kbar, I->S, I->g, I->b, I->n,
+                                        I->nch, inv_sqrt_d, tau, I->vhat, I->shat, I->pest, I->jsd,
+                                        I->pattern);
+  if ((rc = launch_status())) return rc;
+  k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->b, I->n, I->qbar);
+  if ((rc = launch_status())) return rc;
+  const size_t sel_bytes = (size_t)(kSelRows * I->n + kSelRows * 128 + 32 * 129) * sizeof(float);
+  k_select<<<dim3((I->n + kSelRows - 1) / kSelRows, I->Hq), 256, sel_bytes, st>>>(
+      I->pattern, I->vhat, I->shat, I->qbar, I->kbar, I->g, I->n, inv_sqrt_d, gamma, I->counts, I->cols);
+  return launch_status();
+}
+
+template <bool I8>
+int attn_impl(const void *q, const void *k, const void *v, const float *q_scale, const float *k_scale,
+              const fp_index *I, void *out, cudaStream_t st) {
+  int rc = set_smem_attrs<I8>();
+  if (rc) return rc;
+  int *err = device_error_word();
+  if (!err) return FP_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, I8, (uint64_t)I->Hq * I->S) || !make_map(&tk, k, I8, (uint64_t)I->Hkv * I->S) ||
+      !make_map(&tv, v, false, (uint64_t)I->Hkv * I->S))
+    return FP_ERR_CUDA;
+  AttnParams ap;
+  ap.S = I->S; ap.Hq = I->Hq; ap.Hkv = I->Hkv; ap.b = I->b; ap.n = I->n; ap.g = I->g;
+  ap.counts = I->counts;
+  ap.cols = I->cols;
+  ap.q_scale = q_scale;
+  ap.k_scale = k_scale;
+  ap.scale2 = kLog2e / sqrtf((float)I->d);
+  ap.out = static_cast<__nv_bfloat16 *>(out);
+  ap.err = err;
+  const unsigned grid = (unsigned)I->Hq * (unsigned)(I->S / 128);
+  k_sparse_attn<I8><<<grid, AttnCfg<I8>::kThreads, AttnCfg<I8>::kSmem, st>>>(tq, tk, tv, ap);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out) {
+  if (!out) return FP_ERR_ARG;
+  *out = nullptr;
+  if (!shape_ok(S, Hq, Hkv, d, b)) return FP_ERR_ARG;
+  fp_index *I = static_cast<fp_index *>(calloc(1, sizeof(fp_index)));
+  if (!I) return FP_ERR_CUDA;
+  I->S = S; I->Hq = Hq; I->Hkv = Hkv; I->d = d; I->b = b;
+  I->n = S / b; I->nch = S / 128; I->g = Hq / Hkv;
+  I->R2 = I->nch < 16 ? I->nch : 16;
+  I->chunks_per_part = (I->nch + I->R2 - 1) / I->R2;
+  I->R2 = (I->nch + I->chunks_per_part - 1) / I->chunks_per_part;
+  cudaGetDevice(&I->device);
+  const size_t n = I->n, nch = I->nch, bb = b;
+  const size_t tri = n * (n + 1) / 2;
+  size_t need = 0;
+  auto add = [&](size_t bytes) { need += ((bytes + 255) / 256) * 256; };
+  for (int i = 0; i < 3; ++i) add((size_t)Hq * nch * bb * 4);
+  for (int i = 0; i < 2; ++i) add((size_t)Hq * I->R2 * bb * 4);
+  for (int i = 0; i < 2; ++i) add((size_t)Hq * nch * 4);
+  add((size_t)Hkv * nch * 128 * 4);
+  add((size_t)Hkv * n * 128 * 4);
+  add((size_t)Hq * n * 128 * 4);
+  for (int i = 0; i < 3; ++i) add((size_t)Hq * n * 4);
+  add((size_t)Hq * 4);
+  add((size_t)Hq * 4);
+  add((size_t)Hq * n * 4);
+  add((size_t)Hq * tri * 4);
+  if (cudaMalloc(&I->slab, need) != cudaSuccess) {
+    free(I);
+    return FP_ERR_CUDA;
+  }
+  I->slab_bytes = need;
+  char *cur = static_cast<char *>(I->slab);
+  I->pm = carve<float>(cur, (size_t)Hq * nch * bb);
+  I->plo = carve<float>(cur, (size_t)Hq * nch * bb);
+  I->phi = carve<float>(cur, (size_t)Hq * nch * bb);
+  I->partM = carve<float>(cur, (size_t)Hq * I->R2 * bb);
+  I->partL = carve<float>(cur, (size_t)Hq * I->R2 * bb);
+  I->LOc = carve<float>(cur, (size_t)Hq * nch);
+  I->HIc = carve<float>(cur, (size_t)Hq * nch);
+  I->ksum = carve<float>(cur, (size_t)Hkv * nch * 128);
+  I->kbar = carve<float>(cur, (size_t)Hkv * n * 128);
+  I->qbar = carve<float>(cur, (size_t)Hq * n * 128);
+  I->vhat = carve<float>(cur, (size_t)Hq * n);
+  I->shat = carve<float>(cur, (size_t)Hq * n);
+  I->pest = carve<float>(cur, (size_t)Hq * n);
+  I->jsd = carve<float>(cur, (size_t)Hq);
+  I->pattern = carve<int>(cur, (size_t)Hq);
+  I->counts = carve<int>(cur, (size_t)Hq * n);
+  I->cols = carve<int>(cur, (size_t)Hq * tri);
+  *out = I;
+  return FP_OK;
+}
+
+void fp_index_free(fp_index *I) {
+  if (!I) return;
+  cudaDeviceSynchronize();
+  if (I->slab) cudaFree(I->slab);
+  free(I);
+}
+
+int fp_build_index(const void *q, const void *k, int S, int Hq, int Hkv, int d, int b, float gamma,
+                   float tau, int qk_dtype, const float *q_scale, const float *k_scale, fp_index *idx,
+                   void *stream) {
+  if (!idx || !q || !k) return FP_ERR_ARG;
+  if (!shape_ok(S, Hq, Hkv, d, b)) return FP_ERR_ARG;
+  if (S != idx->S || Hq != idx->Hq || Hkv != idx->Hkv || d != idx->d || b != idx->b) return FP_ERR_STATE;
+  if (!(gamma > 0.f && gamma <= 1.f) || !(tau >= 0.f) || std::isnan(gamma) || std::isnan(tau)) return FP_ERR_ARG;
+  if (qk_dtype != FP_QK_BF16 && qk_dtype != FP_QK_INT8) return FP_ERR_ARG;
+  if (qk_dtype == FP_QK_INT8 && (!q_scale || !k_scale)) return FP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k)) return FP_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  idx->built = 0;
+  const int rc = qk_dtype == FP_QK_INT8 ? build_index_impl<true>(q, k, gamma, tau, q_scale, k_scale, idx, st)
+                                        : build_index_impl<false>(q, k, gamma, tau, nullptr, nullptr, idx, st);
+  if (rc == FP_OK) {
+    idx->built = 1;
+    idx->qk_dtype = qk_dtype;
+  }
+  return rc;
+}
+
+int fp_sparse_attn(const void *q, const void *k, const void *v, const float *q_scale, const float *k_scale,
+                   const fp_index *idx, void *out, void *stream) {
+  if (!idx || !q || !k || !v || !out) return FP_ERR_ARG;
+  if (!idx->built) return FP_ERR_STATE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FP_ERR_ARG;
+  if (idx->qk_dtype == FP_QK_INT8 && (!q_scale || !k_scale)) return FP_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return idx->qk_dtype == FP_QK_INT8 ? attn_impl<true>(q, k, v, q_scale, k_scale, idx, out, st)
+                                     : attn_impl<false>(q, k, v, nullptr, nullptr, idx, out, st);
+}
+
+int fp_index_info(const fp_index *idx, int *S, int *Hq, int *Hkv, int *d, int *b, int *qk_dtype) {
+  if (!idx) return FP_ERR_ARG;
+  if (S) *S = idx->S;
+  if (Hq) *Hq = idx->Hq;
+  if (Hkv) *Hkv = idx->Hkv;
+  if (d) *d = idx->d;
+  if (b) *b = idx->b;
+  if (qk_dtype) *qk_dtype = idx->qk_dtype;
+  return FP_OK;
+}
+
+int fp_index_nnz(const fp_index *idx, int64_t *nnz, void *stream) {
+  if (!idx || !nnz) return FP_ERR_ARG;
+  if (!idx->built) return FP_ERR_STATE;
+  std::vector<int> counts((size_t)idx->Hq * idx->n);
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP_ERR_CUDA;
+  if (cudaMemcpy(counts.data(), idx->counts, counts.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FP_ERR_CUDA;
+  int64_t s = 0;
+  for (int c : counts) s += c;
+  *nnz = s;
+  return FP_OK;
+}
+
+int fp_index_export(const fp_index *idx, int32_t *row_ptr, int32_t *col, uint8_t *pattern, float *jsd,
+                    float *vhat, float *shat, float *pest, void *stream) {
+  if (!idx) return FP_ERR_ARG;
+  if (!idx->built) return FP_ERR_STATE;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP_ERR_CUDA;
+  const size_t Hn = (size_t)idx->Hq * idx->n;
+  const size_t tri = (size_t)idx->n * (idx->n + 1) / 2;
+  if (row_ptr || col) {
+    std::vector<int> counts(Hn);
+    if (cudaMemcpy(counts.data(), idx->counts, Hn * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return FP_ERR_CUDA;
+    std::vector<int> padded;
+    if (col) {
+      padded.resize((size_t)idx->Hq * tri);
+      if (cudaMemcpy(padded.data(), idx->cols, padded.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return FP_ERR_CUDA;
+    }
+    int64_t pos = 0;
+    for (int h = 0; h < idx->Hq; ++h)
+      for (int r = 0; r < idx->n; ++r) {
+        const size_t row = (size_t)h * idx->n + r;
+        if (row_ptr) row_ptr[row] = (int32_t)pos;
+        const int c = counts[row];
+        if (col)
+          memcpy(col + pos, padded.data() + (size_t)h * tri + (size_t)r * (r + 1) / 2, (size_t)c * 4);
+        pos += c;
+      }
+    if (row_ptr) row_ptr[Hn] = (int32_t)pos;
+  }
+  if (pattern) {
+    std::vector<int> p(idx->Hq);
+    if (cudaMemcpy(p.data(), idx->pattern, p.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+      return FP_ERR_CUDA;
+    for (int h = 0; h < idx->Hq; ++h) pattern[h] = (uint8_t)p[h];
+  }
+  if (jsd && cudaMemcpy(jsd, idx->jsd, (size_t)idx->Hq * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FP_ERR_CUDA;
+  if (vhat && cudaMemcpy(vhat, idx->vhat, Hn * 4, cudaMemcpyDeviceToHost) != cudaSuccess) return FP_ERR_CUDA;
+  if (shat && cudaMemcpy(shat, idx->shat, Hn * 4, cudaMemcpyDeviceToHost) != cudaSuccess) return FP_ERR_CUDA;
+  if (pest && cudaMemcpy(pest, idx->pest, Hn * 4, cudaMemcpyDeviceToHost) != cudaSuccess) return FP_ERR_CUDA;
+  return FP_OK;
+}
+
+int fp_get_device_error(void *stream) {
+  int *err = device_error_word();
+  if (!err) return FP_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return FP_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(err, &zero, 4, cudaMemcpyHostToDevice) != cudaSuccess) return FP_ERR_CUDA;
+    return (v & kDevErrTimeout) ? FP_ERR_TIMEOUT : FP_ERR_CUDA;
+  }
+  return FP_OK;
+}
+
+int fp_debug_wait_timeout(int timeout_us, void *stream) {
+  if (timeout_us < 1 || timeout_us > 10000000) return FP_ERR_ARG;
+  int *err = device_error_word();
+  if (!err) return FP_ERR_CUDA;
+  k_wait_timeout<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((unsigned long long)timeout_us * 1000ull, err);
+  return launch_status();
+}
+
+int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int Hkv, int d, int h, int p0,
+                        int j0, int32_t *out, void *stream) {
+  if (!q8 || !k8 || !out || d != 128 || S <= 0 || S % 128 || Hq <= 0 || Hkv <= 0 || Hq % Hkv) return FP_ERR_ARG;
+  if (h < 0 || h >= Hq || p0 < 0 || j0 < 0 || p0 % 128 || j0 % 128 || p0 >= S || j0 >= S) return FP_ERR_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(out)) return FP_ERR_ARG;
+  int *err = device_error_word();
+  if (!err) return FP_ERR_CUDA;
+  CUtensorMap tq, tk;
+  if (!make_map(&tq, q8, true, (uint64_t)Hq * S) || !make_map(&tk, k8, true, (uint64_t)Hkv * S))
+    return FP_ERR_CUDA;
+  const int g = Hq / Hkv;
+  k_qk_tile_i8<<<1, 128, 32768 + 1024, static_cast<cudaStream_t>(stream)>>>(
+      tq, tk, h * S + p0, (h / g) * S + j0, out, err);
+  return launch_status();
+}
+
+const char *fp_strerror(int code) {
+  switch (code) {
+    case FP_OK: return "ok";
+    case FP_ERR_ARG: return "invalid argument";
+    case FP_ERR_CUDA: return "CUDA call failed";
+    case FP_ERR_TIMEOUT: return "device wait timed out";
+    case FP_ERR_STATE: return "index not built or built for another shape";
+    default: return "unknown error";
+  }
+}
+
+}  // extern "C"

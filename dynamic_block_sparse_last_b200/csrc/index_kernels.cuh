@@ -1,0 +1,730 @@
+// index_kernels.cuh -- sparse-index generation on sm_100a.
+//
+// Method (FAST-Prefill article, sections 1.2, 2.1 and 3.1; maplevalley
+// article, section 1.1): score the last query block of every head against
+// all keys, pool the softmax probabilities into vertical (per key block) and
+// slash (per diagonal offset block) statistics, decide the head's pattern by
+// the Jensen-Shannon divergence between the exact pooled distribution and
+// the block-mean estimate, then keep for every query block the smallest set
+// of key blocks (diagonal forced) whose normalised score reaches gamma.
+//
+// Kernels, in launch order:
+//   k_score_last   tcgen05 Q_last.K^T per 128-key chunk, K streamed once per
+//                  KV group through a TMA ring; per (row, chunk) max and the
+//                  two offset-half sums; per-chunk K column sums.  Nothing of
+//                  size S x b reaches global memory.
+//   k_row_stats    per (head, row, chunk range): running max / sum.
+//   k_block_mass   per (head, chunk): row-normalised lo/hi masses.
+//   k_kbar         block means of K.
+//   k_pattern      per head: vhat, shat, P_est, JSD, pattern.
+//   k_qbar         block means of Q for query-aware heads only.
+//   k_select       per (head, query block): scores, gamma cut, sorted list.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace fpk {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// k_score_last
+//
+// CTA = (KV head, group of up to 4 row tiles of 128 query rows of the last
+// block, range of 128-key chunks).  A "tile" is (query head of the group,
+// 128-row slice of the b-row last block).  Warps:
+//   0..15  statistics: warpgroup t owns tile t; thread = one query row
+//   16     TMA producer     17  MMA issuer + TMEM owner
+//   18,19  K column sums for the block means (only CTAs of tile group 0)
+// TMEM: tile t's 128x128 fp32 score tile at columns [128t, 128t+128).
+// ---------------------------------------------------------------------------
+struct ScoreParams {
+  int S, Hq, Hkv, b, n, nch, g;
+  int tiles_per_group;  // g * b / 128
+  int chunks_per_cta;
+  float scale2;          // log2(e)/sqrt(d) (bf16); int8: multiplied by per-head scales
+  const float *q_scale;  // int8 only
+  const float *k_scale;
+  float *pm, *plo, *phi;  // [Hq][nch][b]
+  float *ksum;            // [Hkv][nch][128]
+  int *err;
+};
+
+template <bool I8>
+struct ScoreCfg {
+  static constexpr int kStages = I8 ? 4 : 3;
+  static constexpr int kTileBytes = I8 ? 16384 : 32768;  // 128 rows x 128 elements
+  static constexpr int kThreads = 640;
+  static constexpr int kSmem = 4 * kTileBytes + kStages * kTileBytes + 1024;
+};
+
+template <bool I8>
+__global__ void __launch_bounds__(640, 1)
+    k_score_last(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 ScoreParams P) {
+  using C = ScoreCfg<I8>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_q, bar_kfull[C::kStages], bar_kempty[C::kStages], bar_sfull[4],
+      bar_sfree[4];
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kvh = blockIdx.z;
+  const int tg0 = blockIdx.y * 4;
+  const int T = min(4, P.tiles_per_group - tg0);
+  const int ch0 = blockIdx.x * P.chunks_per_cta;
+  const int ch1 = min(P.nch, ch0 + P.chunks_per_cta);
+  const int U = ch1 - ch0;
+  const bool do_ksum = (blockIdx.y == 0);
+  const int n_ksum_warps = do_ksum ? (I8 ? 1 : 2) : 0;
+  const int tiles_per_head = P.b / 128;
+
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const uint32_t q_smem = base;                                // 4 tiles
+  const uint32_t k_smem = base + 4 * C::kTileBytes;            // ring
+  uint8_t *const k_gen = smem_raw + (k_smem - smem_u32(smem_raw));
+
+  if (threadIdx.x == 0) {
+    abort_sh = 0;
+    mbar_init(smem_u32(&bar_q), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(smem_u32(&bar_kfull[s]), 1);
+      mbar_init(smem_u32(&bar_kempty[s]), 1 + n_ksum_warps);
+    }
+    for (int t = 0; t < 4; ++t) {
+      mbar_init(smem_u32(&bar_sfull[t]), 1);
+      mbar_init(smem_u32(&bar_sfree[t]), 4);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 17) {
+    tmem_alloc(smem_u32(&tmem_base_sh), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int *abort_flag = &abort_sh;
+
+  if (U > 0) {
+    if (warp == 16) {
+      // ------------------------------------------------------------ producer
+      if (lane == 0) {
+        tma_prefetch_map(&tm_q);
+        tma_prefetch_map(&tm_k);
+        mbar_expect_tx(smem_u32(&bar_q), T * C::kTileBytes);
+        for (int t = 0; t < T; ++t) {
+          const int tile = tg0 + t;
+          const int hh = kvh * P.g + tile / tiles_per_head;
+          const int row = hh * P.S + (P.n - 1) * P.b + (tile % tiles_per_head) * 128;
+          const uint32_t dst = q_smem + t * C::kTileBytes;
+          if (I8) {
+            tma_load_2d(dst, &tm_q, 0, row, smem_u32(&bar_q));
+          } else {
+            tma_load_2d(dst, &tm_q, 0, row, smem_u32(&bar_q));
+            tma_load_2d(dst + 16384, &tm_q, 64, row, smem_u32(&bar_q));
+          }
+        }
+        for (int u = 0; u < U; ++u) {
+          const int st = u % C::kStages;
+          if (u >= C::kStages &&
+              !mbar_wait(smem_u32(&bar_kempty[st]), ((u / C::kStages) - 1) & 1, abort_flag, P.err))
+            break;
+          const uint32_t dst = k_smem + st * C::kTileBytes;
+          const int row = kvh * P.S + (ch0 + u) * 128;
+          mbar_expect_tx(smem_u32(&bar_kfull[st]), C::kTileBytes);
+          tma_load_2d(dst, &tm_k, 0, row, smem_u32(&bar_kfull[st]));
+          if (!I8) tma_load_2d(dst + 16384, &tm_k, 64, row, smem_u32(&bar_kfull[st]));
+        }
+      }
+    } else if (warp == 17) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc = I8 ? idesc_i8(128, 128) : idesc_bf16(128, 128, 0);
+        bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, P.err);
+        for (int u = 0; ok && u < U; ++u) {
+          const int st = u % C::kStages;
+          if (!mbar_wait(smem_u32(&bar_kfull[st]), (u / C::kStages) & 1, abort_flag, P.err)) break;
+          const uint32_t kb = k_smem + st * C::kTileBytes;
+          for (int t = 0; t < T && ok; ++t) {
+            if (u > 0 && !mbar_wait(smem_u32(&bar_sfree[t]), (u - 1) & 1, abort_flag, P.err)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t qb = q_smem + t * C::kTileBytes;
+            const uint32_t d_tmem = tmem + t * 128;
+            if (I8) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_i8_ss(d_tmem, umma_desc_sw128(qb + kk * 32, 16, 1024),
+                          umma_desc_sw128(kb + kk * 32, 16, 1024), idesc, kk > 0);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16_ss(d_tmem, umma_desc_sw128(qb + off, 16, 1024),
+                            umma_desc_sw128(kb + off, 16, 1024), idesc, kk > 0);
+              }
+            }
+            tc_commit(smem_u32(&bar_sfull[t]));
+          }
+          if (!ok) break;
+          tc_commit(smem_u32(&bar_kempty[st]));
+        }
+      }
+    } else if (warp >= 18) {
+      // ------------------------------------------------------------ K column sums
+      const int kw = warp - 18;
+      if (kw < n_ksum_warps) {
+        for (int u = 0; u < U; ++u) {
+          const int st = u % C::kStages;
+          if (!mbar_wait(smem_u32(&bar_kfull[st]), (u / C::kStages) & 1, abort_flag, P.err)) break;
+          const uint8_t *tile = k_gen + st * C::kTileBytes;
+          float* out = P.ksum + ((size_t)kvh * P.nch + (ch0 + u)) * 128;
+          if (I8) {
+            // one 128-byte row per key; lane owns bytes 4*lane .. 4*lane+3
+            int acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;
+            for (int r = 0; r < 128; ++r) {
+              const int phys = (((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) << 2);
+              const uint32_t w = *reinterpret_cast<const uint32_t *>(tile + r * 128 + phys);
+              acc0 += (int)(int8_t)(w & 0xff);
+              acc1 += (int)(int8_t)((w >> 8) & 0xff);
+              acc2 += (int)(int8_t)((w >> 16) & 0xff);
+              acc3 += (int)(int8_t)(w >> 24);
+            }
+            out[4 * lane + 0] = (float)acc0;
+            out[4 * lane + 1] = (float)acc1;
+            out[4 * lane + 2] = (float)acc2;
+            out[4 * lane + 3] = (float)acc3;
+          } else {
+            // warp kw reads the 64-column half kw; lane owns columns 2*lane, 2*lane+1
+            const uint8_t *half = tile + kw * 16384;
+            float a0 = 0.f, a1 = 0.f;
+            for (int r = 0; r < 128; ++r) {
+              const int phys = (((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) << 2);
+              const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(half + r * 128 + phys);
+              const float2 f = __bfloat1622float2(v);
+              a0 += f.x;
+              a1 += f.y;
+            }
+            out[kw * 64 + 2 * lane] = a0;
+            out[kw * 64 + 2 * lane + 1] = a1;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bar_kempty[st]));
+        }
+      }
+    } else {
+      // ------------------------------------------------------------ statistics
+      const int t = warp >> 2;
+      if (t < T) {
+        const int tile = tg0 + t;
+        const int hh = kvh * P.g + tile / tiles_per_head;
+        const int rloc = (warp & 3) * 32 + lane;                 // TMEM lane
+        const int i = (tile % tiles_per_head) * 128 + rloc;      // row of the last block
+        float scale2 = P.scale2;
+        if (I8) scale2 *= P.q_scale[hh] * P.k_scale[kvh];
+        const uint32_t taddr = tmem + t * 128 + (((warp & 3) * 32) << 16);
+        for (int u = 0; u < U; ++u) {
+          if (!mbar_wait(smem_u32(&bar_sfull[t]), u & 1, abort_flag, P.err)) break;
+          tc_fence_after();
+          const int ch = ch0 + u;
+          const int tb = (ch * 128) % P.b;                 // chunk offset inside its block
+          const bool last_block = (ch * 128) / P.b == P.n - 1;
+          // pass 1: row max over the causal columns t <= i of the last block
+          float mx = -INFINITY;
+#pragma unroll 1
+          for (int qq = 0; qq < 4; ++qq) {
+            uint32_t r[32];
+            tmem_ld32(taddr + qq * 32, r);
+            tmem_ld_wait(r);
+            const int t0 = tb + qq * 32;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+              const bool valid = !last_block || (t0 + e <= i);
+              mx = valid ? fmaxf(mx, s) : mx;
+            }
+          }
+          float lo = 0.f, hi = 0.f;
+          const float m2 = mx * scale2;
+          if (mx != -INFINITY) {
+#pragma unroll 1
+            for (int qq = 0; qq < 4; ++qq) {
+              uint32_t r[32];
+              tmem_ld32(taddr + qq * 32, r);
+              tmem_ld_wait(r);
+              const int dlt = i - (tb + qq * 32);   // columns e <= dlt are on the lo side
+              if (dlt >= 31) {
+                float acc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+                  acc += ex2(fmaf(s, scale2, -m2));
+                }
+                lo += acc;
+              } else if (dlt < 0) {
+                if (!last_block) {
+                  float acc = 0.f;
+#pragma unroll
+                  for (int e = 0; e < 32; ++e) {
+                    const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+                    acc += ex2(fmaf(s, scale2, -m2));
+                  }
+                  hi += acc;
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                  const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+                  const float p = ex2(fmaf(s, scale2, -m2));
+                  if (e <= dlt) lo += p;
+                  else if (!last_block) hi += p;
+                }
+              }
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&bar_sfree[t]));
+          const size_t o = ((size_t)hh * P.nch + ch) * P.b + i;
+          P.pm[o] = m2;
+          P.plo[o] = lo;
+          P.phi[o] = hi;
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 17) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k_row_stats: grid (Hq, R2), block b threads.  Row i's running max M and
+// sum L = sum_chunks (lo + hi) 2^(m - M) over the CTA's chunk range.
+// ---------------------------------------------------------------------------
+__global__ void k_row_stats(const float *__restrict__ pm, const float *__restrict__ plo,
+                            const float *__restrict__ phi, int nch, int b, int chunks_per_part,
+                            float *__restrict__ partM, float *__restrict__ partL) {
+  const int h = blockIdx.x, part = blockIdx.y, R2 = gridDim.y, i = threadIdx.x;
+  const int c0 = part * chunks_per_part, c1 = min(nch, c0 + chunks_per_part);
+  float M = -INFINITY, L = 0.f;
+  for (int ch = c0; ch < c1; ++ch) {
+    const size_t o = ((size_t)h * nch + ch) * b + i;
+    const float m = pm[o];
+    if (m == -INFINITY) continue;
+    const float s = plo[o] + phi[o];
+    if (m > M) {
+      L = L * ex2(M - m) + s;
+      M = m;
+    } else {
+      L += s * ex2(m - M);
+    }
+  }
+  partM[((size_t)h * R2 + part) * b + i] = M;
+  partL[((size_t)h * R2 + part) * b + i] = L;
+}
+
+// ---------------------------------------------------------------------------
+// k_block_mass: grid (Hq, R2), block b threads.  Combines the R2 partial row
+// statistics, then for every chunk of the CTA's range sums over rows
+//   LOc[ch] = sum_i lo_i 2^(m_i - M_i) / L_i,  HIc[ch] likewise,
+// in a fixed order (per-warp shuffle tree, then warps in index order).
+// ---------------------------------------------------------------------------
+__global__ void k_block_mass(const float *__restrict__ pm, const float *__restrict__ plo,
+                             const float *__restrict__ phi, const float *__restrict__ partM,
+                             const float *__restrict__ partL, int nch, int b, int chunks_per_part,
+                             float *__restrict__ LOc, float *__restrict__ HIc) {
+  extern __shared__ float red[];  // [nwarps][chunks_per_part][2]
+  const int h = blockIdx.x, part = blockIdx.y, R2 = gridDim.y, i = threadIdx.x;
+  const int warp = i >> 5, lane = i & 31, nw = blockDim.x >> 5;
+  float M = -INFINITY;
+  for (int r = 0; r < R2; ++r) M = fmaxf(M, partM[((size_t)h * R2 + r) * b + i]);
+  float L = 0.f;
+  for (int r = 0; r < R2; ++r) {
+    const float m = partM[((size_t)h * R2 + r) * b + i];
+    if (m != -INFINITY) L += partL[((size_t)h * R2 + r) * b + i] * ex2(m - M);
+  }
+  const float invL = 1.f / L;
+  const int c0 = part * chunks_per_part, c1 = min(nch, c0 + chunks_per_part);
+  for (int ch = c0; ch < c1; ++ch) {
+    const size_t o = ((size_t)h * nch + ch) * b + i;
+    const float m = pm[o];
+    const float w = (m == -INFINITY) ? 0.f : ex2(m - M) * invL;
+    float a = plo[o] * w, c = phi[o] * w;
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, s);
+      c += __shfl_xor_sync(0xffffffffu, c, s);
+    }
+    if (lane == 0) {
+      red[(warp * chunks_per_part + (ch - c0)) * 2 + 0] = a;
+      red[(warp * chunks_per_part + (ch - c0)) * 2 + 1] = c;
+    }
+  }
+  __syncthreads();
+  for (int ch = c0 + i; ch < c1; ch += blockDim.x) {
+    float a = 0.f, c = 0.f;
+    for (int w = 0; w < nw; ++w) {
+      a += red[(w * chunks_per_part + (ch - c0)) * 2 + 0];
+      c += red[(w * chunks_per_part + (ch - c0)) * 2 + 1];
+    }
+    LOc[(size_t)h * nch + ch] = a;
+    HIc[(size_t)h * nch + ch] = c;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k_kbar: grid (n, Hkv), block 128: kbar[kvh][c][t] = (1/b) sum of K rows of block c.
+// ---------------------------------------------------------------------------
+__global__ void k_kbar(const float *__restrict__ ksum, int nch, int b, int n, float *__restrict__ kbar) {
+  const int c = blockIdx.x, kvh = blockIdx.y, t = threadIdx.x;
+  const int per = b / 128;
+  float s = 0.f;
+  for (int k = 0; k < per; ++k) s += ksum[((size_t)kvh * nch + c * per + k) * 128 + t];
+  kbar[((size_t)kvh * n + c) * 128 + t] = s / (float)b;
+}
+
+// ---------------------------------------------------------------------------
+// k_pattern: grid (Hq), block 1024.  vhat[c] = (LO[c] + HI[c]) / b,
+// shat[o] = (LO[n-1-o] + HI[n-2-o]) / b, P_est = softmax_c(qbar_last . kbar_c
+// / sqrt(d)), JSD(vhat, P_est) (natural log), pattern = QA iff JSD < tau.
+// ---------------------------------------------------------------------------
+template <bool I8>
+__global__ void __launch_bounds__(1024)
+    k_pattern(const void *__restrict__ q, const float *__restrict__ q_scale,
+              const float *__restrict__ LOc, const float *__restrict__ HIc,
+              const float *__restrict__ kbar, int S, int g, int b, int n, int nch, float inv_sqrt_d,
+              float tau, float *__restrict__ vhat, float *__restrict__ shat,
+              float *__restrict__ pest, float *__restrict__ jsd, int *__restrict__ pattern) {
+  __shared__ float qb[128];
+  __shared__ float part[1024 / 32];
+  __shared__ float lo_s[1024], hi_s[1024];
+  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int kvh = h / g, per = b / 128;
+  // block masses
+  for (int c = tid; c < n; c += blockDim.x) {
+    float a = 0.f, e = 0.f;
+    for (int k = 0; k < per; ++k) {
+      a += LOc[(size_t)h * nch + c * per + k];
+      e += HIc[(size_t)h * nch + c * per + k];
+    }
+    lo_s[c] = a / (float)b;
+    hi_s[c] = e / (float)b;
+  }
+  // mean of the last block's query rows
+  if (tid < 128) {
+    const size_t base = ((size_t)h * S + (size_t)(n - 1) * b) * 128 + tid;
+    if (I8) {
+      const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
+      int acc = 0;
+      for (int r = 0; r < b; ++r) acc += q8[base + (size_t)r * 128];
+      qb[tid] = (float)acc * q_scale[h] / (float)b;
+    } else {
+      const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(q);
+      float acc = 0.f;
+      for (int r = 0; r < b; ++r) acc += __bfloat162float(qh[base + (size_t)r * 128]);
+      qb[tid] = acc / (float)b;
+    }
+  }
+  __syncthreads();
+  for (int c = tid; c < n; c += blockDim.x) {
+    vhat[(size_t)h * n + c] = lo_s[c] + hi_s[c];
+    const int o = c;
+    shat[(size_t)h * n + o] = lo_s[n - 1 - o] + (o <= n - 2 ? hi_s[n - 2 - o] : 0.f);
+  }
+  // logits of P_est, one warp per block c
+  float *z = lo_s;  // reuse after vhat/shat are written
+  __syncthreads();
+  for (int c = warp; c < n; c += blockDim.x / 32) {
+    const float *kr = kbar + ((size_t)kvh * n + c) * 128;
+    float a = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) a = fmaf(qb[lane + 32 * t], kr[lane + 32 * t], a);
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) a += __shfl_xor_sync(0xffffffffu, a, s);
+    if (lane == 0) z[c] = a * inv_sqrt_d;
+  }
+  __syncthreads();
+  float mx = -INFINITY;
+  for (int c = tid; c < n; c += blockDim.x) mx = fmaxf(mx, z[c]);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+  if (lane == 0) part[warp] = mx;
+  __syncthreads();
+  mx = part[0];
+  for (int w = 1; w < (int)(blockDim.x / 32); ++w) mx = fmaxf(mx, part[w]);
+  __syncthreads();
+  float sum = 0.f;
+  for (int c = tid; c < n; c += blockDim.x) {
+    const float e = expf(z[c] - mx);
+    hi_s[c] = e;
+    sum += e;
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, s);
+  if (lane == 0) part[warp] = sum;
+  __syncthreads();
+  sum = 0.f;
+  for (int w = 0; w < (int)(blockDim.x / 32); ++w) sum += part[w];
+  __syncthreads();
+  float js = 0.f;
+  for (int c = tid; c < n; c += blockDim.x) {
+    const float pe = hi_s[c] / sum;
+    pest[(size_t)h * n + c] = pe;
+    const float pv = vhat[(size_t)h * n + c];
+    const float m = 0.5f * (pv + pe);
+    if (pv > 0.f) js += 0.5f * pv * logf(pv / m);
+    if (pe > 0.f) js += 0.5f * pe * logf(pe / m);
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) js += __shfl_xor_sync(0xffffffffu, js, s);
+  if (lane == 0) part[warp] = js;
+  __syncthreads();
+  if (tid == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < (int)(blockDim.x / 32); ++w) tot += part[w];
+    jsd[h] = tot;
+    pattern[h] = (tot < tau) ? 1 : 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k_qbar: grid (n, Hq), block 256: qbar[h][r][t] = (1/b) sum of Q rows of
+// block r, only for heads whose pattern is query-aware (others exit).
+// ---------------------------------------------------------------------------
+template <bool I8>
+__global__ void __launch_bounds__(256)
+    k_qbar(const void *__restrict__ q, const float *__restrict__ q_scale,
+           const int *__restrict__ pattern, int S, int b, int n, float *__restrict__ qbar) {
+  const int r = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  if (pattern[h] != 1) return;
+  __shared__ float red[16][128];
+  const size_t row0 = (size_t)h * S + (size_t)r * b;
+  if (I8) {
+    // 8 threads per 128-byte row, 32 rows per pass; thread owns 16 columns
+    const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
+    const int c16 = tid & 7, rr = tid >> 3;
+    int acc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = 0;
+    for (int p = rr; p < b; p += 32) {
+      const int4 v = *reinterpret_cast<const int4 *>(q8 + (row0 + p) * 128 + c16 * 16);
+      const int w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[e] += (int)(int8_t)((w[e >> 2] >> (8 * (e & 3))) & 0xff);
+    }
+    // reduce over rr (32 groups) via shuffles within the 4 groups of a warp then smem
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      int a = acc[e];
+      a += __shfl_xor_sync(0xffffffffu, a, 8);
+      a += __shfl_xor_sync(0xffffffffu, a, 16);
+      acc[e] = a;
+    }
+    const int warp = tid >> 5, lane = tid & 31;
+    if (lane < 8) {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) red[warp][lane * 16 + e] = (float)acc[e];
+    }
+    __syncthreads();
+    if (tid < 128) {
+      float s = 0.f;
+      for (int w = 0; w < 8; ++w) s += red[w][tid];
+      qbar[((size_t)h * n + r) * 128 + tid] = s * q_scale[h] / (float)b;
+    }
+  } else {
+    // 16 threads per 256-byte row, 16 rows per pass; thread owns 8 columns
+    const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(q);
+    const int c8 = tid & 15, rr = tid >> 4;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+    for (int p = rr; p < b; p += 16) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(qh + (row0 + p) * 128 + c8 * 8);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    const int warp = tid >> 5, lane = tid & 31;
+    if (lane < 16) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
+    }
+    __syncthreads();
+    if (tid < 128) {
+      float s = 0.f;
+      for (int w = 0; w < 8; ++w) s += red[w][tid];
+      qbar[((size_t)h * n + r) * 128 + tid] = s / (float)b;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k_select: grid (ceil(n / 16), Hq), block 256 (8 warps, 2 query blocks per
+// warp).  Scores of query block r over c <= r:
+//   VS: w_c = vhat[c] + shat[r - c];   QA: w_c = exp(qbar_r . kbar_c / sqrt(d) - max)
+// normalised to sum 1.  The diagonal is kept; the others are kept in order
+// of descending score (ties: lower index) while the kept sum is below gamma.
+// The cut is found by bisection on the fp32 bit pattern of the scores
+// (monotone for positive floats): T = largest t with
+// sum_{c < r, bits(w_c) >= t} w_c >= gamma - w_r; everything above T is kept,
+// then ties at T by ascending index until the sum reaches the target.
+// Output: counts[h*n + r], ascending list at cols[h*n(n+1)/2 + r(r+1)/2].
+// ---------------------------------------------------------------------------
+constexpr int kSelRows = 16;
+constexpr int kSelMaxN = 1024;
+
+__global__ void __launch_bounds__(256)
+    k_select(const int *__restrict__ pattern, const float *__restrict__ vhat,
+             const float *__restrict__ shat, const float *__restrict__ qbar,
+             const float *__restrict__ kbar, int g, int n, float inv_sqrt_d, float gamma,
+             int *__restrict__ counts, int *__restrict__ cols) {
+  extern __shared__ float sh[];
+  float *wbuf = sh;                              // [kSelRows][n]
+  float *qs = wbuf + kSelRows * n;               // [kSelRows][128]
+  float *ks = qs + kSelRows * 128;               // [32][129]
+  const int h = blockIdx.y, r0 = blockIdx.x * kSelRows;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rows = min(kSelRows, n - r0);
+  const int pat = pattern[h];
+  const int kvh = h / g;
+  const float *vh = vhat + (size_t)h * n;
+  const float *shh = shat + (size_t)h * n;
+
+  if (pat == 1) {
+    // logits z[rr][c] = qbar_{r0+rr} . kbar_c / sqrt(d) for c <= r0+rows-1
+    for (int e = tid; e < rows * 128; e += blockDim.x)
+      qs[e] = qbar[((size_t)h * n + r0) * 128 + e];
+    const int cmax = r0 + rows;  // exclusive
+    for (int c0 = 0; c0 < cmax; c0 += 32) {
+      __syncthreads();
+      for (int e = tid; e < 32 * 128; e += blockDim.x) {
+        const int cc = e >> 7, t = e & 127;
+        ks[cc * 129 + t] = (c0 + cc < cmax) ? kbar[((size_t)kvh * n + c0 + cc) * 128 + t] : 0.f;
+      }
+      __syncthreads();
+      // thread -> (rr = tid / 16, two columns cc = 2 * (tid % 16) + {0, 1})
+      const int rr = tid >> 4, cc = (tid & 15) * 2;
+      if (rr < rows) {
+        float a0 = 0.f, a1 = 0.f;
+        const float *qr = qs + rr * 128;
+#pragma unroll 8
+        for (int t = 0; t < 128; ++t) {
+          const float qv = qr[t];
+          a0 = fmaf(qv, ks[cc * 129 + t], a0);
+          a1 = fmaf(qv, ks[(cc + 1) * 129 + t], a1);
+        }
+        if (c0 + cc < cmax) wbuf[rr * n + c0 + cc] = a0 * inv_sqrt_d;
+        if (c0 + cc + 1 < cmax) wbuf[rr * n + c0 + cc + 1] = a1 * inv_sqrt_d;
+      }
+    }
+    __syncthreads();
+  }
+
+  for (int rr = warp; rr < rows; rr += 8) {
+    const int r = r0 + rr;
+    float *w = wbuf + rr * n;
+    // raw scores
+    if (pat == 1) {
+      float mx = -INFINITY;
+      for (int c = lane; c <= r; c += 32) mx = fmaxf(mx, w[c]);
+#pragma unroll
+      for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+      for (int c = lane; c <= r; c += 32) w[c] = expf(w[c] - mx);
+    } else {
+      for (int c = lane; c <= r; c += 32) w[c] = vh[c] + shh[r - c];
+    }
+    float z = 0.f;
+    for (int c = lane; c <= r; c += 32) z += w[c];
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) z += __shfl_xor_sync(0xffffffffu, z, s);
+    for (int c = lane; c <= r; c += 32) w[c] = w[c] / z;
+    __syncwarp();
+    const float wr = w[r];
+    const float need = gamma - wr;
+    // selection mode: 0 = all, 1 = diagonal only, 2 = cut at threshold T
+    int mode;
+    uint32_t T = 0;
+    float s_gt = 0.f;
+    if (gamma >= 1.f) {
+      mode = 0;
+    } else if (need <= 0.f) {
+      mode = 1;
+    } else {
+      float tot = 0.f;
+      for (int c = lane; c < r; c += 32) tot += w[c];
+#pragma unroll
+      for (int s = 16; s > 0; s >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, s);
+      if (tot < need) {
+        mode = 0;
+      } else {
+        mode = 2;
+        uint32_t lo = 0u, hi = 0x7F800000u;  // f(lo) >= need > f(hi) = 0
+        while (hi - lo > 1u) {
+          const uint32_t mid = lo + ((hi - lo) >> 1);
+          float f = 0.f;
+          for (int c = lane; c < r; c += 32) f += (__float_as_uint(w[c]) >= mid) ? w[c] : 0.f;
+#pragma unroll
+          for (int s = 16; s > 0; s >>= 1) f += __shfl_xor_sync(0xffffffffu, f, s);
+          if (f >= need) lo = mid; else hi = mid;
+        }
+        T = lo;
+        for (int c = lane; c < r; c += 32) s_gt += (__float_as_uint(w[c]) > T) ? w[c] : 0.f;
+#pragma unroll
+        for (int s = 16; s > 0; s >>= 1) s_gt += __shfl_xor_sync(0xffffffffu, s_gt, s);
+      }
+    }
+    // emit ascending, ties at T in index order until the target is reached
+    int* out = cols + (size_t)h * ((size_t)n * (n + 1) / 2) + (size_t)r * (r + 1) / 2;
+    int written = 0;
+    float tie_acc = s_gt;
+    const float tval = __uint_as_float(T);
+    bool ties_done = false;
+    for (int c0 = 0; c0 <= r; c0 += 32) {
+      const int c = c0 + lane;
+      bool keep = false;
+      bool is_tie = false;
+      if (c <= r) {
+        if (mode == 0 || c == r) keep = true;
+        else if (mode == 2) {
+          const uint32_t bits = __float_as_uint(w[c]);
+          keep = bits > T;
+          is_tie = (bits == T);
+        }
+      }
+      if (mode == 2) {
+        uint32_t tmask = __ballot_sync(0xffffffffu, is_tie);
+        uint32_t take = 0u;
+        while (tmask && !ties_done) {
+          if (tie_acc >= need) { ties_done = true; break; }
+          const int bpos = __ffs(tmask) - 1;
+          take |= 1u << bpos;
+          tie_acc += tval;
+          tmask &= tmask - 1u;
+        }
+        if (take & (1u << lane)) keep = true;
+      }
+      const uint32_t km = __ballot_sync(0xffffffffu, keep);
+      if (keep) out[written + __popc(km & ((1u << lane) - 1u))] = c;
+      written += __popc(km);
+    }
+    if (lane == 0) counts[(size_t)h * n + r] = written;
+  }
+}
+
+}  // namespace fpk

@@ -1,0 +1,175 @@
+"""Python binding of the C ABI in include/fp_sparse.h (ctypes).
+
+Argument marshalling only: torch tensors are passed as device pointers and
+the current CUDA stream as a handle; every step of the computation runs in
+the library's CUDA kernels.  Importing fails loudly when the library has not
+been built -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "_lib", "libfpsparse.so")
+
+FP_OK, FP_ERR_ARG, FP_ERR_CUDA, FP_ERR_TIMEOUT, FP_ERR_STATE = 0, 1, 2, 3, 4
+FP_QK_BF16, FP_QK_INT8 = 0, 1
+FP_PATTERN_VS, FP_PATTERN_QA = 0, 1
+
+SYMBOLS = ("fp_index_create", "fp_index_free", "fp_build_index", "fp_sparse_attn", "fp_index_info",
+           "fp_index_nnz", "fp_index_export", "fp_get_device_error", "fp_debug_wait_timeout",
+           "fp_debug_qk_tile_i8", "fp_strerror")
+
+
+class FpError(RuntimeError):
+    def __init__(self, code, where):
+        super().__init__(f"{where}: {fp_strerror(code)} (code {code})")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"CUDA library not built: {_LIB_PATH} is missing "
+                          "(run python -m dynamic_block_sparse_last_b200.build)")
+    L = ctypes.CDLL(_LIB_PATH)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    L.fp_index_create.argtypes = [i, i, i, i, i, ctypes.POINTER(vp)]
+    L.fp_index_free.argtypes = [vp]
+    L.fp_index_free.restype = None
+    L.fp_build_index.argtypes = [vp, vp, i, i, i, i, i, f, f, i, vp, vp, vp, vp]
+    L.fp_sparse_attn.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+    L.fp_index_info.argtypes = [vp] + [ctypes.POINTER(i)] * 6
+    L.fp_index_nnz.argtypes = [vp, ctypes.POINTER(ctypes.c_int64), vp]
+    L.fp_index_export.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.fp_get_device_error.argtypes = [vp]
+    L.fp_debug_wait_timeout.argtypes = [i, vp]
+    L.fp_debug_qk_tile_i8.argtypes = [vp, vp, i, i, i, i, i, i, i, vp, vp]
+    L.fp_strerror.argtypes = [i]
+    L.fp_strerror.restype = ctypes.c_char_p
+    for s in SYMBOLS:
+        if s != "fp_index_free" and s != "fp_strerror":
+            getattr(L, s).restype = i
+    return L
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def library_path():
+    return _LIB_PATH
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(rc, where):
+    if rc != FP_OK:
+        raise FpError(rc, where)
+
+
+def fp_strerror(code: int) -> str:
+    return _lib.fp_strerror(int(code)).decode()
+
+
+class Index:
+    """Owns one fp_index handle (device workspace for one layer shape)."""
+
+    def __init__(self, handle, S, Hq, Hkv, d, b):
+        self.handle = handle
+        self.S, self.Hq, self.Hkv, self.d, self.b = S, Hq, Hkv, d, b
+        self.n = S // b
+
+    def free(self):
+        if self.handle:
+            _lib.fp_index_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def fp_index_create(S, Hq, Hkv, d, b) -> Index:
+    h = ctypes.c_void_p()
+    _check(_lib.fp_index_create(S, Hq, Hkv, d, b, ctypes.byref(h)), "fp_index_create")
+    return Index(h.value, S, Hq, Hkv, d, b)
+
+
+def fp_index_free(idx: Index):
+    idx.free()
+
+
+def fp_build_index(q, k, S, Hq, Hkv, d, b, gamma, tau, qk_dtype, q_scale, k_scale, idx: Index, stream=None):
+    _check(_lib.fp_build_index(_ptr(q), _ptr(k), S, Hq, Hkv, d, b, float(gamma), float(tau), int(qk_dtype),
+                               _ptr(q_scale), _ptr(k_scale), idx.handle, _stream(stream)), "fp_build_index")
+
+
+def fp_sparse_attn(q, k, v, q_scale, k_scale, idx: Index, out, stream=None):
+    _check(_lib.fp_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(q_scale), _ptr(k_scale), idx.handle,
+                               _ptr(out), _stream(stream)), "fp_sparse_attn")
+
+
+def fp_index_info(idx: Index):
+    vals = [ctypes.c_int() for _ in range(6)]
+    _check(_lib.fp_index_info(idx.handle, *[ctypes.byref(v) for v in vals]), "fp_index_info")
+    return dict(zip(("S", "Hq", "Hkv", "d", "b", "qk_dtype"), [v.value for v in vals]))
+
+
+def fp_index_nnz(idx: Index, stream=None) -> int:
+    v = ctypes.c_int64()
+    _check(_lib.fp_index_nnz(idx.handle, ctypes.byref(v), _stream(stream)), "fp_index_nnz")
+    return v.value
+
+
+def fp_index_export(idx: Index, stream=None):
+    """Host copies: CSR (row_ptr, col) over rows h*n + r, pattern, jsd, vhat, shat, pest."""
+    import numpy as np
+    nnz = fp_index_nnz(idx, stream)
+    Hn = idx.Hq * idx.n
+    row_ptr = np.zeros(Hn + 1, dtype=np.int32)
+    col = np.zeros(max(nnz, 1), dtype=np.int32)
+    pattern = np.zeros(idx.Hq, dtype=np.uint8)
+    jsd = np.zeros(idx.Hq, dtype=np.float32)
+    vhat = np.zeros(Hn, dtype=np.float32)
+    shat = np.zeros(Hn, dtype=np.float32)
+    pest = np.zeros(Hn, dtype=np.float32)
+    _check(_lib.fp_index_export(idx.handle, row_ptr.ctypes.data, col.ctypes.data, pattern.ctypes.data,
+                                jsd.ctypes.data, vhat.ctypes.data, shat.ctypes.data, pest.ctypes.data,
+                                _stream(stream)), "fp_index_export")
+    return {"row_ptr": row_ptr, "col": col[:nnz], "pattern": pattern, "jsd": jsd,
+            "vhat": vhat.reshape(idx.Hq, idx.n), "shat": shat.reshape(idx.Hq, idx.n),
+            "pest": pest.reshape(idx.Hq, idx.n), "nnz": nnz}
+
+
+def fp_get_device_error(stream=None) -> int:
+    return int(_lib.fp_get_device_error(_stream(stream)))
+
+
+def fp_debug_wait_timeout(timeout_us: int, stream=None):
+    _check(_lib.fp_debug_wait_timeout(int(timeout_us), _stream(stream)), "fp_debug_wait_timeout")
+
+
+def fp_debug_qk_tile_i8(q8, k8, S, Hq, Hkv, d, h, p0, j0, out, stream=None):
+    _check(_lib.fp_debug_qk_tile_i8(_ptr(q8), _ptr(k8), S, Hq, Hkv, d, h, p0, j0, _ptr(out), _stream(stream)),
+           "fp_debug_qk_tile_i8")

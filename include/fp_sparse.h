@@ -1,0 +1,138 @@
+/*
+ * fp_sparse.h -- C ABI of the B200 (sm_100a) dynamic block-sparse prefill
+ * attention library (Flex-Prefill method).
+ *
+ * The operation is defined by two web articles on FAST-Prefill:
+ *   "FPGA24成果：FAST-Prefill稀疏注意力加速器，长上下文LLM推理提速2.5倍"
+ *     section 1.1  causal attention softmax(Q K^T / sqrt(d)) V
+ *     section 1.2  b x b block partition; per-head vertical-slash or
+ *                  query-aware pattern chosen by a Jensen-Shannon divergence
+ *     section 2.1  the last query block scores every key block (softmax,
+ *                  block pooling)
+ *     section 3.1  vertical and slash accumulators; blocks added until the
+ *                  cumulative score reaches gamma
+ *     section 3.3  INT8 multiply with INT32 accumulation
+ *   "FPGA加速动态稀疏注意力技术解析与优化"
+ *     section 1.1  representative last query block, JSD pattern decision with
+ *                  threshold tau (usually 0.1), block-level index generation
+ *
+ * Conventions (all arguments): batch 1, tensors head-major and contiguous,
+ * q[Hq][S][d], k[Hkv][S][d], v[Hkv][S][d], out[Hq][S][d]; query head h reads
+ * KV head h / (Hq/Hkv).  Supported: d = 128, b in {128, 256}, S a multiple of
+ * b with S/b <= 1024 blocks, Hq a multiple of Hkv.  Device pointers must be
+ * 16-byte aligned.  All calls are asynchronous on `stream` (a cudaStream_t,
+ * NULL = legacy default stream) unless stated; the caller keeps every buffer
+ * alive until the stream has passed the call.
+ *
+ * Errors: functions return FP_OK (0) or an FP_ERR_* code; nothing aborts the
+ * process.  Argument errors are detected on the host before any launch.  A
+ * device-side bounded wait that gives up records FP_ERR_TIMEOUT in a sticky
+ * per-device word read by fp_get_device_error().
+ */
+#ifndef FP_SPARSE_H
+#define FP_SPARSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    FP_OK = 0,
+    FP_ERR_ARG = 1,      /* invalid argument (shape, pointer, alignment, range) */
+    FP_ERR_CUDA = 2,     /* a CUDA runtime/driver call failed (launch, copy, alloc) */
+    FP_ERR_TIMEOUT = 3,  /* a device-side bounded wait gave up */
+    FP_ERR_STATE = 4     /* index used before it was built, or built for other shapes */
+};
+
+enum { FP_QK_BF16 = 0, FP_QK_INT8 = 1 };        /* element type of q and k */
+enum { FP_PATTERN_VS = 0, FP_PATTERN_QA = 1 };  /* vertical-slash / query-aware */
+
+/* Opaque, library-owned index: per-(head, query block) KV-block lists plus the
+ * per-head statistics and pattern, resident in device memory. */
+typedef struct fp_index fp_index;
+
+/* Allocates an index and its device workspace for one layer shape on the
+ * current CUDA device.  Sizes: S tokens, Hq query heads, Hkv KV heads, head
+ * dim d, block size b (see the supported set above).  *out receives the
+ * handle (NULL on error).  The workspace holds the worst case (gamma = 1),
+ * Hq*n(n+1)/2 block indices, so building never allocates.
+ * Returns FP_ERR_ARG for unsupported shapes, FP_ERR_CUDA if allocation fails. */
+int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out);
+
+/* Frees an index and its workspace (NULL is ignored).  Synchronises the
+ * device before freeing. */
+void fp_index_free(fp_index *idx);
+
+/* Sparse-index generation (articles above: section 2.1 and 3.1 of the
+ * first; section 1.1 of the second).  For every query head h:
+ *   1. the last query block (rows (n-1)b..S-1) is scored against every key
+ *      j <= p and softmax-normalised per row;
+ *   2. vertical vhat[c] and slash shat[o] statistics pool those probabilities
+ *      over key blocks and over diagonal offset blocks floor((p-j)/b);
+ *   3. P_est = softmax_c(qbar_{n-1} . kbar_c / sqrt(d)) from block means;
+ *      JSD(vhat, P_est) < tau selects query-aware, otherwise vertical-slash;
+ *   4. for every query block r: block scores over c <= r (VS: vhat[c] +
+ *      shat[r-c]; QA: softmax of qbar_r . kbar_c / sqrt(d)), normalised; the
+ *      diagonal block is kept, then blocks by descending score (ties: lower
+ *      index) until the kept sum reaches gamma; gamma >= 1 keeps all.
+ * q, k: device, bf16 (qk_dtype FP_QK_BF16) or int8 (FP_QK_INT8) in the layout
+ * above.  q_scale[Hq], k_scale[Hkv]: device fp32 per-head dequantisation
+ * scales for FP_QK_INT8 (logit = int32 dot * q_scale * k_scale / sqrt(d)),
+ * NULL for bf16.  gamma in (0, 1]; tau >= 0.  S, Hq, Hkv, d, b must equal
+ * the values idx was created with.  Writes only into idx. */
+int fp_build_index(const void *q, const void *k, int S, int Hq, int Hkv, int d, int b,
+                   float gamma, float tau, int qk_dtype, const float *q_scale,
+                   const float *k_scale, fp_index *idx, void *stream);
+
+/* Block-sparse GQA causal attention over exactly the blocks in idx (first
+ * article: section 1.1 and figure 3; section 2.2 on KV reuse across the
+ * heads of a GQA group): out[h][p] = sum over keys j <= p in the listed
+ * blocks of softmax_j(q_p . k_j / sqrt(d)) v_j, fp32 softmax, bf16 output.
+ * q, k: device bf16 or int8 (the qk_dtype idx was built with; scales as in
+ * fp_build_index); v: device bf16; out: device bf16 [Hq][S][d].
+ * Returns FP_ERR_STATE if idx has not been built. */
+int fp_sparse_attn(const void *q, const void *k, const void *v, const float *q_scale,
+                   const float *k_scale, const fp_index *idx, void *out, void *stream);
+
+/* Shape of an index (any pointer may be NULL). */
+int fp_index_info(const fp_index *idx, int *S, int *Hq, int *Hkv, int *d, int *b, int *qk_dtype);
+
+/* Synchronises `stream` and returns the number of selected (head, query
+ * block, key block) triples in *nnz. */
+int fp_index_nnz(const fp_index *idx, int64_t *nnz, void *stream);
+
+/* Synchronises `stream` and copies the index to HOST buffers (any may be
+ * NULL): row_ptr[Hq*n + 1] and col[nnz] as CSR over rows h*n + r with
+ * ascending key blocks; pattern[Hq] (FP_PATTERN_*); jsd[Hq]; vhat[Hq*n];
+ * shat[Hq*n]; pest[Hq*n]. */
+int fp_index_export(const fp_index *idx, int32_t *row_ptr, int32_t *col, uint8_t *pattern,
+                    float *jsd, float *vhat, float *shat, float *pest, void *stream);
+
+/* Synchronises `stream`, returns FP_OK or the sticky device error recorded by
+ * a kernel on the current device (FP_ERR_TIMEOUT), and clears it. */
+int fp_get_device_error(void *stream);
+
+/* Test hook for the bounded-wait path: launches one CTA that waits on a
+ * barrier nothing will complete, giving up after timeout_us microseconds and
+ * recording FP_ERR_TIMEOUT; the context stays usable.  timeout_us in
+ * [1, 10000000]. */
+int fp_debug_wait_timeout(int timeout_us, void *stream);
+
+/* Test hook for the int8 score tiles: computes the exact int32 tile
+ * out[i][t] = q8[h][p0 + i] . k8[h/g][j0 + t] for i, t in [0, 128) with the
+ * same tensor-core path the int8 kernels use, into device out[128][128].
+ * p0, j0 multiples of 128 inside [0, S). */
+int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int Hkv, int d, int h,
+                        int p0, int j0, int32_t *out, void *stream);
+
+/* Static message for an FP_* code. */
+const char *fp_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP_SPARSE_H */

@@ -209,7 +209,7 @@ void orc_row_scores(int pattern, int r, const double *vhat, const double *shat,
     for (int c = 0; c <= r; ++c) w[c] /= z;
 }
 
-static const double *g_sort_w;
+static __thread const double *g_sort_w;  /* per-thread: callers may run heads in parallel threads */
 static int by_score_desc(const void *x, const void *y)
 {
     int a = *(const int *)x, b = *(const int *)y;

@@ -28,7 +28,7 @@ def build(force: bool = False) -> str:
     os.makedirs(os.path.dirname(LIB), exist_ok=True)
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
         tmp = LIB + f".{os.getpid()}.tmp"
-        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-std=c99",
+        subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-std=gnu99",
                                "-shared", "-fPIC", SRC, "-o", tmp, "-lm"])
         os.replace(tmp, LIB)
     return LIB

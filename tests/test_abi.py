@@ -1,0 +1,62 @@
+"""The C ABI library without a GPU: it loads, exports every function that
+include/fp_sparse.h declares, and rejects bad arguments on the host before
+any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def fp():
+    from dynamic_block_sparse_last_b200 import build
+    build.build()
+    from dynamic_block_sparse_last_b200 import fp as mod
+    return mod
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "fp_sparse.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(fp):
+    names = declared_functions()
+    assert "fp_build_index" in names and "fp_sparse_attn" in names
+    lib = ctypes.CDLL(fp.library_path())
+    for name in names:
+        assert hasattr(lib, name), name
+    assert set(names) <= set(fp.SYMBOLS) | set(n for n in names if hasattr(fp, n))
+
+
+def test_strerror(fp):
+    assert fp.fp_strerror(fp.FP_OK) == "ok"
+    assert "timed out" in fp.fp_strerror(fp.FP_ERR_TIMEOUT)
+
+
+@pytest.mark.parametrize("S,Hq,Hkv,d,b", [(1000, 4, 2, 128, 128), (1024, 4, 3, 128, 128), (1024, 4, 2, 64, 128),
+                                           (1024, 4, 2, 128, 64), (0, 4, 2, 128, 128), (262144, 4, 2, 128, 128),
+                                           (1024, 0, 2, 128, 128)])
+def test_create_rejects_unsupported_shapes(fp, S, Hq, Hkv, d, b):
+    h = ctypes.c_void_p()
+    assert fp.lib().fp_index_create(S, Hq, Hkv, d, b, ctypes.byref(h)) == fp.FP_ERR_ARG
+    assert h.value is None
+
+
+def test_calls_reject_null_and_misaligned_pointers(fp):
+    L = fp.lib()
+    assert L.fp_build_index(None, None, 1024, 4, 2, 128, 128, 0.9, 0.1, 0, None, None, None, None) == fp.FP_ERR_ARG
+    assert L.fp_sparse_attn(None, None, None, None, None, None, None, None) == fp.FP_ERR_ARG
+    assert L.fp_index_nnz(None, None, None) == fp.FP_ERR_ARG
+    assert L.fp_index_export(None, None, None, None, None, None, None, None, None) == fp.FP_ERR_ARG
+    assert L.fp_debug_wait_timeout(0, None) == fp.FP_ERR_ARG
+    assert L.fp_debug_qk_tile_i8(8, 16, 1024, 4, 2, 128, 0, 0, 0, 16, None) == fp.FP_ERR_ARG   # q8 misaligned
+    assert L.fp_debug_qk_tile_i8(16, 16, 1024, 4, 2, 128, 0, 64, 0, 16, None) == fp.FP_ERR_ARG  # p0 % 128
+
+
+def test_index_info_rejects_null(fp):
+    assert fp.lib().fp_index_info(None, None, None, None, None, None, None) == fp.FP_ERR_ARG

@@ -1,0 +1,169 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Index sets, per-head statistics and patterns are compared in full; attention
+outputs on every tile for the small layers and on seeded samples of tiles
+(at the launch configuration the benchmark times) for the 32K and 128K
+layers.  Tolerances are listed in tests/parity.py.
+"""
+import math
+import random
+
+import numpy as np
+import pytest
+import torch
+
+from dynamic_block_sparse_last_b200 import synth
+from oracle import oracle as orc
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fp():
+    from dynamic_block_sparse_last_b200 import fp as mod
+    assert torch.cuda.is_available(), "CUDA device required"
+    return mod
+
+
+def run_gpu(fp, x, w):
+    dev = torch.device("cuda:0")
+    q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    if w.int8:
+        qq, kk = x["q8"].to(dev), x["k8"].to(dev)
+        qs, ks = x["q_scale"].to(dev), x["k_scale"].to(dev)
+        dt = fp.FP_QK_INT8
+    else:
+        qq, kk, qs, ks, dt = q, k, None, None, fp.FP_QK_BF16
+    idx = fp.fp_index_create(w.S, w.Hq, w.Hkv, w.d, w.b)
+    fp.fp_build_index(qq, kk, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, dt, qs, ks, idx)
+    out = torch.empty_like(q)
+    fp.fp_sparse_attn(qq, kk, v, qs, ks, idx, out)
+    torch.cuda.synchronize()
+    assert fp.fp_get_device_error() == fp.FP_OK
+    exp = fp.fp_index_export(idx)
+    return exp, out, idx
+
+
+def oracle_problem(x, w):
+    if w.int8:
+        return orc.OracleProblem(x["q"], x["k"], x["v"], w.b, q8=x["q8"], k8=x["k8"],
+                                 q_scale=x["q_scale"], k_scale=x["k_scale"])
+    return orc.OracleProblem(x["q"], x["k"], x["v"], w.b)
+
+
+def check_index(P, exp, w):
+    heads = parity.run_parallel(lambda h: P.build_index_head(h, w.gamma, w.tau), range(w.Hq))
+    stats = parity.compare_index(exp, heads, w.S // w.b, w.gamma, w.tau,
+                                 oracle_forced=lambda h, pat: P.build_index_head(h, w.gamma, w.tau, pat))
+    print(f"[{w.name}] index: {stats}; patterns {exp['pattern'].tolist()}; "
+          f"density {exp['nnz'] / (w.Hq * (w.S // w.b) * (w.S // w.b + 1) / 2):.4f}")
+    return heads, stats
+
+
+def check_tiles(P, exp, out, w, tiles):
+    n = w.S // w.b
+
+    def one(t):
+        h, qc = t
+        r = qc * 128 // w.b
+        rows = parity.gpu_rows(exp, h, n)[r]
+        ref = P.attn_rows(h, qc * 128, qc * 128 + 128, rows)
+        return ref
+
+    refs = parity.run_parallel(one, tiles)
+    worst_max, sum_mean = 0.0, 0.0
+    for (h, qc), ref in zip(tiles, refs):
+        got = out[h, qc * 128: qc * 128 + 128].float().cpu().numpy()
+        mx, mean = parity.compare_tile(got, ref)
+        assert mx <= parity.OUT_MAX_ABS and mean <= parity.OUT_MEAN_ABS, (h, qc, mx, mean)
+        worst_max = max(worst_max, mx)
+        sum_mean += mean
+    print(f"[{w.name}] {len(tiles)} tiles: worst max-abs {worst_max:.3e}, mean of mean-abs "
+          f"{sum_mean / len(tiles):.3e}")
+
+
+SMALL = [
+    synth.WORKLOADS["tiny"],
+    synth.Workload("g3_b256", S=2048, Hq=6, Hkv=2, b=256, seed=3),
+    synth.Workload("g1_gamma08", S=1536, Hq=4, Hkv=4, b=128, gamma=0.8, seed=4),
+    synth.Workload("g4_gamma095", S=4096, Hq=8, Hkv=2, b=128, gamma=0.95, seed=5),
+    synth.Workload("gamma1_b256", S=512, Hq=4, Hkv=1, b=256, gamma=1.0, seed=6),
+    synth.Workload("one_block", S=128, Hq=2, Hkv=1, b=128, seed=7),
+    synth.Workload("one_block_b256", S=256, Hq=2, Hkv=2, b=256, seed=8),
+    synth.Workload("two_blocks_tau0", S=256, Hq=2, Hkv=1, b=128, tau=0.0, seed=12),
+    synth.Workload("int8_small", S=2048, Hq=4, Hkv=2, b=128, int8=True, seed=9),
+    synth.Workload("int8_b256", S=2048, Hq=4, Hkv=1, b=256, gamma=0.95, int8=True, seed=10),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=[w.name for w in SMALL])
+def test_small_layers_full_parity(fp, w):
+    x = synth.make_inputs(w)
+    exp, out, idx = run_gpu(fp, x, w)
+    P = oracle_problem(x, w)
+    check_index(P, exp, w)
+    tiles = [(h, qc) for h in range(w.Hq) for qc in range(w.S // 128)]
+    check_tiles(P, exp, out, w, tiles)
+
+
+def test_gamma_one_matches_dense_sdpa(fp):
+    w = synth.Workload("dense", S=2048, Hq=8, Hkv=2, b=128, gamma=1.0, seed=13)
+    x = synth.make_inputs(w)
+    exp, out, idx = run_gpu(fp, x, w)
+    n = w.S // w.b
+    assert exp["nnz"] == w.Hq * n * (n + 1) // 2
+    q, k, v = (x[t].cuda().float() for t in ("q", "k", "v"))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q[None], k.repeat_interleave(4, 0)[None], v.repeat_interleave(4, 0)[None], is_causal=True)[0]
+    diff = (out.float() - ref).abs()
+    assert float(diff.max()) <= parity.OUT_MAX_ABS and float(diff.mean()) <= parity.OUT_MEAN_ABS
+
+
+def test_int8_score_tiles_bit_exact(fp):
+    w = synth.Workload("i8tiles", S=1024, Hq=4, Hkv=2, b=128, int8=True, seed=14)
+    x = synth.make_inputs(w)
+    P = oracle_problem(x, w)
+    q8, k8 = x["q8"].cuda(), x["k8"].cuda()
+    out = torch.empty(128, 128, dtype=torch.int32, device="cuda")
+    for h, p0, j0 in [(0, 0, 0), (1, 896, 0), (2, 512, 384), (3, 896, 896)]:
+        fp.fp_debug_qk_tile_i8(q8, k8, w.S, w.Hq, w.Hkv, w.d, h, p0, j0, out)
+        torch.cuda.synchronize()
+        ref = P.qk_int_tile(h, p0, j0, 128, 128)
+        assert np.array_equal(out.cpu().numpy(), ref), (h, p0, j0)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(fp):
+    fp.fp_debug_wait_timeout(200000)
+    assert fp.fp_get_device_error() == fp.FP_ERR_TIMEOUT
+    assert fp.fp_get_device_error() == fp.FP_OK
+    w = synth.Workload("after_timeout", S=256, Hq=2, Hkv=1, b=128, seed=15)
+    x = synth.make_inputs(w)
+    exp, out, idx = run_gpu(fp, x, w)
+    assert exp["nnz"] >= w.Hq * (w.S // w.b)
+
+
+def sampled_tiles(w, count, seed):
+    rng = random.Random(seed)
+    nq = w.S // 128
+    tiles = {(h, nq - 1) for h in range(0, w.Hq, max(1, w.Hq // 4))}      # longest rows
+    while len(tiles) < count:
+        tiles.add((rng.randrange(w.Hq), rng.randrange(nq)))
+    return sorted(tiles)
+
+
+@pytest.mark.parametrize("name,ntiles", [("llama3b", 24), ("llama8b", 64), ("llama8b_w8a8", 64)])
+def test_full_size_layers(fp, name, ntiles):
+    w = synth.WORKLOADS[name]
+    x = synth.make_inputs(w)
+    exp, out, idx = run_gpu(fp, x, w)
+    P = oracle_problem(x, w)
+    check_index(P, exp, w)
+    check_tiles(P, exp, out, w, sampled_tiles(w, ntiles, seed=w.seed))
+    if w.int8:
+        q8, k8 = x["q8"].cuda(), x["k8"].cuda()
+        t = torch.empty(128, 128, dtype=torch.int32, device="cuda")
+        for h, p0, j0 in [(0, w.S - 128, 0), (31, w.S - 128, w.S - 128), (17, 65536, 4096)]:
+            fp.fp_debug_qk_tile_i8(q8, k8, w.S, w.Hq, w.Hkv, w.d, h, p0, j0, t)
+            torch.cuda.synchronize()
+            assert np.array_equal(t.cpu().numpy(), P.qk_int_tile(h, p0, j0, 128, 128))
