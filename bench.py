@@ -1,0 +1,364 @@
+"""Benchmark: one sparse-prefill attention layer per step (index build + block-sparse attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama8b] [--impl ours|reference]
+
+Default workload: the Llama-3-8B-shaped layer at 128K context (S=131072, Hq=32,
+Hkv=8, d=128, b=128, gamma=0.9, tau=0.1, bf16), seeded synthetic inputs.  A step
+is fp_build_index + fp_sparse_attn on inputs resident in HBM; value is the
+dense-equivalent throughput 2*Hq*d*S^2 / t (TFLOP/s) summed over ranks, and
+ms_per_step is ms per layer.  Inputs (Q 1 GiB, K and V 256 MiB each) exceed the
+126 MB L2, so no flush is needed between steps.  Under torchrun every rank runs
+an independent replica (the layer does not shard on one node here).
+
+--impl reference times the fp64 CPU oracle on the host cores on bounded samples
+of the same workload (rank 0 only) and prints the same JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_block_sparse_last_b200 import synth  # noqa: E402
+
+METRIC = "sparse-prefill ms/layer & dense-equiv TFLOPS at S=128K; % of HBM/TC roofline"
+UNIT = "dense-equiv TFLOP/s"
+KERNELS_PER_STEP = 8  # k_score_last, k_row_stats, k_block_mass, k_kbar, k_pattern, k_qbar, k_select, k_sparse_attn
+ATTN_SRC = os.path.join(ROOT, "dynamic_block_sparse_last_b200", "csrc", "attn_kernel.cuh")
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def attn_traffic_record():
+    """Per-launch DRAM bytes of the attention kernel from a committed ncu summary,
+    or None when the kernel source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "attn_traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p))
+    sha = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
+    if rec.get("kernel_src_sha256") != sha:
+        return None
+    return rec
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def make_line(args, w, value, ms_per_step, extra):
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int8" if w.int8 else "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "b": w.b,
+                       "gamma": w.gamma, "tau": w.tau, "seed": w.seed, "batch": 1,
+                       "l2": "inputs larger than L2 (no flush)", "parallelism": "replicas"}}
+    line.update(extra)
+    return line
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+def oracle_sample(w, x, P, step, tiles_per_step=1):
+    """One bounded oracle sample: the full index of one head plus attention of
+    `tiles_per_step` 128-row tiles of that head; returns (seconds, extrapolated
+    seconds per layer, description)."""
+    h = step % w.Hq
+    nq = w.S // 128
+    t0 = time.perf_counter()
+    o = P.build_index_head(h, w.gamma, w.tau, want_scores=False)
+    t1 = time.perf_counter()
+    rng = np.random.default_rng(1000 + step)
+    tile_t = []
+    for _ in range(tiles_per_step):
+        qc = int(rng.integers(0, nq))
+        r = qc * 128 // w.b
+        s = time.perf_counter()
+        P.attn_rows(h, qc * 128, qc * 128 + 128, o["rows"][r])
+        tile_t.append(time.perf_counter() - s)
+    t2 = time.perf_counter()
+    per_layer = (t1 - t0) * w.Hq + float(np.mean(tile_t)) * w.Hq * nq
+    desc = (f"oracle index of head {h} ({t1 - t0:.2f} s) x {w.Hq} heads + {tiles_per_step} attention "
+            f"tile(s) of 128 rows ({np.mean(tile_t):.2f} s mean) x {w.Hq * nq} tiles; 1 thread; extrapolated")
+    return t2 - t0, per_layer, desc
+
+
+def oracle_problem(w, x):
+    from oracle import oracle as orc
+    if w.int8:
+        return orc.OracleProblem(x["q"], x["k"], x["v"], w.b, q8=x["q8"], k8=x["k8"],
+                                 q_scale=x["q_scale"], k_scale=x["k_scale"])
+    return orc.OracleProblem(x["q"], x["k"], x["v"], w.b)
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    x = synth.make_inputs(w)
+    P = oracle_problem(w, x)
+    dense = synth.dense_equiv_flops(w.S, w.Hq, w.d)
+    for s in range(args.warmup):
+        oracle_sample(w, x, P, s)
+    per_layer, wall, desc = [], 0.0, ""
+    for s in range(args.steps):
+        t, pl, desc = oracle_sample(w, x, P, args.warmup + s)
+        wall += t
+        per_layer.append(pl)
+    layer_s = float(np.mean(per_layer))
+    value = dense / layer_s / 1e12
+    cpu = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+    line = make_line(args, w, value, layer_s * 1e3,
+                     {"impl": "reference", "cpu_baseline": cpu,
+                      "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                      "reference_note": f"fp64 oracle on host cores, {args.steps} bounded samples "
+                                        f"({wall:.1f} s), ms_per_step = extrapolated ms per layer"})
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- CUDA path
+
+def run_ours(args, w):
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    from dynamic_block_sparse_last_b200 import fp
+
+    x = synth.make_inputs(w)
+    q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    if w.int8:
+        qq, kk = x["q8"].to(dev), x["k8"].to(dev)
+        qs, ks = x["q_scale"].to(dev), x["k_scale"].to(dev)
+        dt = fp.FP_QK_INT8
+    else:
+        qq, kk, qs, ks, dt = q, k, None, None, fp.FP_QK_BF16
+    out = torch.empty_like(q)
+    idx = fp.fp_index_create(w.S, w.Hq, w.Hkv, w.d, w.b)
+    stream = torch.cuda.Stream(device=dev)
+
+    def step():
+        fp.fp_build_index(qq, kk, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, dt, qs, ks, idx, stream)
+        fp.fp_sparse_attn(qq, kk, v, qs, ks, idx, out, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    stream.synchronize()
+    assert fp.fp_get_device_error(stream) == fp.FP_OK
+    exp = fp.fp_index_export(idx, stream)
+    nq = w.S // 128
+    n = w.S // w.b
+    rp = exp["row_ptr"]
+    counts = np.diff(rp).reshape(w.Hq, n)
+    per = w.b // 128
+    chunks = 0
+    for qc in range(nq):
+        r = qc * 128 // w.b
+        chunks += int(((counts[:, r] - 1) * per + (qc % per) + 1).sum())
+    attn_flops = chunks * 4.0 * 128 * 128 * 128
+    density = exp["nnz"] / (w.Hq * n * (n + 1) / 2)
+
+    # timed region: K steps, events around each stage on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    sampler.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t_start.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            fp.fp_build_index(qq, kk, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, dt, qs, ks, idx, stream)
+            ev[s][1].record(stream)
+            fp.fp_sparse_attn(qq, kk, v, qs, ks, idx, out, stream)
+            ev[s][2].record(stream)
+        t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    index_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
+    attn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
+    assert fp.fp_get_device_error(stream) == fp.FP_OK
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    dense = synth.dense_equiv_flops(w.S, w.Hq, w.d)
+    value = world * dense * args.steps / (total_ms / 1e3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    h_q = x["q8"].pin_memory() if w.int8 else x["q"].pin_memory()
+    h_k = x["k8"].pin_memory() if w.int8 else x["k"].pin_memory()
+    h_v = x["v"].pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    d_q, d_k, d_v = torch.empty_like(qq), torch.empty_like(kk), torch.empty_like(v)
+    e2e_steps = max(2, min(5, args.steps))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        for it in range(e2e_steps + 1):
+            if it == 1:
+                e0.record(stream)
+            d_q.copy_(h_q, non_blocking=True)
+            d_k.copy_(h_k, non_blocking=True)
+            d_v.copy_(h_v, non_blocking=True)
+            fp.fp_build_index(d_q, d_k, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, dt, qs, ks, idx, stream)
+            fp.fp_sparse_attn(d_q, d_k, d_v, qs, ks, idx, out, stream)
+            h_out.copy_(out, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = h_q.numel() * h_q.element_size() + h_k.numel() * h_k.element_size() + h_v.numel() * h_v.element_size()
+    d2h = h_out.numel() * h_out.element_size()
+    e2e = {"value": world * dense / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    peaks = load_peaks()
+    peak = peaks["bf16_tflops_sustained"]
+    achieved = attn_flops / (attn_ms / 1e3) / 1e12
+    trec = attn_traffic_record()
+    roof = {"kernel": "k_sparse_attn", "bound": "tensor", "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": (trec["dram_bytes_per_launch"] if trec else None),
+            "peak_source": f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)"
+            if peaks["source"] == "measured" else "fallback 1.4 PFLOP/s sustained",
+            "algorithmic_flops_per_launch": attn_flops,
+            "note": "algorithmic FLOPs = 4*128^3 per computed 128x128 query-key chunk tile"}
+    # index pass against HBM: K once, Q of query-aware heads, the last query block
+    elt = 1 if w.int8 else 2
+    qa_heads = int((exp["pattern"] == 1).sum())
+    idx_bytes = (w.Hkv * w.S * w.d + qa_heads * w.S * w.d + w.Hq * w.b * w.d) * elt
+    idx_gbs = idx_bytes / (index_ms / 1e3) / 1e9
+    extra = {"roofline": roof,
+             "index_pass": {"ms": index_ms, "algorithmic_bytes": idx_bytes, "achieved_gbs": idx_gbs,
+                            "frac_of_hbm": idx_gbs / peaks["hbm_gbs"], "qa_heads": qa_heads},
+             "attn_ms": attn_ms, "density": density, "chunks": chunks,
+             "e2e": e2e, "clocks": clocks, "gpu_launches": KERNELS_PER_STEP * args.steps,
+             "gpu": torch.cuda.get_device_name(dev)}
+    if world == 1 and not args.no_cpu_baseline and rank == 0:
+        P = oracle_problem(w, x)
+        t, per_layer, desc = oracle_sample(w, x, P, 0)
+        extra["cpu_baseline"] = {"value": synth.dense_equiv_flops(w.S, w.Hq, w.d) / per_layer / 1e12,
+                                 "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
+                                 "host_cpus": os.cpu_count()}
+    if rank == 0:
+        print(json.dumps(make_line(args, w, value, ms_per_step, extra)), flush=True)
+    idx.free()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -232,11 +232,14 @@ __global__ void __launch_bounds__(192, 1)
       const bool raise = rmax2 > m_ref + 8.f;
       const float m_new = raise ? rmax2 : m_ref;
       const float alpha = raise ? ex2(m_ref - m_new) : 1.f;
+      // P in bf16 (the P.V operand); the row sum adds the same rounded values
+      // so numerator and denominator use identical weights.
+      uint32_t pk[64];
       float rs = 0.f;
 #pragma unroll
-      for (int t = 0; t < 128; ++t) {
-        s[t] = ex2(fmaf(s[t], scale2, -m_new));
-        rs += s[t];
+      for (int t = 0; t < 128; t += 2) {
+        pk[t >> 1] = pack_bf16x2(ex2(fmaf(s[t], scale2, -m_new)), ex2(fmaf(s[t + 1], scale2, -m_new)));
+        rs += __uint_as_float(pk[t >> 1] << 16) + __uint_as_float(pk[t >> 1] & 0xFFFF0000u);
       }
       l = l * alpha + rs;
       m_ref = m_new;
@@ -261,12 +264,7 @@ __global__ void __launch_bounds__(192, 1)
       // lives in 64-key half t/64, 16-byte chunk ((t%64)/8) ^ (row%8).
 #pragma unroll
       for (int c8 = 0; c8 < 16; ++c8) {
-        const int t = c8 * 8;
-        uint4 v;
-        v.x = pack_bf16x2(s[t + 0], s[t + 1]);
-        v.y = pack_bf16x2(s[t + 2], s[t + 3]);
-        v.z = pack_bf16x2(s[t + 4], s[t + 5]);
-        v.w = pack_bf16x2(s[t + 6], s[t + 7]);
+        const uint4 v = make_uint4(pk[c8 * 4 + 0], pk[c8 * 4 + 1], pk[c8 * 4 + 2], pk[c8 * 4 + 3]);
         const int half = c8 >> 3, chunk = (c8 & 7) ^ (row & 7);
         *reinterpret_cast<uint4 *>(p_gen + half * 16384 + row * 128 + chunk * 16) = v;
       }

@@ -171,7 +171,7 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
                                                             I->nch, I->b, I->chunks_per_part, I->LOc,
                                                             I->HIc);
   if ((rc = launch_status())) return rc;
-  k_kbar<<<dim3(I->n, I->Hkv), 128, 0, st>>>(I->ksum, I->nch, I->b, I->n, I->kbar);
+  k_kbar<<<dim3(I->n, I->Hkv), 128, 0, st>>>(I->ksum, I8 ? k_scale : nullptr, I->nch, I->b, I->n, I->kbar);
   if ((rc = launch_status())) return rc;
   const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
   k_pattern<I8><<<I->Hq, 1024, 0, st>>>(q, q_scale, I->LOc, I->HIc, I->kbar, I->S, I->g, I->b, I->n,

@@ -382,13 +382,16 @@ __global__ void k_block_mass(const float *__restrict__ pm, const float *__restri
 }
 
 // ---------------------------------------------------------------------------
-// k_kbar: grid (n, Hkv), block 128: kbar[kvh][c][t] = (1/b) sum of K rows of block c.
+// k_kbar: grid (n, Hkv), block 128: kbar[kvh][c][t] = (1/b) sum of K rows of
+// block c; for int8 keys the exact integer sum times k_scale[kvh].
 // ---------------------------------------------------------------------------
-__global__ void k_kbar(const float *__restrict__ ksum, int nch, int b, int n, float *__restrict__ kbar) {
+__global__ void k_kbar(const float *__restrict__ ksum, const float *__restrict__ k_scale, int nch, int b,
+                       int n, float *__restrict__ kbar) {
   const int c = blockIdx.x, kvh = blockIdx.y, t = threadIdx.x;
   const int per = b / 128;
   float s = 0.f;
   for (int k = 0; k < per; ++k) s += ksum[((size_t)kvh * nch + c * per + k) * 128 + t];
+  if (k_scale) s *= k_scale[kvh];
   kbar[((size_t)kvh * n + c) * 128 + t] = s / (float)b;
 }
 
