@@ -413,6 +413,119 @@ int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int H
   return launch_status();
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free pattern statistics: the scratch of the statistics kernels
+// lives in this fixed device array instead of an fp_index workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_fp_stats_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+unsigned char *g_scratch_ptr[128] = {nullptr};
+
+// Device address of g_fp_stats_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+unsigned char *stats_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fp_stats_scratch) != cudaSuccess || p == nullptr) return nullptr;
+    g_scratch_ptr[dev] = static_cast<unsigned char *>(p);
+  }
+  return g_scratch_ptr[dev];
+}
+
+size_t round256(size_t x) { return ((x + 255) / 256) * 256; }
+
+template <bool I8>
+int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int d, int b, float tau,
+                       const float *q_scale, const float *k_scale, float *vhat, float *shat, float *pest,
+                       float *jsd, int32_t *pattern, cudaStream_t st) {
+  const int n = S / b, nch = S / 128, g = Hq / Hkv;
+  int R2 = nch < 16 ? nch : 16;
+  const int cpp = (nch + R2 - 1) / R2;
+  R2 = (nch + cpp - 1) / cpp;
+  const size_t e_part = (size_t)Hq * nch * b, e_rs = (size_t)Hq * R2 * b, e_blk = (size_t)Hq * nch;
+  const size_t e_ksum = (size_t)Hkv * nch * 128, e_kbar = (size_t)Hkv * n * 128;
+  const size_t need = 3 * round256(e_part * 4) + 2 * round256(e_rs * 4) + 2 * round256(e_blk * 4) +
+                      round256(e_ksum * 4) + round256(e_kbar * 4);
+  if (need > kNoAllocScratchBytes) return FP_ERR_ARG;
+  unsigned char *base = stats_scratch();
+  if (!base) return FP_ERR_CUDA;
+  int rc = set_smem_attrs<I8>();
+  if (rc) return rc;
+  int *err = device_error_word();
+  if (!err) return FP_ERR_CUDA;
+  char *cur = reinterpret_cast<char *>(base);
+  float *pm = carve<float>(cur, e_part), *plo = carve<float>(cur, e_part), *phi = carve<float>(cur, e_part);
+  float *partM = carve<float>(cur, e_rs), *partL = carve<float>(cur, e_rs);
+  float *LOc = carve<float>(cur, e_blk), *HIc = carve<float>(cur, e_blk);
+  float *ksum = carve<float>(cur, e_ksum), *kbar = carve<float>(cur, e_kbar);
+
+  CUtensorMap tq, tk;
+  if (!make_map(&tq, q, I8, (uint64_t)Hq * S) || !make_map(&tk, k, I8, (uint64_t)Hkv * S)) return FP_ERR_CUDA;
+  const int tiles_per_group = g * (b / 128);
+  const int tgroups = (tiles_per_group + 3) / 4;
+  int R = sm_count() / (tgroups * Hkv);
+  if (R < 1) R = 1;
+  if (R > nch) R = nch;
+  const int cpc = (nch + R - 1) / R;
+  R = (nch + cpc - 1) / cpc;
+  ScoreParams sp;
+  sp.S = S; sp.Hq = Hq; sp.Hkv = Hkv; sp.b = b; sp.n = n; sp.nch = nch; sp.g = g;
+  sp.tiles_per_group = tiles_per_group;
+  sp.chunks_per_cta = cpc;
+  sp.scale2 = kLog2e / sqrtf((float)d);
+  sp.q_scale = q_scale;
+  sp.k_scale = k_scale;
+  sp.pm = pm; sp.plo = plo; sp.phi = phi; sp.ksum = ksum;
+  sp.err = err;
+  k_score_last<I8><<<dim3(R, tgroups, Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
+  if ((rc = launch_status())) return rc;
+  k_row_stats<<<dim3(Hq, R2), b, 0, st>>>(pm, plo, phi, nch, b, cpp, partM, partL);
+  if ((rc = launch_status())) return rc;
+  k_block_mass<<<dim3(Hq, R2), b, (size_t)(b / 32) * cpp * 2 * sizeof(float), st>>>(pm, plo, phi, partM, partL,
+                                                                                    nch, b, cpp, LOc, HIc);
+  if ((rc = launch_status())) return rc;
+  k_kbar<<<dim3(n, Hkv), 128, 0, st>>>(ksum, I8 ? k_scale : nullptr, nch, b, n, kbar);
+  if ((rc = launch_status())) return rc;
+  k_pattern<I8><<<Hq, 1024, 0, st>>>(q, q_scale, LOc, HIc, kbar, S, g, b, n, nch, 1.0f / sqrtf((float)d), tau,
+                                     vhat, shat, pest, jsd, pattern);
+  return launch_status();
+}
+
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int fp_pattern_stats_noalloc(const void *q, const void *k, int S, int Hq, int Hkv, int d, int b, float tau,
+                             int qk_dtype, const float *q_scale, const float *k_scale, float *vhat, float *shat,
+                             float *pest, float *jsd, int32_t *pattern, void *stream) {
+  if (!q || !k || !vhat || !shat || !pest || !jsd || !pattern) return FP_ERR_ARG;
+  if (!shape_ok(S, Hq, Hkv, d, b)) return FP_ERR_ARG;
+  if (!(tau >= 0.f) || std::isnan(tau)) return FP_ERR_ARG;
+  if (qk_dtype != FP_QK_BF16 && qk_dtype != FP_QK_INT8) return FP_ERR_ARG;
+  if (qk_dtype == FP_QK_INT8 && (!q_scale || !k_scale)) return FP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k)) return FP_ERR_ARG;
+  if (!aligned4(vhat) || !aligned4(shat) || !aligned4(pest) || !aligned4(jsd) || !aligned4(pattern))
+    return FP_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return qk_dtype == FP_QK_INT8
+             ? stats_noalloc_impl<true>(q, k, S, Hq, Hkv, d, b, tau, q_scale, k_scale, vhat, shat, pest, jsd,
+                                        pattern, st)
+             : stats_noalloc_impl<false>(q, k, S, Hq, Hkv, d, b, tau, nullptr, nullptr, vhat, shat, pest, jsd,
+                                         pattern, st);
+}
+
 const char *fp_strerror(int code) {
   switch (code) {
     case FP_OK: return "ok";

@@ -20,7 +20,7 @@ FP_PATTERN_VS, FP_PATTERN_QA = 0, 1
 
 SYMBOLS = ("fp_index_create", "fp_index_free", "fp_build_index", "fp_sparse_attn", "fp_index_info",
            "fp_index_nnz", "fp_index_export", "fp_get_device_error", "fp_debug_wait_timeout",
-           "fp_debug_qk_tile_i8", "fp_strerror")
+           "fp_debug_qk_tile_i8", "fp_pattern_stats_noalloc", "fp_strerror")
 
 
 class FpError(RuntimeError):
@@ -46,6 +46,7 @@ def _load():
     L.fp_get_device_error.argtypes = [vp]
     L.fp_debug_wait_timeout.argtypes = [i, vp]
     L.fp_debug_qk_tile_i8.argtypes = [vp, vp, i, i, i, i, i, i, i, vp, vp]
+    L.fp_pattern_stats_noalloc.argtypes = [vp, vp, i, i, i, i, i, f, i, vp, vp, vp, vp, vp, vp, vp, vp]
     L.fp_strerror.argtypes = [i]
     L.fp_strerror.restype = ctypes.c_char_p
     for s in SYMBOLS:
@@ -173,3 +174,12 @@ def fp_debug_wait_timeout(timeout_us: int, stream=None):
 def fp_debug_qk_tile_i8(q8, k8, S, Hq, Hkv, d, h, p0, j0, out, stream=None):
     _check(_lib.fp_debug_qk_tile_i8(_ptr(q8), _ptr(k8), S, Hq, Hkv, d, h, p0, j0, _ptr(out), _stream(stream)),
            "fp_debug_qk_tile_i8")
+
+
+def fp_pattern_stats_noalloc(q, k, S, Hq, Hkv, d, b, tau, qk_dtype, q_scale, k_scale, vhat, shat, pest, jsd,
+                             pattern, stream=None):
+    """Per-head vhat/shat/pest/jsd/pattern into caller-owned device buffers,
+    using the library's fixed scratch array instead of any allocation."""
+    _check(_lib.fp_pattern_stats_noalloc(_ptr(q), _ptr(k), S, Hq, Hkv, d, b, float(tau), int(qk_dtype),
+                                         _ptr(q_scale), _ptr(k_scale), _ptr(vhat), _ptr(shat), _ptr(pest),
+                                         _ptr(jsd), _ptr(pattern), _stream(stream)), "fp_pattern_stats_noalloc")

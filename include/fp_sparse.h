@@ -128,6 +128,36 @@ int fp_debug_wait_timeout(int timeout_us, void *stream);
 int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int Hkv, int d, int h,
                         int p0, int j0, int32_t *out, void *stream);
 
+/* Per-head pattern statistics with no device allocation at all.  The papers
+ * have no counterpart of this call; it exists for callers that must not
+ * allocate device memory -- for example a host framework that owns every
+ * byte of device memory through its own caching allocator or memory budget,
+ * or a latency-critical loop that cannot afford the device-wide
+ * synchronisation cudaMalloc/cudaFree imply.  It computes what
+ * fp_build_index computes up to the pattern decision (steps 1-3 there):
+ * vhat[Hq*n], shat[Hq*n], pest[Hq*n], jsd[Hq] and pattern[Hq]
+ * (FP_PATTERN_*, int32), all caller-owned device buffers.  Inputs as in
+ * fp_build_index (gamma is not needed).
+ *
+ * Scratch: a fixed 32 MiB array inside the library (a file-scope device
+ * array; every GPU that loads the library keeps it until process exit).  A
+ * problem needs at most 12*Hq*S + 128*Hq*b + 8*Hq*(S/128) + 4*Hkv*S +
+ * 512*Hkv*(S/b) bytes of it plus 2 KiB of alignment; e.g. S=32768 with
+ * Hq=32, Hkv=8 fits, and so does S=131072 with Hq=16, Hkv=4.
+ * Larger problems are rejected with FP_ERR_ARG before anything is launched.
+ * The first call on a device looks up the array's device address (set-up,
+ * once per device, with that device current); make that first call before
+ * any stream capture.  All calls share the one array and it keeps the last
+ * call's contents; every scratch word a call reads is written earlier in
+ * the same call, so nothing needs clearing.  Calls whose executions overlap
+ * on the GPU (different streams, or different host threads) race on the
+ * scratch and must be serialised by the caller.  Makes no cudaMalloc,
+ * cudaFree or other allocating call. */
+int fp_pattern_stats_noalloc(const void *q, const void *k, int S, int Hq, int Hkv, int d, int b,
+                             float tau, int qk_dtype, const float *q_scale, const float *k_scale,
+                             float *vhat, float *shat, float *pest, float *jsd, int32_t *pattern,
+                             void *stream);
+
 /* Static message for an FP_* code. */
 const char *fp_strerror(int code);
 
