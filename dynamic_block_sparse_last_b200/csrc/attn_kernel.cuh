@@ -4,30 +4,35 @@
 // article, figure 3 and section 1.1): out_p = sum over listed keys j <= p of
 // softmax_j(q_p . k_j / sqrt(d)) v_j.  Online softmax in fp32, bf16 P.V.
 //
-// CTA = (query head h, 128-row query tile qc).  CTAs are numbered heavy first
-// (descending qc) and, inside one qc, by head, so the g heads of a GQA group
-// run side by side and their K/V chunks are served from L2 after the first
-// fetch.  A KV block of b keys is processed as b/128 chunks of 128 keys.
+// CTA = two 128-row query tiles that read the same KV head, so every K/V
+// chunk the CTA loads serves both (KV reuse across the heads of a GQA group,
+// FAST-Prefill article section 2.2):
+//   b = 256:            the two 128-row halves of one 256-row query block
+//   b = 128, g >= 2:    the same query tile of two heads of one GQA group
+//   b = 128, g == 1:    two neighbouring query tiles of one head
+// The CTA walks the union of the two tiles' chunk lists (ascending 128-key
+// chunks); a chunk only one tile needs is computed for that tile only.
+// CTAs are numbered heavy first (descending query position).
 //
-// Warp roles (192 threads):
-//   warps 0-3  softmax / correction / epilogue; thread = one query row = one
-//              TMEM lane
-//   warp 4     TMA producer: Q tile once, then K chunks (3-stage ring) and V
-//              chunks (2-stage ring) in list order
-//   warp 5     TMEM owner and MMA issuer (one thread)
-// TMEM (512 columns): S double buffer at [0,128) and [128,256), O at [256,384).
-// Shared memory: Q 32 KiB, K 3 x 32 KiB, V 2 x 32 KiB, P 32 KiB (bf16 Q/K;
-// half the Q/K bytes for int8), all in the 128-byte-swizzled K-major layout
-// (V is read MN-major).
+// Warp roles (320 threads):
+//   warps 0-3 / 4-7  softmax, correction and epilogue of tile 0 / tile 1;
+//                    thread = one query row = one TMEM lane
+//   warp 8           TMA producer: Q tiles once, then K and V chunks
+//                    (2-stage rings each) in union order
+//   warp 9           TMEM owner and MMA issuer (one thread)
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// The softmax writes P (bf16, two per column) over the first 64 columns of
+// its S tile and the P.V product reads it from TMEM (tcgen05.mma A operand
+// in tensor memory), so P never touches shared memory.
 //
-// Pipeline per chunk j (MMA thread order):
-//   QK(j+1) -> S[(j+1)&1]      as soon as K(j+1) has landed
-//   wait P(j), V(j); PV(j): O += P V
-// Softmax thread for chunk j: S -> registers, rowmax, P = 2^(s*scale2 - m)
-// with a lazily raised reference max m (raised only when the row max exceeds
-// it by more than 2^8; the correction O *= 2^(m_old - m_new) then runs after
-// PV(j-1) has completed), P -> shared memory, signal.
+// MMA issue order per union entry u: for each tile t, PV_t(u-1) then
+// QK_t(u).  While softmax t works on S_t(u), the tensor pipe runs the other
+// tile's PV and QK.  The reference max of a row is raised lazily (only when
+// the row max exceeds it by more than 2^8); the correction O *= 2^(m_old -
+// m_new) runs in TMEM after PV_t(u-1) has completed.
 #pragma once
+
+#include <climits>
 
 #include "ptx.cuh"
 
@@ -45,68 +50,144 @@ struct AttnParams {
 
 template <bool I8>
 struct AttnCfg {
-  static constexpr int kQKTile = I8 ? 16384 : 32768;
+  static constexpr int kQKTile = I8 ? 16384 : 32768;   // 128 rows x 128 elements
   static constexpr int kVTile = 32768;
-  static constexpr int kKStages = 3;
-  static constexpr int kVStages = 2;
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kQOff + kQKTile;
-  static constexpr int kVOff = kKOff + kKStages * kQKTile;
-  static constexpr int kPOff = kVOff + kVStages * kVTile;
-  static constexpr int kSmem = kPOff + 32768 + 1024;
-  static constexpr int kThreads = 192;
+  static constexpr int kQOff = 0;                        // two Q tiles
+  static constexpr int kKOff = kQOff + 2 * kQKTile;      // two K stages
+  static constexpr int kVOff = kKOff + 2 * kQKTile;      // two V stages
+  static constexpr int kSmem = kVOff + 2 * kVTile + 1024;
+  static constexpr int kThreads = 320;
 };
 
-// Number of 128-key chunks query tile qc attends to, given the list length of
-// its query block (ascending block list whose last entry is the diagonal).
-__device__ __forceinline__ int attn_chunks(int cnt, int b, int qc) {
-  const int per = b / 128;
-  return (cnt - 1) * per + (qc % per) + 1;
+// Number of CTAs (tile pairs) for a layer shape.
+__host__ __device__ inline int attn_pairs(int Hq, int Hkv, int S, int b) {
+  const int nq = S / 128, g = Hq / Hkv;
+  if (b == 256) return Hq * (S / b);
+  if (g >= 2) return Hkv * ((g + 1) / 2) * nq;
+  return Hq * ((nq + 1) / 2);
+}
+
+struct AttnTile {
+  int valid, h, qc, r, cnt, L;
+  const int *list;
+};
+
+// The two query tiles of CTA `pair`, heavy pairs first.
+__device__ inline void attn_pair_tiles(const AttnParams &P, int pair, AttnTile (&t)[2]) {
+  const int nq = P.S / 128, g = P.g;
+  int h0, h1, q0, q1, v1;
+  if (P.b == 256) {
+    const int rr = P.n - 1 - pair / P.Hq;
+    h0 = h1 = pair % P.Hq;
+    q0 = 2 * rr;
+    q1 = 2 * rr + 1;
+    v1 = 1;
+  } else if (g >= 2) {
+    const int hp = (g + 1) / 2, per_qc = P.Hkv * hp;
+    const int qc = nq - 1 - pair / per_qc, rem = pair % per_qc;
+    h0 = (rem / hp) * g + 2 * (rem % hp);
+    h1 = h0 + 1;
+    v1 = (2 * (rem % hp) + 1) < g;
+    q0 = q1 = qc;
+  } else {
+    const int m = (nq + 1) / 2 - 1 - pair / P.Hq;
+    h0 = h1 = pair % P.Hq;
+    q0 = 2 * m;
+    q1 = 2 * m + 1;
+    v1 = q1 < nq;
+  }
+  const int hs[2] = {h0, h1}, qs[2] = {q0, q1}, vs[2] = {1, v1};
+  const int per = P.b / 128;
+  for (int i = 0; i < 2; ++i) {
+    t[i].valid = vs[i];
+    t[i].h = hs[i];
+    t[i].qc = qs[i];
+    t[i].r = (qs[i] * 128) / P.b;
+    if (vs[i]) {
+      t[i].cnt = P.counts[(size_t)hs[i] * P.n + t[i].r];
+      t[i].list = P.cols + (size_t)hs[i] * ((size_t)P.n * (P.n + 1) / 2) + (size_t)t[i].r * (t[i].r + 1) / 2;
+      // the list is ascending and ends with the diagonal block r
+      t[i].L = t[i].cnt > 0 ? (t[i].cnt - 1) * per + (qs[i] % per) + 1 : 0;
+    } else {
+      t[i].cnt = 0;
+      t[i].list = nullptr;
+      t[i].L = 0;
+    }
+  }
+}
+
+// Walks one tile's 128-key chunks in ascending order (INT_MAX when done).
+struct ChunkCursor {
+  const int *lst;
+  int cnt, e, k, per, qc, next;
+  __device__ void init(const AttnTile &t, int per_) {
+    lst = t.list;
+    cnt = t.valid ? t.cnt : 0;
+    e = 0;
+    k = 0;
+    per = per_;
+    qc = t.qc;
+    advance();
+  }
+  __device__ void advance() {
+    next = INT_MAX;
+    if (e < cnt) {
+      const int kc = lst[e] * per + k;
+      if (++k == per) {
+        k = 0;
+        ++e;
+      }
+      if (kc <= qc) next = kc;
+      else e = cnt;
+    }
+  }
+};
+
+// Next entry of the union of two chunk sequences: chunk index and tile mask.
+__device__ inline bool union_next(ChunkCursor &a, ChunkCursor &b, int &kc, int &mask) {
+  kc = min(a.next, b.next);
+  if (kc == INT_MAX) return false;
+  mask = (a.next == kc ? 1 : 0) | (b.next == kc ? 2 : 0);
+  if (mask & 1) a.advance();
+  if (mask & 2) b.advance();
+  return true;
 }
 
 template <bool I8>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     k_sparse_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, AttnParams P) {
   using C = AttnCfg<I8>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_kfull[3], bar_kempty[3], bar_vfull[2], bar_vempty[2],
-      bar_sfull[2], bar_pfull, bar_odone;
+  __shared__ __align__(8) uint64_t bar_q, bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2],
+      bar_sfull[2], bar_pfull[2], bar_odone[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nq = P.S / 128;
-  const int qc = nq - 1 - (int)(blockIdx.x / P.Hq);
-  const int h = blockIdx.x % P.Hq;
-  const int kvh = h / P.g;
+  AttnTile tl[2];
+  attn_pair_tiles(P, blockIdx.x, tl);
+  const int kvh = tl[0].h / P.g;
   const int per = P.b / 128;
-  const int r = (qc * 128) / P.b;
-  const size_t list_off = (size_t)h * ((size_t)P.n * (P.n + 1) / 2) + (size_t)r * (r + 1) / 2;
-  const int cnt = P.counts[(size_t)h * P.n + r];
-  const int L = attn_chunks(cnt, P.b, qc);
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  const uint32_t sq = base + C::kQOff, sk = base + C::kKOff, sv = base + C::kVOff, sp = base + C::kPOff;
-  uint8_t *const p_gen = smem_raw + (sp - smem_u32(smem_raw));
+  const uint32_t sq = base + C::kQOff, sk = base + C::kKOff, sv = base + C::kVOff;
 
   if (threadIdx.x == 0) {
     abort_sh = 0;
     mbar_init(smem_u32(&bar_q), 1);
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bar_kfull[s]), 1);
       mbar_init(smem_u32(&bar_kempty[s]), 1);
-    }
-    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bar_vfull[s]), 1);
       mbar_init(smem_u32(&bar_vempty[s]), 1);
       mbar_init(smem_u32(&bar_sfull[s]), 1);
+      mbar_init(smem_u32(&bar_pfull[s]), 4);
+      mbar_init(smem_u32(&bar_odone[s]), 1);
     }
-    mbar_init(smem_u32(&bar_pfull), 4);
-    mbar_init(smem_u32(&bar_odone), 1);
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&tmem_base_sh), 512);
     tmem_relinquish();
   }
@@ -116,118 +197,142 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = tmem_base_sh;
   volatile int *abort_flag = &abort_sh;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
-      const int qrow = h * P.S + qc * 128;
-      mbar_expect_tx(smem_u32(&bar_q), C::kQKTile);
-      tma_load_2d(sq, &tm_q, 0, qrow, smem_u32(&bar_q));
-      if (!I8) tma_load_2d(sq + 16384, &tm_q, 64, qrow, smem_u32(&bar_q));
-      const int *lst = P.cols + list_off;
-      int j = 0;
-      bool ok = true;
-      for (int e = 0; e < cnt && ok; ++e) {
-        const int c = lst[e];
-        for (int k = 0; k < per && ok; ++k) {
-          const int kc = c * per + k;
-          if (kc > qc) break;
-          const int krow = kvh * P.S + kc * 128;
-          const int ks = j % 3, vs = j & 1;
-          if (j >= 3 && !mbar_wait(smem_u32(&bar_kempty[ks]), ((j / 3) - 1) & 1, abort_flag, P.err)) {
-            ok = false;
-            break;
-          }
-          mbar_expect_tx(smem_u32(&bar_kfull[ks]), C::kQKTile);
-          tma_load_2d(sk + ks * C::kQKTile, &tm_k, 0, krow, smem_u32(&bar_kfull[ks]));
-          if (!I8) tma_load_2d(sk + ks * C::kQKTile + 16384, &tm_k, 64, krow, smem_u32(&bar_kfull[ks]));
-          if (j >= 2 && !mbar_wait(smem_u32(&bar_vempty[vs]), ((j / 2) - 1) & 1, abort_flag, P.err)) {
-            ok = false;
-            break;
-          }
-          mbar_expect_tx(smem_u32(&bar_vfull[vs]), C::kVTile);
-          tma_load_2d(sv + vs * C::kVTile, &tm_v, 0, krow, smem_u32(&bar_vfull[vs]));
-          tma_load_2d(sv + vs * C::kVTile + 16384, &tm_v, 64, krow, smem_u32(&bar_vfull[vs]));
-          ++j;
-        }
+      const int nt = tl[1].valid ? 2 : 1;
+      mbar_expect_tx(smem_u32(&bar_q), nt * C::kQKTile);
+      for (int t = 0; t < nt; ++t) {
+        const int qrow = tl[t].h * P.S + tl[t].qc * 128;
+        const uint32_t dst = sq + t * C::kQKTile;
+        tma_load_2d(dst, &tm_q, 0, qrow, smem_u32(&bar_q));
+        if (!I8) tma_load_2d(dst + 16384, &tm_q, 64, qrow, smem_u32(&bar_q));
+      }
+      ChunkCursor ca, cb;
+      ca.init(tl[0], per);
+      cb.init(tl[1], per);
+      int kc, mask;
+      for (int u = 0; union_next(ca, cb, kc, mask); ++u) {
+        const int st = u & 1;
+        const int krow = kvh * P.S + kc * 128;
+        if (u >= 2 && !mbar_wait(smem_u32(&bar_kempty[st]), ((u >> 1) - 1) & 1, abort_flag, P.err)) break;
+        mbar_expect_tx(smem_u32(&bar_kfull[st]), C::kQKTile);
+        tma_load_2d(sk + st * C::kQKTile, &tm_k, 0, krow, smem_u32(&bar_kfull[st]));
+        if (!I8) tma_load_2d(sk + st * C::kQKTile + 16384, &tm_k, 64, krow, smem_u32(&bar_kfull[st]));
+        if (u >= 2 && !mbar_wait(smem_u32(&bar_vempty[st]), ((u >> 1) - 1) & 1, abort_flag, P.err)) break;
+        mbar_expect_tx(smem_u32(&bar_vfull[st]), C::kVTile);
+        tma_load_2d(sv + st * C::kVTile, &tm_v, 0, krow, smem_u32(&bar_vfull[st]));
+        tma_load_2d(sv + st * C::kVTile + 16384, &tm_v, 64, krow, smem_u32(&bar_vfull[st]));
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = I8 ? idesc_i8(128, 128) : idesc_bf16(128, 128, 0);
       const uint32_t id_pv = idesc_bf16(128, 128, 1);
-      auto issue_qk = [&](int j) -> bool {
-        const int ks = j % 3;
-        if (!mbar_wait(smem_u32(&bar_kfull[ks]), (j / 3) & 1, abort_flag, P.err)) return false;
+      ChunkCursor ca, cb;
+      ca.init(tl[0], per);
+      cb.init(tl[1], per);
+      int npv[2] = {0, 0};
+      int prev = 0;
+      bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, P.err);
+      int u = 0;
+      // issue_pv: O_t += P_t(TMEM) . V(stage), for the entry before u
+      auto issue_pv = [&](int t, int vst) -> bool {
+        if (!mbar_wait(smem_u32(&bar_pfull[t]), npv[t] & 1, abort_flag, P.err)) return false;
         tc_fence_after();
-        const uint32_t kb = sk + ks * C::kQKTile;
-        const uint32_t d_tmem = tmem + (j & 1) * 128;
-        if (I8) {
+        const uint32_t vb = sv + vst * C::kVTile;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_i8_ss(d_tmem, umma_desc_sw128(sq + kk * 32, 16, 1024),
-                      umma_desc_sw128(kb + kk * 32, 16, 1024), id_qk, kk > 0);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(d_tmem, umma_desc_sw128(sq + off, 16, 1024),
-                        umma_desc_sw128(kb + off, 16, 1024), id_qk, kk > 0);
-          }
-        }
-        tc_commit(smem_u32(&bar_sfull[j & 1]));
-        tc_commit(smem_u32(&bar_kempty[ks]));
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
+                      umma_desc_sw128(vb + kk * 2048, 16384, 1024), id_pv, (npv[t] > 0 || kk > 0));
+        tc_commit(smem_u32(&bar_odone[t]));
+        ++npv[t];
         return true;
       };
-      bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, P.err) && issue_qk(0);
-      for (int j = 0; ok && j < L; ++j) {
-        if (j + 1 < L && !issue_qk(j + 1)) break;
-        if (!mbar_wait(smem_u32(&bar_pfull), j & 1, abort_flag, P.err)) break;
-        const int vs = j & 1;
-        if (!mbar_wait(smem_u32(&bar_vfull[vs]), (j >> 1) & 1, abort_flag, P.err)) break;
-        tc_fence_after();
-        const uint32_t vb = sv + vs * C::kVTile;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t aoff = (kk >> 2) * 16384 + (kk & 3) * 32;
-          mma_bf16_ss(tmem + 256, umma_desc_sw128(sp + aoff, 16, 1024),
-                      umma_desc_sw128(vb + kk * 2048, 16384, 1024), id_pv, (j > 0 || kk > 0));
+      int kc, mask;
+      while (ok) {
+        const bool more = union_next(ca, cb, kc, mask);
+        if (prev) {
+          const int pst = (u - 1) & 1;
+          if (!mbar_wait(smem_u32(&bar_vfull[pst]), ((u - 1) >> 1) & 1, abort_flag, P.err)) break;
         }
-        tc_commit(smem_u32(&bar_odone));
-        tc_commit(smem_u32(&bar_vempty[vs]));
+        bool kwaited = false;
+        const int st = u & 1;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if ((prev >> t) & 1) ok = issue_pv(t, (u - 1) & 1);
+          if (ok && more && ((mask >> t) & 1)) {
+            if (!kwaited) {
+              if (!mbar_wait(smem_u32(&bar_kfull[st]), (u >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
+              tc_fence_after();
+              kwaited = true;
+            }
+            const uint32_t qb = sq + t * C::kQKTile, kb = sk + st * C::kQKTile;
+            const uint32_t d_tmem = tmem + t * 128;
+            if (I8) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_i8_ss(d_tmem, umma_desc_sw128(qb + kk * 32, 16, 1024),
+                          umma_desc_sw128(kb + kk * 32, 16, 1024), id_qk, kk > 0);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16_ss(d_tmem, umma_desc_sw128(qb + off, 16, 1024),
+                            umma_desc_sw128(kb + off, 16, 1024), id_qk, kk > 0);
+              }
+            }
+            tc_commit(smem_u32(&bar_sfull[t]));
+          }
+        }
+        if (!ok) break;
+        if (prev) tc_commit(smem_u32(&bar_vempty[(u - 1) & 1]));
+        if (!more) break;
+        tc_commit(smem_u32(&bar_kempty[st]));
+        prev = mask;
+        ++u;
       }
     }
   } else {
     // ---------------------------------------------------------------- softmax
-    const int row = warp * 32 + lane;
-    const uint32_t lane_off = ((uint32_t)(warp * 32)) << 16;
+    const int t = warp >> 2;
+    const AttnTile &me = tl[t];
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
+    const uint32_t s_tm = tmem + t * 128 + lane_off, o_tm = tmem + 256 + t * 128 + lane_off;
     float scale2 = P.scale2;
-    if (I8) scale2 *= P.q_scale[h] * P.k_scale[kvh];
+    if (I8 && me.valid) scale2 *= P.q_scale[me.h] * P.k_scale[kvh];
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    const int L = me.L;
     for (int j = 0; j < L; ++j) {
-      if (!mbar_wait(smem_u32(&bar_sfull[j & 1]), (j >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
+      if (!mbar_wait(smem_u32(&bar_sfull[t]), j & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
+      // the whole 128-column row in one TMEM load, one wait
+      uint32_t rr[128];
+      tmem_ld128(s_tm, rr);
+      tmem_ld_wait128(rr);
       float s[128];
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
-        uint32_t rr[32];
-        tmem_ld32(tmem + (j & 1) * 128 + lane_off + qq * 32, rr);
-        tmem_ld_wait(rr);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[qq * 32 + e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
-      }
+      for (int e = 0; e < 128; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
       if (j == L - 1) {
-        // diagonal chunk: key t of the chunk is visible iff t <= row
+        // diagonal chunk: key e of the chunk is visible iff e <= row
 #pragma unroll
-        for (int t = 0; t < 128; ++t) s[t] = (t <= row) ? s[t] : -INFINITY;
+        for (int e = 0; e < 128; ++e) s[e] = (e <= row) ? s[e] : -INFINITY;
       }
-      float mx = s[0];
+      // row max as 8 independent chains, then a short tree
+      float m8[8];
 #pragma unroll
-      for (int t = 1; t < 128; ++t) mx = fmaxf(mx, s[t]);
+      for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+      for (int c = 8; c < 128; c += 8)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[c + e]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float rmax2 = mx * scale2;
       const bool raise = rmax2 > m_ref + 8.f;
       const float m_new = raise ? rmax2 : m_ref;
@@ -235,52 +340,48 @@ __global__ void __launch_bounds__(192, 1)
       // P in bf16 (the P.V operand); the row sum adds the same rounded values
       // so numerator and denominator use identical weights.
       uint32_t pk[64];
-      float rs = 0.f;
+      float r8[8];
 #pragma unroll
-      for (int t = 0; t < 128; t += 2) {
-        pk[t >> 1] = pack_bf16x2(ex2(fmaf(s[t], scale2, -m_new)), ex2(fmaf(s[t + 1], scale2, -m_new)));
-        rs += __uint_as_float(pk[t >> 1] << 16) + __uint_as_float(pk[t >> 1] & 0xFFFF0000u);
+      for (int e = 0; e < 8; ++e) r8[e] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 128; e += 2) {
+        pk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], scale2, -m_new)), ex2(fmaf(s[e + 1], scale2, -m_new)));
+        r8[(e >> 1) & 7] += __uint_as_float(pk[e >> 1] << 16) + __uint_as_float(pk[e >> 1] & 0xFFFF0000u);
       }
+      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l = l * alpha + rs;
       m_ref = m_new;
       if (j > 0) {
-        // PV(j-1) complete: O is stable and the P buffer is free
-        if (!mbar_wait(smem_u32(&bar_odone), (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
+        // PV(j-1) complete: O is stable
+        if (!mbar_wait(smem_u32(&bar_odone[t]), (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
           for (int qq = 0; qq < 4; ++qq) {
             uint32_t o[32];
-            tmem_ld32(tmem + 256 + lane_off + qq * 32, o);
+            tmem_ld32(o_tm + qq * 32, o);
             tmem_ld_wait(o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tmem + 256 + lane_off + qq * 32, o);
+            tmem_st32(o_tm + qq * 32, o);
           }
-          tmem_st_wait();
         }
       }
-      // P row -> shared memory, K-major 128-byte swizzle: key t of row `row`
-      // lives in 64-key half t/64, 16-byte chunk ((t%64)/8) ^ (row%8).
-#pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        const uint4 v = make_uint4(pk[c8 * 4 + 0], pk[c8 * 4 + 1], pk[c8 * 4 + 2], pk[c8 * 4 + 3]);
-        const int half = c8 >> 3, chunk = (c8 & 7) ^ (row & 7);
-        *reinterpret_cast<uint4 *>(p_gen + half * 16384 + row * 128 + chunk * 16) = v;
-      }
-      fence_proxy_async_smem();
+      // P over the first 64 columns of this tile's S
+      tmem_st64(s_tm, pk);
+      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bar_pfull));
+      if (lane == 0) mbar_arrive(smem_u32(&bar_pfull[t]));
     }
-    if (ok && L > 0 && mbar_wait(smem_u32(&bar_odone), (L - 1) & 1, abort_flag, P.err)) {
+    if (ok && L > 0 && mbar_wait(smem_u32(&bar_odone[t]), (L - 1) & 1, abort_flag, P.err)) {
       tc_fence_after();
       const float inv = 1.f / l;
-      __nv_bfloat16 *orow = P.out + ((size_t)h * P.S + (size_t)qc * 128 + row) * 128;
+      __nv_bfloat16 *orow = P.out + ((size_t)me.h * P.S + (size_t)me.qc * 128 + row) * 128;
 #pragma unroll 1
       for (int qq = 0; qq < 4; ++qq) {
         uint32_t o[32];
-        tmem_ld32(tmem + 256 + lane_off + qq * 32, o);
+        tmem_ld32(o_tm + qq * 32, o);
         tmem_ld_wait(o);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
@@ -296,7 +397,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -206,7 +206,7 @@ int attn_impl(const void *q, const void *k, const void *v, const float *q_scale,
   ap.scale2 = kLog2e / sqrtf((float)I->d);
   ap.out = static_cast<__nv_bfloat16 *>(out);
   ap.err = err;
-  const unsigned grid = (unsigned)I->Hq * (unsigned)(I->S / 128);
+  const unsigned grid = (unsigned)attn_pairs(I->Hq, I->Hkv, I->S, I->b);
   k_sparse_attn<I8><<<grid, AttnCfg<I8>::kThreads, AttnCfg<I8>::kSmem, st>>>(tq, tk, tv, ap);
   return launch_status();
 }

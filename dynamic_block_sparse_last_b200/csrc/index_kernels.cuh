@@ -35,7 +35,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // 128-row slice of the b-row last block).  Warps:
 //   0..15  statistics: warpgroup t owns tile t; thread = one query row
 //   16     TMA producer     17  MMA issuer + TMEM owner
-//   18,19  K column sums for the block means (only CTAs of tile group 0)
+//   18     K column sums for the block means (only CTAs of tile group 0)
 // TMEM: tile t's 128x128 fp32 score tile at columns [128t, 128t+128).
 // ---------------------------------------------------------------------------
 struct ScoreParams {
@@ -54,12 +54,14 @@ template <bool I8>
 struct ScoreCfg {
   static constexpr int kStages = I8 ? 4 : 3;
   static constexpr int kTileBytes = I8 ? 16384 : 32768;  // 128 rows x 128 elements
-  static constexpr int kThreads = 640;
+  static constexpr int kThreads = 608;
   static constexpr int kSmem = 4 * kTileBytes + kStages * kTileBytes + 1024;
+  // warps 0-15 statistics, 16 producer, 17 MMA, 18 K column sums
+  static_assert(kThreads == 19 * 32, "k_score_last warp roles need exactly 19 warps");
 };
 
 template <bool I8>
-__global__ void __launch_bounds__(640, 1)
+__global__ void __launch_bounds__(608, 1)
     k_score_last(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  ScoreParams P) {
   using C = ScoreCfg<I8>;
@@ -77,7 +79,7 @@ __global__ void __launch_bounds__(640, 1)
   const int ch1 = min(P.nch, ch0 + P.chunks_per_cta);
   const int U = ch1 - ch0;
   const bool do_ksum = (blockIdx.y == 0);
-  const int n_ksum_warps = do_ksum ? (I8 ? 1 : 2) : 0;
+  const int n_ksum_warps = do_ksum ? 1 : 0;
   const int tiles_per_head = P.b / 128;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -200,18 +202,22 @@ __global__ void __launch_bounds__(640, 1)
             out[4 * lane + 2] = (float)acc2;
             out[4 * lane + 3] = (float)acc3;
           } else {
-            // warp kw reads the 64-column half kw; lane owns columns 2*lane, 2*lane+1
-            const uint8_t *half = tile + kw * 16384;
-            float a0 = 0.f, a1 = 0.f;
+            // lane owns columns 2*lane, 2*lane+1 of each 64-column half
+            float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
             for (int r = 0; r < 128; ++r) {
               const int phys = (((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) << 2);
-              const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(half + r * 128 + phys);
-              const float2 f = __bfloat1622float2(v);
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(tile + r * 128 + phys));
+              const float2 e = __bfloat1622float2(
+                  *reinterpret_cast<const __nv_bfloat162 *>(tile + 16384 + r * 128 + phys));
               a0 += f.x;
               a1 += f.y;
+              c0 += e.x;
+              c1 += e.y;
             }
-            out[kw * 64 + 2 * lane] = a0;
-            out[kw * 64 + 2 * lane + 1] = a1;
+            out[2 * lane] = a0;
+            out[2 * lane + 1] = a1;
+            out[64 + 2 * lane] = c0;
+            out[64 + 2 * lane + 1] = c1;
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bar_kempty[st]));
@@ -235,7 +241,8 @@ __global__ void __launch_bounds__(640, 1)
           const int tb = (ch * 128) % P.b;                 // chunk offset inside its block
           const bool last_block = (ch * 128) / P.b == P.n - 1;
           // pass 1: row max over the causal columns t <= i of the last block
-          float mx = -INFINITY;
+          // (four independent max chains)
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
           for (int qq = 0; qq < 4; ++qq) {
             uint32_t r[32];
@@ -246,10 +253,11 @@ __global__ void __launch_bounds__(640, 1)
             for (int e = 0; e < 32; ++e) {
               const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
               const bool valid = !last_block || (t0 + e <= i);
-              mx = valid ? fmaxf(mx, s) : mx;
+              m4[e & 3] = valid ? fmaxf(m4[e & 3], s) : m4[e & 3];
             }
           }
-          float lo = 0.f, hi = 0.f;
+          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          float lo4[4] = {0.f, 0.f, 0.f, 0.f}, hi4[4] = {0.f, 0.f, 0.f, 0.f};
           const float m2 = mx * scale2;
           if (mx != -INFINITY) {
 #pragma unroll 1
@@ -259,34 +267,32 @@ __global__ void __launch_bounds__(640, 1)
               tmem_ld_wait(r);
               const int dlt = i - (tb + qq * 32);   // columns e <= dlt are on the lo side
               if (dlt >= 31) {
-                float acc = 0.f;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                   const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
-                  acc += ex2(fmaf(s, scale2, -m2));
+                  lo4[e & 3] += ex2(fmaf(s, scale2, -m2));
                 }
-                lo += acc;
               } else if (dlt < 0) {
                 if (!last_block) {
-                  float acc = 0.f;
 #pragma unroll
                   for (int e = 0; e < 32; ++e) {
                     const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
-                    acc += ex2(fmaf(s, scale2, -m2));
+                    hi4[e & 3] += ex2(fmaf(s, scale2, -m2));
                   }
-                  hi += acc;
                 }
               } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                   const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
                   const float p = ex2(fmaf(s, scale2, -m2));
-                  if (e <= dlt) lo += p;
-                  else if (!last_block) hi += p;
+                  if (e <= dlt) lo4[e & 3] += p;
+                  else if (!last_block) hi4[e & 3] += p;
                 }
               }
             }
           }
+          const float lo = (lo4[0] + lo4[1]) + (lo4[2] + lo4[3]);
+          const float hi = (hi4[0] + hi4[1]) + (hi4[2] + hi4[3]);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bar_sfree[t]));
