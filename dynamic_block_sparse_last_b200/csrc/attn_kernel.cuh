@@ -32,8 +32,6 @@
 // m_new) runs in TMEM after PV_t(u-1) has completed.
 #pragma once
 
-#include <climits>
-
 #include "ptx.cuh"
 
 namespace fpk {
@@ -116,42 +114,47 @@ __device__ inline void attn_pair_tiles(const AttnParams &P, int pair, AttnTile (
   }
 }
 
-// Walks one tile's 128-key chunks in ascending order (INT_MAX when done).
-struct ChunkCursor {
-  const int *lst;
-  int cnt, e, k, per, qc, next;
-  __device__ void init(const AttnTile &t, int per_) {
-    lst = t.list;
-    cnt = t.valid ? t.cnt : 0;
-    e = 0;
-    k = 0;
-    per = per_;
-    qc = t.qc;
-    advance();
-  }
-  __device__ void advance() {
-    next = INT_MAX;
-    if (e < cnt) {
-      const int kc = lst[e] * per + k;
-      if (++k == per) {
-        k = 0;
-        ++e;
-      }
-      if (kc <= qc) next = kc;
-      else e = cnt;
+// Chunk bitmaps: bit kc of tile t's map is set when the tile attends to the
+// 128-key chunk kc.  Built once per CTA in shared memory from the block lists
+// (coalesced loads by 64 lanes), so the producer and the MMA issuer walk the
+// union without global-memory round trips.
+constexpr int kMaxChunkWords = 64;  // 2048 chunks: S/128 <= 2048 for S/b <= 1024, b <= 256
+
+__device__ inline void build_chunk_bitmap(const AttnTile &t, int per, uint32_t *bm, int lane64) {
+  if (!t.valid) return;
+  for (int e = lane64; e < t.cnt; e += 64) {
+    const int c = t.list[e];
+    for (int k = 0; k < per; ++k) {
+      const int kc = c * per + k;
+      if (kc <= t.qc) atomicOr(&bm[kc >> 5], 1u << (kc & 31));
     }
   }
-};
-
-// Next entry of the union of two chunk sequences: chunk index and tile mask.
-__device__ inline bool union_next(ChunkCursor &a, ChunkCursor &b, int &kc, int &mask) {
-  kc = min(a.next, b.next);
-  if (kc == INT_MAX) return false;
-  mask = (a.next == kc ? 1 : 0) | (b.next == kc ? 2 : 0);
-  if (mask & 1) a.advance();
-  if (mask & 2) b.advance();
-  return true;
 }
+
+// Iterates the union of the two tiles' chunk sets in ascending order.
+struct UnionWalk {
+  const uint32_t *a, *b;
+  int words, wi;
+  uint32_t cur;
+  __device__ void init(const uint32_t *a_, const uint32_t *b_, int words_) {
+    a = a_;
+    b = b_;
+    words = words_;
+    wi = 0;
+    cur = words > 0 ? (a[0] | b[0]) : 0u;
+  }
+  __device__ bool next(int &kc, int &mask) {
+    while (cur == 0u) {
+      if (++wi >= words) return false;
+      cur = a[wi] | b[wi];
+    }
+    const int bit = __ffs(cur) - 1;
+    cur &= cur - 1u;
+    kc = wi * 32 + bit;
+    mask = (int)((a[wi] >> bit) & 1u) | (int)(((b[wi] >> bit) & 1u) << 1);
+    return true;
+  }
+};
 
 template <bool I8>
 __global__ void __launch_bounds__(320, 1)
@@ -163,12 +166,14 @@ __global__ void __launch_bounds__(320, 1)
       bar_sfull[2], bar_pfull[2], bar_odone[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
+  __shared__ uint32_t chunk_bm[2][kMaxChunkWords];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   AttnTile tl[2];
   attn_pair_tiles(P, blockIdx.x, tl);
   const int kvh = tl[0].h / P.g;
   const int per = P.b / 128;
+  const int words = (max(tl[0].qc, tl[1].valid ? tl[1].qc : 0) >> 5) + 1;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t sq = base + C::kQOff, sk = base + C::kKOff, sv = base + C::kVOff;
@@ -187,9 +192,16 @@ __global__ void __launch_bounds__(320, 1)
     }
     fence_mbar_init();
   }
+  for (int i = threadIdx.x; i < 2 * kMaxChunkWords; i += blockDim.x) (&chunk_bm[0][0])[i] = 0u;
   if (warp == 9) {
     tmem_alloc(smem_u32(&tmem_base_sh), 512);
     tmem_relinquish();
+  }
+  __syncthreads();
+  if (warp >= 8) {
+    const int lane64 = threadIdx.x - 256;
+    build_chunk_bitmap(tl[0], per, chunk_bm[0], lane64);
+    build_chunk_bitmap(tl[1], per, chunk_bm[1], lane64);
   }
   tc_fence_before();
   __syncthreads();
@@ -211,11 +223,10 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_2d(dst, &tm_q, 0, qrow, smem_u32(&bar_q));
         if (!I8) tma_load_2d(dst + 16384, &tm_q, 64, qrow, smem_u32(&bar_q));
       }
-      ChunkCursor ca, cb;
-      ca.init(tl[0], per);
-      cb.init(tl[1], per);
+      UnionWalk uw;
+      uw.init(chunk_bm[0], chunk_bm[1], words);
       int kc, mask;
-      for (int u = 0; union_next(ca, cb, kc, mask); ++u) {
+      for (int u = 0; uw.next(kc, mask); ++u) {
         const int st = u & 1;
         const int krow = kvh * P.S + kc * 128;
         if (u >= 2 && !mbar_wait(smem_u32(&bar_kempty[st]), ((u >> 1) - 1) & 1, abort_flag, P.err)) break;
@@ -233,9 +244,8 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       const uint32_t id_qk = I8 ? idesc_i8(128, 128) : idesc_bf16(128, 128, 0);
       const uint32_t id_pv = idesc_bf16(128, 128, 1);
-      ChunkCursor ca, cb;
-      ca.init(tl[0], per);
-      cb.init(tl[1], per);
+      UnionWalk uw;
+      uw.init(chunk_bm[0], chunk_bm[1], words);
       int npv[2] = {0, 0};
       int prev = 0;
       bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, P.err);
@@ -255,7 +265,7 @@ __global__ void __launch_bounds__(320, 1)
       };
       int kc, mask;
       while (ok) {
-        const bool more = union_next(ca, cb, kc, mask);
+        const bool more = uw.next(kc, mask);
         if (prev) {
           const int pst = (u - 1) & 1;
           if (!mbar_wait(smem_u32(&bar_vfull[pst]), ((u - 1) >> 1) & 1, abort_flag, P.err)) break;
