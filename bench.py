@@ -343,6 +343,46 @@ def run_ours(args, w):
     return 0
 
 
+def run_sweep(args):
+    """The S x b x gamma sweep on the 128K generator (Hq=32, Hkv=8): one JSON
+    line per point with density next to time (not the headline line)."""
+    from dynamic_block_sparse_last_b200 import fp
+    dev = torch.device("cuda", 0)
+    cache = {}
+    for w in synth.sweep_workloads():
+        if w.S not in cache:
+            cache.clear()
+            x = synth.make_inputs(w)
+            cache[w.S] = (x["q"].to(dev), x["k"].to(dev), x["v"].to(dev))
+        q, k, v = cache[w.S]
+        out = torch.empty_like(q)
+        idx = fp.fp_index_create(w.S, w.Hq, w.Hkv, w.d, w.b)
+        for _ in range(args.warmup):
+            fp.fp_build_index(q, k, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, fp.FP_QK_BF16, None, None, idx)
+            fp.fp_sparse_attn(q, k, v, None, None, idx, out)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+        for e in ev:
+            e[0].record()
+            fp.fp_build_index(q, k, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, fp.FP_QK_BF16, None, None, idx)
+            e[1].record()
+            fp.fp_sparse_attn(q, k, v, None, None, idx, out)
+            e[2].record()
+        torch.cuda.synchronize()
+        assert fp.fp_get_device_error() == fp.FP_OK
+        n = w.S // w.b
+        nnz = fp.fp_index_nnz(idx)
+        idx_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
+        attn_ms = float(np.median([e[1].elapsed_time(e[2]) for e in ev]))
+        layer = idx_ms + attn_ms
+        print(json.dumps({"sweep": w.name, "S": w.S, "b": w.b, "gamma": w.gamma,
+                          "density": nnz / (w.Hq * n * (n + 1) / 2), "index_ms": idx_ms, "attn_ms": attn_ms,
+                          "ms_per_layer": layer,
+                          "dense_equiv_tflops": synth.dense_equiv_flops(w.S, w.Hq, w.d) / (layer / 1e3) / 1e12}),
+              flush=True)
+        idx.free()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -351,9 +391,12 @@ def main():
     ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="S x b x gamma sweep (one line per point)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.sweep:
+        return run_sweep(args)
     w = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

@@ -14,12 +14,12 @@
 // chunks); a chunk only one tile needs is computed for that tile only.
 // CTAs are numbered heavy first (descending query position).
 //
-// Warp roles (320 threads):
+// Warp roles (352 threads):
 //   warps 0-3 / 4-7  softmax, correction and epilogue of tile 0 / tile 1;
 //                    thread = one query row = one TMEM lane
-//   warp 8           TMA producer: Q tiles once, then K and V chunks
-//                    (2-stage rings each) in union order
+//   warp 8           TMA producer: Q tiles once, then K chunks (3-stage ring)
 //   warp 9           TMEM owner and MMA issuer (one thread)
+//   warp 10          TMA producer of V chunks (2-stage ring)
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // The softmax writes P (bf16, two per column) over the first 64 columns of
 // its S tile and the P.V product reads it from TMEM (tcgen05.mma A operand
@@ -50,11 +50,16 @@ template <bool I8>
 struct AttnCfg {
   static constexpr int kQKTile = I8 ? 16384 : 32768;   // 128 rows x 128 elements
   static constexpr int kVTile = 32768;
-  static constexpr int kQOff = 0;                        // two Q tiles
-  static constexpr int kKOff = kQOff + 2 * kQKTile;      // two K stages
-  static constexpr int kVOff = kKOff + 2 * kQKTile;      // two V stages
-  static constexpr int kSmem = kVOff + 2 * kVTile + 1024;
-  static constexpr int kThreads = 320;
+  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr int kQOff = 0;                                 // two Q tiles
+  static constexpr int kKOff = kQOff + 2 * kQKTile;               // K ring
+  static constexpr int kVOff = kKOff + kKStages * kQKTile;        // V ring
+  static constexpr int kSmem = kVOff + kVStages * kVTile + 1024;
+  static constexpr int kThreads = 352;
+  // Every kExpFmaEvery-th exponential of an off-diagonal chunk runs on the
+  // FMA pipe (ex2_fma) instead of MUFU; 0 keeps all on MUFU.  A share of 1/4
+  // measured no faster on the 128K layer (power-capped clocks), so it is off.
+  static constexpr int kExpFmaEvery = 0;
 };
 
 // Number of CTAs (tile pairs) for a layer shape.
@@ -157,12 +162,12 @@ struct UnionWalk {
 };
 
 template <bool I8>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     k_sparse_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, AttnParams P) {
   using C = AttnCfg<I8>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2],
+  __shared__ __align__(8) uint64_t bar_q, bar_kfull[3], bar_kempty[3], bar_vfull[2], bar_vempty[2],
       bar_sfull[2], bar_pfull[2], bar_odone[2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -181,9 +186,11 @@ __global__ void __launch_bounds__(320, 1)
   if (threadIdx.x == 0) {
     abort_sh = 0;
     mbar_init(smem_u32(&bar_q), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 3; ++s) {
       mbar_init(smem_u32(&bar_kfull[s]), 1);
       mbar_init(smem_u32(&bar_kempty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bar_vfull[s]), 1);
       mbar_init(smem_u32(&bar_vempty[s]), 1);
       mbar_init(smem_u32(&bar_sfull[s]), 1);
@@ -198,7 +205,7 @@ __global__ void __launch_bounds__(320, 1)
     tmem_relinquish();
   }
   __syncthreads();
-  if (warp >= 8) {
+  if (warp == 8 || warp == 9) {
     const int lane64 = threadIdx.x - 256;
     build_chunk_bitmap(tl[0], per, chunk_bm[0], lane64);
     build_chunk_bitmap(tl[1], per, chunk_bm[1], lane64);
@@ -214,7 +221,6 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
-      tma_prefetch_map(&tm_v);
       const int nt = tl[1].valid ? 2 : 1;
       mbar_expect_tx(smem_u32(&bar_q), nt * C::kQKTile);
       for (int t = 0; t < nt; ++t) {
@@ -223,20 +229,36 @@ __global__ void __launch_bounds__(320, 1)
         tma_load_2d(dst, &tm_q, 0, qrow, smem_u32(&bar_q));
         if (!I8) tma_load_2d(dst + 16384, &tm_q, 64, qrow, smem_u32(&bar_q));
       }
-      UnionWalk uw;
-      uw.init(chunk_bm[0], chunk_bm[1], words);
+      // K runs up to three chunks ahead of the MMA issuer; V (warp 10) has
+      // its own ring and producer, so neither waits on the other's slots.
+      UnionWalk wk;
+      wk.init(chunk_bm[0], chunk_bm[1], words);
       int kc, mask;
-      for (int u = 0; uw.next(kc, mask); ++u) {
-        const int st = u & 1;
-        const int krow = kvh * P.S + kc * 128;
-        if (u >= 2 && !mbar_wait(smem_u32(&bar_kempty[st]), ((u >> 1) - 1) & 1, abort_flag, P.err)) break;
+      for (int u = 0; wk.next(kc, mask); ++u) {
+        const int st = u % C::kKStages, krow = kvh * P.S + kc * 128;
+        if (u >= C::kKStages &&
+            !mbar_wait(smem_u32(&bar_kempty[st]), ((u / C::kKStages) - 1) & 1, abort_flag, P.err))
+          break;
         mbar_expect_tx(smem_u32(&bar_kfull[st]), C::kQKTile);
         tma_load_2d(sk + st * C::kQKTile, &tm_k, 0, krow, smem_u32(&bar_kfull[st]));
         if (!I8) tma_load_2d(sk + st * C::kQKTile + 16384, &tm_k, 64, krow, smem_u32(&bar_kfull[st]));
-        if (u >= 2 && !mbar_wait(smem_u32(&bar_vempty[st]), ((u >> 1) - 1) & 1, abort_flag, P.err)) break;
+      }
+    }
+  } else if (warp == 10) {
+    // ---------------------------------------------------------------- V producer
+    if (lane == 0) {
+      tma_prefetch_map(&tm_v);
+      UnionWalk wv;
+      wv.init(chunk_bm[0], chunk_bm[1], words);
+      int kc, mask;
+      for (int u = 0; wv.next(kc, mask); ++u) {
+        const int st = u % C::kVStages, vrow = kvh * P.S + kc * 128;
+        if (u >= C::kVStages &&
+            !mbar_wait(smem_u32(&bar_vempty[st]), ((u / C::kVStages) - 1) & 1, abort_flag, P.err))
+          break;
         mbar_expect_tx(smem_u32(&bar_vfull[st]), C::kVTile);
-        tma_load_2d(sv + st * C::kVTile, &tm_v, 0, krow, smem_u32(&bar_vfull[st]));
-        tma_load_2d(sv + st * C::kVTile + 16384, &tm_v, 64, krow, smem_u32(&bar_vfull[st]));
+        tma_load_2d(sv + st * C::kVTile, &tm_v, 0, vrow, smem_u32(&bar_vfull[st]));
+        tma_load_2d(sv + st * C::kVTile + 16384, &tm_v, 64, vrow, smem_u32(&bar_vfull[st]));
       }
     }
   } else if (warp == 9) {
@@ -271,12 +293,12 @@ __global__ void __launch_bounds__(320, 1)
           if (!mbar_wait(smem_u32(&bar_vfull[pst]), ((u - 1) >> 1) & 1, abort_flag, P.err)) break;
         }
         bool kwaited = false;
-        const int st = u & 1;
+        const int st = u % C::kKStages;
         for (int t = 0; t < 2 && ok; ++t) {
           if ((prev >> t) & 1) ok = issue_pv(t, (u - 1) & 1);
           if (ok && more && ((mask >> t) & 1)) {
             if (!kwaited) {
-              if (!mbar_wait(smem_u32(&bar_kfull[st]), (u >> 1) & 1, abort_flag, P.err)) { ok = false; break; }
+              if (!mbar_wait(smem_u32(&bar_kfull[st]), (u / C::kKStages) & 1, abort_flag, P.err)) { ok = false; break; }
               tc_fence_after();
               kwaited = true;
             }
@@ -349,22 +371,34 @@ __global__ void __launch_bounds__(320, 1)
       const float alpha = raise ? ex2(m_ref - m_new) : 1.f;
       // P in bf16 (the P.V operand); the row sum adds the same rounded values
       // so numerator and denominator use identical weights.
+      // Off the diagonal chunk every fourth exponential runs on the FMA pipe
+      // (ex2_fma), the rest on MUFU; the diagonal chunk has masked (-inf)
+      // entries and uses MUFU only, which maps them to exactly 0.
       uint32_t pk[64];
       float r8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
+      if (C::kExpFmaEvery > 0 && j != L - 1) {
 #pragma unroll
-      for (int e = 0; e < 128; e += 2) {
-        pk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], scale2, -m_new)), ex2(fmaf(s[e + 1], scale2, -m_new)));
-        r8[(e >> 1) & 7] += __uint_as_float(pk[e >> 1] << 16) + __uint_as_float(pk[e >> 1] & 0xFFFF0000u);
+        for (int e = 0; e < 128; e += 2) {
+          const float x0 = fmaf(s[e], scale2, -m_new), x1 = fmaf(s[e + 1], scale2, -m_new);
+          const bool f1 = C::kExpFmaEvery > 0 && ((e + 1) % (C::kExpFmaEvery > 0 ? C::kExpFmaEvery : 1)) == 0;
+          pk[e >> 1] = pack_bf16x2(ex2(x0), f1 ? ex2_fma(x1) : ex2(x1));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 128; e += 2)
+          pk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], scale2, -m_new)), ex2(fmaf(s[e + 1], scale2, -m_new)));
       }
+#pragma unroll
+      for (int e = 0; e < 64; ++e)
+        r8[e & 7] += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
       const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l = l * alpha + rs;
       m_ref = m_new;
+      // The commit that signalled S(j) also covers PV(j-1), issued before
+      // QK(j): O is stable here and may be rescaled in place.
       if (j > 0) {
-        // PV(j-1) complete: O is stable
-        if (!mbar_wait(smem_u32(&bar_odone[t]), (j - 1) & 1, abort_flag, P.err)) { ok = false; break; }
-        tc_fence_after();
         if (__any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
           for (int qq = 0; qq < 4; ++qq) {

@@ -128,7 +128,7 @@ int set_smem_attrs() {
                            AttnCfg<I8>::kSmem) != cudaSuccess)
     return FP_ERR_CUDA;
   if (cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (kSelRows * kSelMaxN + kSelRows * 128 + 32 * 129) * 4) != cudaSuccess)
+                           kSelSmemFloats * (int)sizeof(float)) != cudaSuccess)
     return FP_ERR_CUDA;
   if (dev >= 0 && dev < 128) done[dev] = true;
   return FP_OK;
@@ -180,7 +180,7 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   if ((rc = launch_status())) return rc;
   k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->b, I->n, I->qbar);
   if ((rc = launch_status())) return rc;
-  const size_t sel_bytes = (size_t)(kSelRows * I->n + kSelRows * 128 + 32 * 129) * sizeof(float);
+  const size_t sel_bytes = (size_t)(kSelRows * I->n + kSelRows * 128 + 128 * kSelKStride) * sizeof(float);
   k_select<<<dim3((I->n + kSelRows - 1) / kSelRows, I->Hq), 256, sel_bytes, st>>>(
       I->pattern, I->vhat, I->shat, I->qbar, I->kbar, I->g, I->n, inv_sqrt_d, gamma, I->counts, I->cols);
   return launch_status();

@@ -322,16 +322,26 @@ __global__ void k_row_stats(const float *__restrict__ pm, const float *__restric
   const int h = blockIdx.x, part = blockIdx.y, R2 = gridDim.y, i = threadIdx.x;
   const int c0 = part * chunks_per_part, c1 = min(nch, c0 + chunks_per_part);
   float M = -INFINITY, L = 0.f;
-  for (int ch = c0; ch < c1; ++ch) {
-    const size_t o = ((size_t)h * nch + ch) * b + i;
-    const float m = pm[o];
-    if (m == -INFINITY) continue;
-    const float s = plo[o] + phi[o];
-    if (m > M) {
-      L = L * ex2(M - m) + s;
-      M = m;
-    } else {
-      L += s * ex2(m - M);
+  for (int ch = c0; ch < c1; ch += 4) {
+    // four chunks' loads in flight, then the running combine in order
+    float mv[4], sv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const size_t o = ((size_t)h * nch + ch + u) * b + i;
+      const bool in = ch + u < c1;
+      mv[u] = in ? pm[o] : -INFINITY;
+      sv[u] = in ? plo[o] + phi[o] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float m = mv[u];
+      if (m == -INFINITY) continue;
+      if (m > M) {
+        L = L * ex2(M - m) + sv[u];
+        M = m;
+      } else {
+        L += sv[u] * ex2(m - M);
+      }
     }
   }
   partM[((size_t)h * R2 + part) * b + i] = M;
@@ -360,19 +370,33 @@ __global__ void k_block_mass(const float *__restrict__ pm, const float *__restri
   }
   const float invL = 1.f / L;
   const int c0 = part * chunks_per_part, c1 = min(nch, c0 + chunks_per_part);
-  for (int ch = c0; ch < c1; ++ch) {
-    const size_t o = ((size_t)h * nch + ch) * b + i;
-    const float m = pm[o];
-    const float w = (m == -INFINITY) ? 0.f : ex2(m - M) * invL;
-    float a = plo[o] * w, c = phi[o] * w;
+  for (int ch = c0; ch < c1; ch += 4) {
+    float a[4], c[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const size_t o = ((size_t)h * nch + ch + u) * b + i;
+      const bool in = ch + u < c1;
+      const float m = in ? pm[o] : -INFINITY;
+      const float w = (m == -INFINITY) ? 0.f : ex2(m - M) * invL;
+      a[u] = in ? plo[o] * w : 0.f;
+      c[u] = in ? phi[o] * w : 0.f;
+    }
 #pragma unroll
     for (int s = 16; s > 0; s >>= 1) {
-      a += __shfl_xor_sync(0xffffffffu, a, s);
-      c += __shfl_xor_sync(0xffffffffu, c, s);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a[u] += __shfl_xor_sync(0xffffffffu, a[u], s);
+        c[u] += __shfl_xor_sync(0xffffffffu, c[u], s);
+      }
     }
     if (lane == 0) {
-      red[(warp * chunks_per_part + (ch - c0)) * 2 + 0] = a;
-      red[(warp * chunks_per_part + (ch - c0)) * 2 + 1] = c;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (ch + u < c1) {
+          red[(warp * chunks_per_part + (ch + u - c0)) * 2 + 0] = a[u];
+          red[(warp * chunks_per_part + (ch + u - c0)) * 2 + 1] = c[u];
+        }
+      }
     }
   }
   __syncthreads();
@@ -591,12 +615,17 @@ __global__ void __launch_bounds__(256)
 // of descending score (ties: lower index) while the kept sum is below gamma.
 // The cut is found by bisection on the fp32 bit pattern of the scores
 // (monotone for positive floats): T = largest t with
-// sum_{c < r, bits(w_c) >= t} w_c >= gamma - w_r; everything above T is kept,
-// then ties at T by ascending index until the sum reaches the target.
+// sum_{c < r, bits(w_c) >= t} w_c >= gamma - w_r, stopping as soon as one
+// candidate is left between the bounds; everything above T is kept, then ties
+// at T by ascending index until the target is reached.
 // Output: counts[h*n + r], ascending list at cols[h*n(n+1)/2 + r(r+1)/2].
 // ---------------------------------------------------------------------------
 constexpr int kSelRows = 16;
 constexpr int kSelMaxN = 1024;
+constexpr int kSelCols = 64;          // key blocks per logits step
+constexpr int kSelKStride = kSelCols + 4;
+// shared floats: scores [16][n] + qbar rows [16][128] + kbar^T [128][68]
+constexpr int kSelSmemFloats = kSelRows * kSelMaxN + kSelRows * 128 + 128 * kSelKStride;
 
 __global__ void __launch_bounds__(256)
     k_select(const int *__restrict__ pattern, const float *__restrict__ vhat,
@@ -605,42 +634,52 @@ __global__ void __launch_bounds__(256)
              int *__restrict__ counts, int *__restrict__ cols) {
   extern __shared__ float sh[];
   float *wbuf = sh;                              // [kSelRows][n]
-  float *qs = wbuf + kSelRows * n;               // [kSelRows][128]
-  float *ks = qs + kSelRows * 128;               // [32][129]
-  const int h = blockIdx.y, r0 = blockIdx.x * kSelRows;
+  float *qs = wbuf + kSelRows * n;               // [kSelRows][128]; VS: vhat[n], shat[n]
+  float *ks = qs + kSelRows * 128;               // [128][kSelKStride], kbar chunk transposed
+  // heaviest row groups (longest causal rows) first
+  const int h = blockIdx.y, r0 = (gridDim.x - 1 - blockIdx.x) * kSelRows;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rows = min(kSelRows, n - r0);
   const int pat = pattern[h];
   const int kvh = h / g;
-  const float *vh = vhat + (size_t)h * n;
-  const float *shh = shat + (size_t)h * n;
 
   if (pat == 1) {
-    // logits z[rr][c] = qbar_{r0+rr} . kbar_c / sqrt(d) for c <= r0+rows-1
-    for (int e = tid; e < rows * 128; e += blockDim.x)
-      qs[e] = qbar[((size_t)h * n + r0) * 128 + e];
+    // logits z[rr][c] = qbar_{r0+rr} . kbar_c / sqrt(d) for c < r0 + rows
+    for (int e = tid; e < rows * 128; e += blockDim.x) qs[e] = qbar[((size_t)h * n + r0) * 128 + e];
     const int cmax = r0 + rows;  // exclusive
-    for (int c0 = 0; c0 < cmax; c0 += 32) {
+    const int rr = tid >> 4, c4 = (tid & 15) * 4;   // thread: one row, four key blocks
+    for (int c0 = 0; c0 < cmax; c0 += kSelCols) {
       __syncthreads();
-      for (int e = tid; e < 32 * 128; e += blockDim.x) {
+      for (int e = tid; e < kSelCols * 128; e += blockDim.x) {
         const int cc = e >> 7, t = e & 127;
-        ks[cc * 129 + t] = (c0 + cc < cmax) ? kbar[((size_t)kvh * n + c0 + cc) * 128 + t] : 0.f;
+        ks[t * kSelKStride + cc] = (c0 + cc < cmax) ? kbar[((size_t)kvh * n + c0 + cc) * 128 + t] : 0.f;
       }
       __syncthreads();
-      // thread -> (rr = tid / 16, two columns cc = 2 * (tid % 16) + {0, 1})
-      const int rr = tid >> 4, cc = (tid & 15) * 2;
       if (rr < rows) {
-        float a0 = 0.f, a1 = 0.f;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
         const float *qr = qs + rr * 128;
 #pragma unroll 8
         for (int t = 0; t < 128; ++t) {
           const float qv = qr[t];
-          a0 = fmaf(qv, ks[cc * 129 + t], a0);
-          a1 = fmaf(qv, ks[(cc + 1) * 129 + t], a1);
+          const float4 kv = *reinterpret_cast<const float4 *>(ks + t * kSelKStride + c4);
+          a0 = fmaf(qv, kv.x, a0);
+          a1 = fmaf(qv, kv.y, a1);
+          a2 = fmaf(qv, kv.z, a2);
+          a3 = fmaf(qv, kv.w, a3);
         }
-        if (c0 + cc < cmax) wbuf[rr * n + c0 + cc] = a0 * inv_sqrt_d;
-        if (c0 + cc + 1 < cmax) wbuf[rr * n + c0 + cc + 1] = a1 * inv_sqrt_d;
+        const float av[4] = {a0, a1, a2, a3};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (c0 + c4 + i < cmax) wbuf[rr * n + c0 + c4 + i] = av[i] * inv_sqrt_d;
       }
+    }
+    __syncthreads();
+  } else {
+    // vertical / slash statistics of the head, staged once
+    float *v_s = qs, *s_s = qs + n;
+    for (int c = tid; c < n; c += blockDim.x) {
+      v_s[c] = vhat[(size_t)h * n + c];
+      s_s[c] = shat[(size_t)h * n + c];
     }
     __syncthreads();
   }
@@ -656,7 +695,8 @@ __global__ void __launch_bounds__(256)
       for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
       for (int c = lane; c <= r; c += 32) w[c] = expf(w[c] - mx);
     } else {
-      for (int c = lane; c <= r; c += 32) w[c] = vh[c] + shh[r - c];
+      const float *v_s = qs, *s_s = qs + n;
+      for (int c = lane; c <= r; c += 32) w[c] = v_s[c] + s_s[r - c];
     }
     float z = 0.f;
     for (int c = lane; c <= r; c += 32) z += w[c];
@@ -683,23 +723,52 @@ __global__ void __launch_bounds__(256)
         mode = 0;
       } else {
         mode = 2;
-        uint32_t lo = 0u, hi = 0x7F800000u;  // f(lo) >= need > f(hi) = 0
-        while (hi - lo > 1u) {
+        // invariant: f(lo) >= need > f(hi); c_lo, c_hi count the candidates
+        // with bits >= lo / >= hi; f_hi = f(hi)
+        uint32_t lo = 0u, hi = 0x7F800000u;
+        int c_lo = r, c_hi = 0;
+        float f_hi = 0.f;
+        while (hi - lo > 1u && c_lo - c_hi > 1) {
           const uint32_t mid = lo + ((hi - lo) >> 1);
           float f = 0.f;
-          for (int c = lane; c < r; c += 32) f += (__float_as_uint(w[c]) >= mid) ? w[c] : 0.f;
+          int cnt = 0;
+          for (int c = lane; c < r; c += 32) {
+            const bool ge = __float_as_uint(w[c]) >= mid;
+            f += ge ? w[c] : 0.f;
+            cnt += ge ? 1 : 0;
+          }
 #pragma unroll
-          for (int s = 16; s > 0; s >>= 1) f += __shfl_xor_sync(0xffffffffu, f, s);
-          if (f >= need) lo = mid; else hi = mid;
+          for (int s = 16; s > 0; s >>= 1) {
+            f += __shfl_xor_sync(0xffffffffu, f, s);
+            cnt += __shfl_xor_sync(0xffffffffu, cnt, s);
+          }
+          if (f >= need) {
+            lo = mid;
+            c_lo = cnt;
+          } else {
+            hi = mid;
+            c_hi = cnt;
+            f_hi = f;
+          }
         }
-        T = lo;
-        for (int c = lane; c < r; c += 32) s_gt += (__float_as_uint(w[c]) > T) ? w[c] : 0.f;
+        if (c_lo - c_hi == 1) {
+          // the one candidate in [lo, hi) is the cut value
+          uint32_t tb = 0u;
+          for (int c = lane; c < r; c += 32) {
+            const uint32_t bits = __float_as_uint(w[c]);
+            if (bits >= lo && bits < hi) tb = bits;
+          }
 #pragma unroll
-        for (int s = 16; s > 0; s >>= 1) s_gt += __shfl_xor_sync(0xffffffffu, s_gt, s);
+          for (int s = 16; s > 0; s >>= 1) tb = max(tb, __shfl_xor_sync(0xffffffffu, tb, s));
+          T = tb;
+        } else {
+          T = lo;
+        }
+        s_gt = f_hi;  // every candidate above T has bits >= hi
       }
     }
     // emit ascending, ties at T in index order until the target is reached
-    int* out = cols + (size_t)h * ((size_t)n * (n + 1) / 2) + (size_t)r * (r + 1) / 2;
+    int *out = cols + (size_t)h * ((size_t)n * (n + 1) / 2) + (size_t)r * (r + 1) / 2;
     int written = 0;
     float tie_acc = s_gt;
     const float tval = __uint_as_float(T);

@@ -52,6 +52,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking probe of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase of `bar` with the given parity.  Gives up (returns
 // false) when another role of the CTA has raised *abort, or after
 // `limit_ns`, in which case it raises *abort and records the timeout in the
@@ -255,6 +268,24 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA and integer pipes only (no MUFU), for x >= -125: Cody-Waite
+// style reduction x = n + f with n = rint(x), obtained by adding and
+// subtracting 1.5 * 2^23, f in [-1/2, 1/2]; 2^f from a degree-3 polynomial
+// fitted to 2^f on [-1/2, 1/2] (least squares reweighted towards minimax
+// relative error, 7.5e-5 at most in float32); 2^n added to the exponent field.
+constexpr float kEx2C0 = 0.9999280572f, kEx2C1 = 0.6932609677f, kEx2C2 = 0.2426111251f,
+                kEx2C3 = 0.0551716648f;
+__device__ __forceinline__ float ex2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float j = x + 12582912.f;
+  const float n = j - 12582912.f;
+  const float f = x - n;
+  float p = fmaf(kEx2C3, f, kEx2C2);
+  p = fmaf(p, f, kEx2C1);
+  p = fmaf(p, f, kEx2C0);
+  return __int_as_float(__float_as_int(p) + ((__float_as_int(j) - 0x4B400000) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

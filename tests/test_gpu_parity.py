@@ -107,15 +107,25 @@ def test_small_layers_full_parity(fp, w):
     check_tiles(P, exp, out, w, tiles)
 
 
-def test_gamma_one_matches_dense_sdpa(fp):
-    w = synth.Workload("dense", S=2048, Hq=8, Hkv=2, b=128, gamma=1.0, seed=13)
+DENSE = [synth.Workload("dense", S=2048, Hq=8, Hkv=2, b=128, gamma=1.0, seed=13),
+         synth.Workload("sweep_gen_b128", S=4096, Hq=32, Hkv=8, b=128, gamma=1.0, n_vertical=64, n_topics=32,
+                        seed=2),
+         synth.Workload("sweep_gen_b256", S=4096, Hq=32, Hkv=8, b=256, gamma=1.0, n_vertical=64, n_topics=32,
+                        seed=2)]
+
+
+@pytest.mark.parametrize("w", DENSE, ids=[w.name for w in DENSE])
+def test_gamma_one_matches_dense_sdpa(fp, w):
+    """gamma = 1 keeps every causal block: the output is dense causal attention
+    (checked against torch SDPA in fp32 on the GPU)."""
     x = synth.make_inputs(w)
     exp, out, idx = run_gpu(fp, x, w)
     n = w.S // w.b
+    g = w.Hq // w.Hkv
     assert exp["nnz"] == w.Hq * n * (n + 1) // 2
     q, k, v = (x[t].cuda().float() for t in ("q", "k", "v"))
     ref = torch.nn.functional.scaled_dot_product_attention(
-        q[None], k.repeat_interleave(4, 0)[None], v.repeat_interleave(4, 0)[None], is_causal=True)[0]
+        q[None], k.repeat_interleave(g, 0)[None], v.repeat_interleave(g, 0)[None], is_causal=True)[0]
     diff = (out.float() - ref).abs()
     assert float(diff.max()) <= parity.OUT_MAX_ABS and float(diff.mean()) <= parity.OUT_MEAN_ABS
 
