@@ -40,6 +40,7 @@ struct fp_index {
   int *pattern;            // [Hq]
   int *counts;             // [Hq][n]
   int *cols;               // [Hq][n(n+1)/2]
+  float *zlog;             // [Hq][n(n+1)/2] q-bar . k-bar logits (query-aware heads)
 };
 
 namespace {
@@ -127,9 +128,6 @@ int set_smem_attrs() {
   if (cudaFuncSetAttribute(k_sparse_attn<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            AttnCfg<I8>::kSmem) != cudaSuccess)
     return FP_ERR_CUDA;
-  if (cudaFuncSetAttribute(k_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSelSmemFloats * (int)sizeof(float)) != cudaSuccess)
-    return FP_ERR_CUDA;
   if (dev >= 0 && dev < 128) done[dev] = true;
   return FP_OK;
 }
@@ -180,9 +178,12 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   if ((rc = launch_status())) return rc;
   k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->b, I->n, I->qbar);
   if ((rc = launch_status())) return rc;
-  const size_t sel_bytes = (size_t)(kSelRows * I->n + kSelRows * 128 + 128 * kSelKStride) * sizeof(float);
-  k_select<<<dim3((I->n + kSelRows - 1) / kSelRows, I->Hq), 256, sel_bytes, st>>>(
-      I->pattern, I->vhat, I->shat, I->qbar, I->kbar, I->g, I->n, inv_sqrt_d, gamma, I->counts, I->cols);
+  const int nt = (I->n + kLgTile - 1) / kLgTile;
+  k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, I->qbar, I->kbar, I->g, I->n,
+                                                               inv_sqrt_d, I->zlog);
+  if ((rc = launch_status())) return rc;
+  k_cut<<<(I->Hq * I->n + 7) / 8, 256, 0, st>>>(I->pattern, I->vhat, I->shat, I->zlog, I->Hq, I->n, gamma,
+                                               I->counts, I->cols);
   return launch_status();
 }
 
@@ -242,6 +243,7 @@ int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out) {
   add((size_t)Hq * 4);
   add((size_t)Hq * n * 4);
   add((size_t)Hq * tri * 4);
+  add((size_t)Hq * tri * 4);
   if (cudaMalloc(&I->slab, need) != cudaSuccess) {
     free(I);
     return FP_ERR_CUDA;
@@ -265,6 +267,7 @@ int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out) {
   I->pattern = carve<int>(cur, (size_t)Hq);
   I->counts = carve<int>(cur, (size_t)Hq * n);
   I->cols = carve<int>(cur, (size_t)Hq * tri);
+  I->zlog = carve<float>(cur, (size_t)Hq * tri);
   *out = I;
   return FP_OK;
 }

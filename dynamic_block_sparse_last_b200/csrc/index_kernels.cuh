@@ -18,7 +18,8 @@
 //   k_kbar         block means of K.
 //   k_pattern      per head: vhat, shat, P_est, JSD, pattern.
 //   k_qbar         block means of Q for query-aware heads only.
-//   k_select       per (head, query block): scores, gamma cut, sorted list.
+//   k_qa_logits    q-bar . k-bar logits of query-aware heads (tiled fp32).
+//   k_cut          per (head, query block): scores, gamma cut, sorted list.
 #pragma once
 
 #include "ptx.cuh"
@@ -36,7 +37,8 @@ constexpr float kLog2e = 1.4426950408889634f;
 //   0..15  statistics: warpgroup t owns tile t; thread = one query row
 //   16     TMA producer     17  MMA issuer + TMEM owner
 //   18     K column sums for the block means (only CTAs of tile group 0)
-// TMEM: tile t's 128x128 fp32 score tile at columns [128t, 128t+128).
+// TMEM: tile t's 128x128 fp32 score tile at columns [128t, 128t+128), filled
+// and drained as two 64-key halves with their own barriers.
 // ---------------------------------------------------------------------------
 struct ScoreParams {
   int S, Hq, Hkv, b, n, nch, g;
@@ -66,8 +68,8 @@ __global__ void __launch_bounds__(608, 1)
                  ScoreParams P) {
   using C = ScoreCfg<I8>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_kfull[C::kStages], bar_kempty[C::kStages], bar_sfull[4],
-      bar_sfree[4];
+  __shared__ __align__(8) uint64_t bar_q, bar_kfull[C::kStages], bar_kempty[C::kStages], bar_sfull[4][2],
+      bar_sfree[4][2];
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -94,10 +96,11 @@ __global__ void __launch_bounds__(608, 1)
       mbar_init(smem_u32(&bar_kfull[s]), 1);
       mbar_init(smem_u32(&bar_kempty[s]), 1 + n_ksum_warps);
     }
-    for (int t = 0; t < 4; ++t) {
-      mbar_init(smem_u32(&bar_sfull[t]), 1);
-      mbar_init(smem_u32(&bar_sfree[t]), 4);
-    }
+    for (int t = 0; t < 4; ++t)
+      for (int hf = 0; hf < 2; ++hf) {
+        mbar_init(smem_u32(&bar_sfull[t][hf]), 1);
+        mbar_init(smem_u32(&bar_sfree[t][hf]), 4);
+      }
     fence_mbar_init();
   }
   if (warp == 17) {
@@ -144,34 +147,40 @@ __global__ void __launch_bounds__(608, 1)
     } else if (warp == 17) {
       // ------------------------------------------------------------ MMA issuer
       if (lane == 0) {
-        const uint32_t idesc = I8 ? idesc_i8(128, 128) : idesc_bf16(128, 128, 0);
+        // Each 128-key chunk is scored as two 64-key halves, all tiles' first
+        // halves before the second ones, so a statistics warpgroup works on
+        // one half while the tensor pipe fills the other.
+        const uint32_t idesc = I8 ? idesc_i8(128, 64) : idesc_bf16(128, 64, 0);
         bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, P.err);
         for (int u = 0; ok && u < U; ++u) {
           const int st = u % C::kStages;
           if (!mbar_wait(smem_u32(&bar_kfull[st]), (u / C::kStages) & 1, abort_flag, P.err)) break;
           const uint32_t kb = k_smem + st * C::kTileBytes;
-          for (int t = 0; t < T && ok; ++t) {
-            if (u > 0 && !mbar_wait(smem_u32(&bar_sfree[t]), (u - 1) & 1, abort_flag, P.err)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t qb = q_smem + t * C::kTileBytes;
-            const uint32_t d_tmem = tmem + t * 128;
-            if (I8) {
-#pragma unroll
-              for (int kk = 0; kk < 4; ++kk)
-                mma_i8_ss(d_tmem, umma_desc_sw128(qb + kk * 32, 16, 1024),
-                          umma_desc_sw128(kb + kk * 32, 16, 1024), idesc, kk > 0);
-            } else {
-#pragma unroll
-              for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(d_tmem, umma_desc_sw128(qb + off, 16, 1024),
-                            umma_desc_sw128(kb + off, 16, 1024), idesc, kk > 0);
+          for (int hf = 0; hf < 2 && ok; ++hf) {
+            for (int t = 0; t < T; ++t) {
+              if (u > 0 && !mbar_wait(smem_u32(&bar_sfree[t][hf]), (u - 1) & 1, abort_flag, P.err)) {
+                ok = false;
+                break;
               }
+              tc_fence_after();
+              const uint32_t qb = q_smem + t * C::kTileBytes;
+              const uint32_t d_tmem = tmem + t * 128 + hf * 64;
+              const uint32_t kh = kb + hf * 8192;  // key rows 64*hf .. 64*hf+63
+              if (I8) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                  mma_i8_ss(d_tmem, umma_desc_sw128(qb + kk * 32, 16, 1024),
+                            umma_desc_sw128(kh + kk * 32, 16, 1024), idesc, kk > 0);
+              } else {
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                  const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                  mma_bf16_ss(d_tmem, umma_desc_sw128(qb + off, 16, 1024),
+                              umma_desc_sw128(kh + off, 16, 1024), idesc, kk > 0);
+                }
+              }
+              tc_commit(smem_u32(&bar_sfull[t][hf]));
             }
-            tc_commit(smem_u32(&bar_sfull[t]));
           }
           if (!ok) break;
           tc_commit(smem_u32(&bar_kempty[st]));
@@ -234,68 +243,78 @@ __global__ void __launch_bounds__(608, 1)
         float scale2 = P.scale2;
         if (I8) scale2 *= P.q_scale[hh] * P.k_scale[kvh];
         const uint32_t taddr = tmem + t * 128 + (((warp & 3) * 32) << 16);
-        for (int u = 0; u < U; ++u) {
-          if (!mbar_wait(smem_u32(&bar_sfull[t]), u & 1, abort_flag, P.err)) break;
-          tc_fence_after();
+        bool ok = true;
+        for (int u = 0; u < U && ok; ++u) {
           const int ch = ch0 + u;
           const int tb = (ch * 128) % P.b;                 // chunk offset inside its block
           const bool last_block = (ch * 128) / P.b == P.n - 1;
-          // pass 1: row max over the causal columns t <= i of the last block
-          // (four independent max chains)
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-          for (int qq = 0; qq < 4; ++qq) {
-            uint32_t r[32];
-            tmem_ld32(taddr + qq * 32, r);
-            tmem_ld_wait(r);
-            const int t0 = tb + qq * 32;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
-              const bool valid = !last_block || (t0 + e <= i);
-              m4[e & 3] = valid ? fmaxf(m4[e & 3], s) : m4[e & 3];
-            }
-          }
-          const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          // One pass over the chunk in 32-column pieces with an online max:
+          // lo/hi are kept relative to the running max m and rescaled when a
+          // piece raises it.  Columns t <= i (block-relative) go to lo, the
+          // rest to hi; in the last block columns t > i are causally masked.
+          float m = -INFINITY;
           float lo4[4] = {0.f, 0.f, 0.f, 0.f}, hi4[4] = {0.f, 0.f, 0.f, 0.f};
-          const float m2 = mx * scale2;
-          if (mx != -INFINITY) {
+          for (int hf = 0; hf < 2; ++hf) {
+            if (!mbar_wait(smem_u32(&bar_sfull[t][hf]), u & 1, abort_flag, P.err)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll 1
-            for (int qq = 0; qq < 4; ++qq) {
+            for (int qq = 0; qq < 2; ++qq) {
               uint32_t r[32];
-              tmem_ld32(taddr + qq * 32, r);
+              tmem_ld32(taddr + hf * 64 + qq * 32, r);
               tmem_ld_wait(r);
-              const int dlt = i - (tb + qq * 32);   // columns e <= dlt are on the lo side
+              const int t0 = tb + hf * 64 + qq * 32;
+              const int dlt = i - t0;  // columns e <= dlt are on the lo side
+              float pm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+                const bool valid = !last_block || (e <= dlt);
+                pm4[e & 3] = valid ? fmaxf(pm4[e & 3], s) : pm4[e & 3];
+              }
+              const float pmx = fmaxf(fmaxf(pm4[0], pm4[1]), fmaxf(pm4[2], pm4[3]));
+              if (pmx == -INFINITY) continue;  // whole piece masked
+              if (pmx > m) {
+                const float f = (m == -INFINITY) ? 0.f : ex2((m - pmx) * scale2);
+#pragma unroll
+                for (int w4 = 0; w4 < 4; ++w4) {
+                  lo4[w4] *= f;
+                  hi4[w4] *= f;
+                }
+                m = pmx;
+              }
+              const float m2p = m * scale2;
               if (dlt >= 31) {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                   const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
-                  lo4[e & 3] += ex2(fmaf(s, scale2, -m2));
+                  lo4[e & 3] += ex2(fmaf(s, scale2, -m2p));
                 }
               } else if (dlt < 0) {
                 if (!last_block) {
 #pragma unroll
                   for (int e = 0; e < 32; ++e) {
                     const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
-                    hi4[e & 3] += ex2(fmaf(s, scale2, -m2));
+                    hi4[e & 3] += ex2(fmaf(s, scale2, -m2p));
                   }
                 }
               } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                   const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
-                  const float p = ex2(fmaf(s, scale2, -m2));
+                  const float p = ex2(fmaf(s, scale2, -m2p));
                   if (e <= dlt) lo4[e & 3] += p;
                   else if (!last_block) hi4[e & 3] += p;
                 }
               }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&bar_sfree[t][hf]));
           }
+          if (!ok) break;
+          const float m2 = m * scale2;
           const float lo = (lo4[0] + lo4[1]) + (lo4[2] + lo4[3]);
           const float hi = (hi4[0] + hi4[1]) + (hi4[2] + hi4[3]);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&bar_sfree[t]));
           const size_t o = ((size_t)hh * P.nch + ch) * P.b + i;
           P.pm[o] = m2;
           P.plo[o] = lo;
@@ -608,201 +627,255 @@ __global__ void __launch_bounds__(256)
 }
 
 // ---------------------------------------------------------------------------
-// k_select: grid (ceil(n / 16), Hq), block 256 (8 warps, 2 query blocks per
-// warp).  Scores of query block r over c <= r:
-//   VS: w_c = vhat[c] + shat[r - c];   QA: w_c = exp(qbar_r . kbar_c / sqrt(d) - max)
-// normalised to sum 1.  The diagonal is kept; the others are kept in order
-// of descending score (ties: lower index) while the kept sum is below gamma.
-// The cut is found by bisection on the fp32 bit pattern of the scores
-// (monotone for positive floats): T = largest t with
-// sum_{c < r, bits(w_c) >= t} w_c >= gamma - w_r, stopping as soon as one
-// candidate is left between the bounds; everything above T is kept, then ties
-// at T by ascending index until the target is reached.
-// Output: counts[h*n + r], ascending list at cols[h*n(n+1)/2 + r(r+1)/2].
+// k_qa_logits: grid (nt(nt+1)/2, Hq) with nt = ceil(n/64), block 256.  For
+// query-aware heads only (others exit): the lower triangle of
+// Z = qbar kbar^T / sqrt(d), z[h][r][c] for c <= r, in the padded triangular
+// layout (row r at h*n(n+1)/2 + r(r+1)/2).  Tiled fp32 product: 64 x 64
+// output tile per CTA, 4 x 4 outputs per thread, d staged through shared
+// memory 32 at a time.
 // ---------------------------------------------------------------------------
-constexpr int kSelRows = 16;
-constexpr int kSelMaxN = 1024;
-constexpr int kSelCols = 64;          // key blocks per logits step
-constexpr int kSelKStride = kSelCols + 4;
-// shared floats: scores [16][n] + qbar rows [16][128] + kbar^T [128][68]
-constexpr int kSelSmemFloats = kSelRows * kSelMaxN + kSelRows * 128 + 128 * kSelKStride;
+constexpr int kLgTile = 64;
+constexpr int kLgK = 32;
+constexpr int kLgStride = kLgTile + 4;  // float4-aligned rows
 
 __global__ void __launch_bounds__(256)
-    k_select(const int *__restrict__ pattern, const float *__restrict__ vhat,
-             const float *__restrict__ shat, const float *__restrict__ qbar,
-             const float *__restrict__ kbar, int g, int n, float inv_sqrt_d, float gamma,
-             int *__restrict__ counts, int *__restrict__ cols) {
-  extern __shared__ float sh[];
-  float *wbuf = sh;                              // [kSelRows][n]
-  float *qs = wbuf + kSelRows * n;               // [kSelRows][128]; VS: vhat[n], shat[n]
-  float *ks = qs + kSelRows * 128;               // [128][kSelKStride], kbar chunk transposed
-  // heaviest row groups (longest causal rows) first
-  const int h = blockIdx.y, r0 = (gridDim.x - 1 - blockIdx.x) * kSelRows;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rows = min(kSelRows, n - r0);
-  const int pat = pattern[h];
+    k_qa_logits(const int *__restrict__ pattern, const float *__restrict__ qbar,
+                const float *__restrict__ kbar, int g, int n, float inv_sqrt_d, float *__restrict__ z) {
+  const int h = blockIdx.y;
+  if (pattern[h] != 1) return;
+  __shared__ __align__(16) float As[kLgK][kLgStride];  // [k][row]
+  __shared__ __align__(16) float Bs[kLgK][kLgStride];  // [k][col]
+  // lower-triangular tile (tr, tc), tc <= tr, from the linear index
+  const int x = blockIdx.x;
+  int tr = (int)((sqrtf(8.f * (float)x + 1.f) - 1.f) * 0.5f);
+  while ((tr + 1) * (tr + 2) / 2 <= x) ++tr;
+  while (tr * (tr + 1) / 2 > x) --tr;
+  const int tc = x - tr * (tr + 1) / 2;
   const int kvh = h / g;
-
-  if (pat == 1) {
-    // logits z[rr][c] = qbar_{r0+rr} . kbar_c / sqrt(d) for c < r0 + rows
-    for (int e = tid; e < rows * 128; e += blockDim.x) qs[e] = qbar[((size_t)h * n + r0) * 128 + e];
-    const int cmax = r0 + rows;  // exclusive
-    const int rr = tid >> 4, c4 = (tid & 15) * 4;   // thread: one row, four key blocks
-    for (int c0 = 0; c0 < cmax; c0 += kSelCols) {
-      __syncthreads();
-      for (int e = tid; e < kSelCols * 128; e += blockDim.x) {
-        const int cc = e >> 7, t = e & 127;
-        ks[t * kSelKStride + cc] = (c0 + cc < cmax) ? kbar[((size_t)kvh * n + c0 + cc) * 128 + t] : 0.f;
-      }
-      __syncthreads();
-      if (rr < rows) {
-        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
-        const float *qr = qs + rr * 128;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int row0 = tr * kLgTile, col0 = tc * kLgTile;
+  const float *qh = qbar + (size_t)h * n * 128;
+  const float *kh = kbar + (size_t)kvh * n * 128;
+  float acc[4][4];
+#pragma unroll
+  for (int a = 0; a < 4; ++a)
+#pragma unroll
+    for (int b2 = 0; b2 < 4; ++b2) acc[a][b2] = 0.f;
+  for (int k0 = 0; k0 < 128; k0 += kLgK) {
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int f = tid + u * 256, rr = f >> 3, k4 = (f & 7) * 4;
+      const float4 qa = (row0 + rr < n) ? *reinterpret_cast<const float4 *>(qh + (size_t)(row0 + rr) * 128 + k0 + k4)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 kb = (col0 + rr < n) ? *reinterpret_cast<const float4 *>(kh + (size_t)(col0 + rr) * 128 + k0 + k4)
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+      As[k4 + 0][rr] = qa.x; As[k4 + 1][rr] = qa.y; As[k4 + 2][rr] = qa.z; As[k4 + 3][rr] = qa.w;
+      Bs[k4 + 0][rr] = kb.x; Bs[k4 + 1][rr] = kb.y; Bs[k4 + 2][rr] = kb.z; Bs[k4 + 3][rr] = kb.w;
+    }
+    __syncthreads();
 #pragma unroll 8
-        for (int t = 0; t < 128; ++t) {
-          const float qv = qr[t];
-          const float4 kv = *reinterpret_cast<const float4 *>(ks + t * kSelKStride + c4);
-          a0 = fmaf(qv, kv.x, a0);
-          a1 = fmaf(qv, kv.y, a1);
-          a2 = fmaf(qv, kv.z, a2);
-          a3 = fmaf(qv, kv.w, a3);
-        }
-        const float av[4] = {a0, a1, a2, a3};
+    for (int k = 0; k < kLgK; ++k) {
+      const float4 a4 = *reinterpret_cast<const float4 *>(&As[k][ty * 4]);
+      const float4 b4 = *reinterpret_cast<const float4 *>(&Bs[k][tx * 4]);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (c0 + c4 + i < cmax) wbuf[rr * n + c0 + c4 + i] = av[i] * inv_sqrt_d;
-      }
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b2 = 0; b2 < 4; ++b2) acc[a][b2] = fmaf(av[a], bv[b2], acc[a][b2]);
     }
-    __syncthreads();
-  } else {
-    // vertical / slash statistics of the head, staged once
-    float *v_s = qs, *s_s = qs + n;
-    for (int c = tid; c < n; c += blockDim.x) {
-      v_s[c] = vhat[(size_t)h * n + c];
-      s_s[c] = shat[(size_t)h * n + c];
-    }
-    __syncthreads();
   }
+  float *zh = z + (size_t)h * ((size_t)n * (n + 1) / 2);
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int r = row0 + ty * 4 + a;
+    if (r >= n) continue;
+#pragma unroll
+    for (int b2 = 0; b2 < 4; ++b2) {
+      const int c = col0 + tx * 4 + b2;
+      if (c <= r) zh[(size_t)r * (r + 1) / 2 + c] = acc[a][b2] * inv_sqrt_d;
+    }
+  }
+}
 
-  for (int rr = warp; rr < rows; rr += 8) {
-    const int r = r0 + rr;
-    float *w = wbuf + rr * n;
-    // raw scores
-    if (pat == 1) {
-      float mx = -INFINITY;
-      for (int c = lane; c <= r; c += 32) mx = fmaxf(mx, w[c]);
+// ---------------------------------------------------------------------------
+// k_cut: one warp per (head, query block r), heavy rows first; block 256.
+// Scores over c <= r:  VS: w_c = vhat[c] + shat[r - c];  QA: w_c = exp(z_c -
+// max); normalised to sum 1.  The diagonal is kept; the others are kept in
+// order of descending score (ties: lower index) while the kept sum is below
+// gamma.  The cut is found by bisection on the fp32 bit pattern of the
+// scores (monotone for positive floats): T = largest t with
+// sum_{c < r, bits(w_c) >= t} w_c >= gamma - w_r, stopping as soon as one
+// candidate is left between the bounds; everything above T is kept, then
+// ties at T by ascending index until the target is reached.  The row lives
+// in registers (element c in lane c % 32, slot c / 32).
+// Output: counts[h*n + r], ascending list at cols[h*n(n+1)/2 + r(r+1)/2].
+// ---------------------------------------------------------------------------
+constexpr int kSelMaxN = 1024;
+
+template <int NL>
+__device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const float *__restrict__ vhat,
+                                        const float *__restrict__ shat, const float *__restrict__ zrow,
+                                        float gamma, int *__restrict__ out, int *__restrict__ count_out) {
+  const int lane = threadIdx.x & 31;
+  float v[NL];
+  if (pat == 1) {
+    float mx = -INFINITY;
 #pragma unroll
-      for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
-      for (int c = lane; c <= r; c += 32) w[c] = expf(w[c] - mx);
-    } else {
-      const float *v_s = qs, *s_s = qs + n;
-      for (int c = lane; c <= r; c += 32) w[c] = v_s[c] + s_s[r - c];
+    for (int i = 0; i < NL; ++i) {
+      const int c = lane + 32 * i;
+      float val = -INFINITY;
+      if (c <= r) val = zrow[c];
+      v[i] = val;
+      mx = fmaxf(mx, val);
     }
-    float z = 0.f;
-    for (int c = lane; c <= r; c += 32) z += w[c];
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1) z += __shfl_xor_sync(0xffffffffu, z, s);
-    for (int c = lane; c <= r; c += 32) w[c] = w[c] / z;
-    __syncwarp();
-    const float wr = w[r];
-    const float need = gamma - wr;
-    // selection mode: 0 = all, 1 = diagonal only, 2 = cut at threshold T
-    int mode;
-    uint32_t T = 0;
-    float s_gt = 0.f;
-    if (gamma >= 1.f) {
-      mode = 0;
-    } else if (need <= 0.f) {
-      mode = 1;
-    } else {
-      float tot = 0.f;
-      for (int c = lane; c < r; c += 32) tot += w[c];
+    for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
 #pragma unroll
-      for (int s = 16; s > 0; s >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, s);
-      if (tot < need) {
-        mode = 0;
-      } else {
-        mode = 2;
-        // invariant: f(lo) >= need > f(hi); c_lo, c_hi count the candidates
-        // with bits >= lo / >= hi; f_hi = f(hi)
-        uint32_t lo = 0u, hi = 0x7F800000u;
-        int c_lo = r, c_hi = 0;
-        float f_hi = 0.f;
-        while (hi - lo > 1u && c_lo - c_hi > 1) {
-          const uint32_t mid = lo + ((hi - lo) >> 1);
-          float f = 0.f;
-          int cnt = 0;
-          for (int c = lane; c < r; c += 32) {
-            const bool ge = __float_as_uint(w[c]) >= mid;
-            f += ge ? w[c] : 0.f;
-            cnt += ge ? 1 : 0;
-          }
+    for (int i = 0; i < NL; ++i) v[i] = (lane + 32 * i <= r) ? expf(v[i] - mx) : 0.f;
+  } else {
+    const float *vh = vhat + (size_t)h * n, *sh = shat + (size_t)h * n;
 #pragma unroll
-          for (int s = 16; s > 0; s >>= 1) {
-            f += __shfl_xor_sync(0xffffffffu, f, s);
-            cnt += __shfl_xor_sync(0xffffffffu, cnt, s);
-          }
-          if (f >= need) {
-            lo = mid;
-            c_lo = cnt;
-          } else {
-            hi = mid;
-            c_hi = cnt;
-            f_hi = f;
-          }
-        }
-        if (c_lo - c_hi == 1) {
-          // the one candidate in [lo, hi) is the cut value
-          uint32_t tb = 0u;
-          for (int c = lane; c < r; c += 32) {
-            const uint32_t bits = __float_as_uint(w[c]);
-            if (bits >= lo && bits < hi) tb = bits;
-          }
-#pragma unroll
-          for (int s = 16; s > 0; s >>= 1) tb = max(tb, __shfl_xor_sync(0xffffffffu, tb, s));
-          T = tb;
-        } else {
-          T = lo;
-        }
-        s_gt = f_hi;  // every candidate above T has bits >= hi
-      }
+    for (int i = 0; i < NL; ++i) {
+      const int c = lane + 32 * i;
+      float val = 0.f;
+      if (c <= r) val = vh[c] + sh[r - c];
+      v[i] = val;
     }
-    // emit ascending, ties at T in index order until the target is reached
-    int *out = cols + (size_t)h * ((size_t)n * (n + 1) / 2) + (size_t)r * (r + 1) / 2;
-    int written = 0;
-    float tie_acc = s_gt;
-    const float tval = __uint_as_float(T);
-    bool ties_done = false;
-    for (int c0 = 0; c0 <= r; c0 += 32) {
-      const int c = c0 + lane;
-      bool keep = false;
-      bool is_tie = false;
-      if (c <= r) {
-        if (mode == 0 || c == r) keep = true;
-        else if (mode == 2) {
-          const uint32_t bits = __float_as_uint(w[c]);
-          keep = bits > T;
-          is_tie = (bits == T);
-        }
-      }
-      if (mode == 2) {
-        uint32_t tmask = __ballot_sync(0xffffffffu, is_tie);
-        uint32_t take = 0u;
-        while (tmask && !ties_done) {
-          if (tie_acc >= need) { ties_done = true; break; }
-          const int bpos = __ffs(tmask) - 1;
-          take |= 1u << bpos;
-          tie_acc += tval;
-          tmask &= tmask - 1u;
-        }
-        if (take & (1u << lane)) keep = true;
-      }
-      const uint32_t km = __ballot_sync(0xffffffffu, keep);
-      if (keep) out[written + __popc(km & ((1u << lane) - 1u))] = c;
-      written += __popc(km);
-    }
-    if (lane == 0) counts[(size_t)h * n + r] = written;
   }
+  float zs = 0.f;
+#pragma unroll
+  for (int i = 0; i < NL; ++i) zs += v[i];
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, s);
+#pragma unroll
+  for (int i = 0; i < NL; ++i) v[i] = v[i] / zs;
+  // diagonal score w_r from lane r % 32, slot r / 32
+  float wr_l = 0.f;
+#pragma unroll
+  for (int i = 0; i < NL; ++i)
+    if (i == (r >> 5)) wr_l = v[i];
+  const float wr = __shfl_sync(0xffffffffu, wr_l, r & 31);
+  const float need = gamma - wr;
+  // candidates: c < r (slot value 0 and bits 0 elsewhere never qualify)
+  int mode;  // 0 = all, 1 = diagonal only, 2 = cut at T
+  uint32_t T = 0;
+  float s_gt = 0.f;
+  if (gamma >= 1.f) {
+    mode = 0;
+  } else if (need <= 0.f) {
+    mode = 1;
+  } else {
+    float tot = 0.f;
+#pragma unroll
+    for (int i = 0; i < NL; ++i) tot += (lane + 32 * i < r) ? v[i] : 0.f;
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, s);
+    if (tot < need) {
+      mode = 0;
+    } else {
+      mode = 2;
+      // invariant: f(lo) >= need > f(hi); c_lo / c_hi count candidates with
+      // bits >= lo / >= hi; f_hi = f(hi)
+      uint32_t lo = 0u, hi = 0x7F800000u;
+      int c_lo = r, c_hi = 0;
+      float f_hi = 0.f;
+      while (hi - lo > 1u && c_lo - c_hi > 1) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        float f = 0.f;
+        int cnt = 0;
+#pragma unroll
+        for (int i = 0; i < NL; ++i) {
+          const bool ge = (lane + 32 * i < r) && __float_as_uint(v[i]) >= mid;
+          f += ge ? v[i] : 0.f;
+          cnt += ge ? 1 : 0;
+        }
+#pragma unroll
+        for (int s = 16; s > 0; s >>= 1) {
+          f += __shfl_xor_sync(0xffffffffu, f, s);
+          cnt += __shfl_xor_sync(0xffffffffu, cnt, s);
+        }
+        if (f >= need) {
+          lo = mid;
+          c_lo = cnt;
+        } else {
+          hi = mid;
+          c_hi = cnt;
+          f_hi = f;
+        }
+      }
+      if (c_lo - c_hi == 1) {
+        uint32_t tb = 0u;
+#pragma unroll
+        for (int i = 0; i < NL; ++i) {
+          const uint32_t bits = __float_as_uint(v[i]);
+          if (lane + 32 * i < r && bits >= lo && bits < hi) tb = bits;
+        }
+#pragma unroll
+        for (int s = 16; s > 0; s >>= 1) tb = max(tb, __shfl_xor_sync(0xffffffffu, tb, s));
+        T = tb;
+      } else {
+        T = lo;
+      }
+      s_gt = f_hi;  // every candidate above T has bits >= hi
+    }
+  }
+  // emit ascending; ties at T in index order until the target is reached
+  int written = 0;
+  float tie_acc = s_gt;
+  const float tval = __uint_as_float(T);
+  bool ties_done = false;
+#pragma unroll
+  for (int i = 0; i < NL; ++i) {
+    const int c = lane + 32 * i;
+    bool keep = false, is_tie = false;
+    if (c <= r) {
+      if (mode == 0 || c == r) keep = true;
+      else if (mode == 2) {
+        const uint32_t bits = __float_as_uint(v[i]);
+        keep = bits > T;
+        is_tie = (bits == T);
+      }
+    }
+    if (mode == 2) {
+      uint32_t tmask = __ballot_sync(0xffffffffu, is_tie);
+      uint32_t take = 0u;
+      while (tmask && !ties_done) {
+        if (tie_acc >= need) {
+          ties_done = true;
+          break;
+        }
+        take |= 1u << (__ffs(tmask) - 1);
+        tie_acc += tval;
+        tmask &= tmask - 1u;
+      }
+      if (take & (1u << lane)) keep = true;
+    }
+    const uint32_t km = __ballot_sync(0xffffffffu, keep);
+    if (keep) out[written + __popc(km & ((1u << lane) - 1u))] = c;
+    written += __popc(km);
+  }
+  if (lane == 0) *count_out = written;
+}
+
+__global__ void __launch_bounds__(256)
+    k_cut(const int *__restrict__ pattern, const float *__restrict__ vhat, const float *__restrict__ shat,
+          const float *__restrict__ z, int Hq, int n, float gamma, int *__restrict__ counts,
+          int *__restrict__ cols) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= Hq * n) return;
+  const int r = n - 1 - row / Hq, h = row % Hq;  // longest rows first
+  const size_t tri = (size_t)n * (n + 1) / 2, off = (size_t)h * tri + (size_t)r * (r + 1) / 2;
+  const int pat = pattern[h];
+  const float *zrow = z + off;
+  int *out = cols + off, *cnt = counts + (size_t)h * n + r;
+  const int nl = (r >> 5) + 1;  // elements per lane
+  if (nl <= 1) cut_row<1>(pat, h, r, n, vhat, shat, zrow, gamma, out, cnt);
+  else if (nl <= 2) cut_row<2>(pat, h, r, n, vhat, shat, zrow, gamma, out, cnt);
+  else if (nl <= 4) cut_row<4>(pat, h, r, n, vhat, shat, zrow, gamma, out, cnt);
+  else if (nl <= 8) cut_row<8>(pat, h, r, n, vhat, shat, zrow, gamma, out, cnt);
+  else if (nl <= 16) cut_row<16>(pat, h, r, n, vhat, shat, zrow, gamma, out, cnt);
+  else cut_row<32>(pat, h, r, n, vhat, shat, zrow, gamma, out, cnt);
 }
 
 }  // namespace fpk
