@@ -124,6 +124,17 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Maximum of a per-rank number over all ranks (identity without a
+    process group): every multi-rank time is the slowest rank's."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def make_line(args, w, value, ms_per_step, extra):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -269,10 +280,7 @@ def run_ours(args, w):
     index_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
     attn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
     assert fp.fp_get_device_error(stream) == fp.FP_OK
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     ms_per_step = total_ms / args.steps
     dense = synth.dense_equiv_flops(w.S, w.Hq, w.d)
     value = world * dense * args.steps / (total_ms / 1e3) / 1e12
@@ -298,10 +306,7 @@ def run_ours(args, w):
         e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = h_q.numel() * h_q.element_size() + h_k.numel() * h_k.element_size() + h_v.numel() * h_v.element_size()
     d2h = h_out.numel() * h_out.element_size()
     e2e = {"value": world * dense / (e2e_ms / 1e3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,

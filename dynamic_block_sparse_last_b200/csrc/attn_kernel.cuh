@@ -14,12 +14,13 @@
 // chunks); a chunk only one tile needs is computed for that tile only.
 // CTAs are numbered heavy first (descending query position).
 //
-// Warp roles (352 threads):
-//   warps 0-3 / 4-7  softmax, correction and epilogue of tile 0 / tile 1;
-//                    thread = one query row = one TMEM lane
-//   warp 8           TMA producer: Q tiles once, then K chunks (3-stage ring)
-//   warp 9           TMEM owner and MMA issuer (one thread)
-//   warp 10          TMA producer of V chunks (2-stage ring)
+// Warp roles (608 threads):
+//   warps 0-7 / 8-15 softmax, correction and epilogue of tile 0 / tile 1:
+//                    two warps per 32-row TMEM lane group, each taking half
+//                    of the 128 keys of a chunk and half of the O columns
+//   warp 16          TMA producer: Q tiles once, then K chunks (2-stage ring)
+//   warp 17          TMEM owner and MMA issuer (one thread)
+//   warp 18          TMA producer of V chunks (2-stage ring)
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // The softmax writes P (bf16, two per column) over the first 64 columns of
 // its S tile and the P.V product reads it from TMEM (tcgen05.mma A operand
@@ -50,12 +51,12 @@ template <bool I8>
 struct AttnCfg {
   static constexpr int kQKTile = I8 ? 16384 : 32768;   // 128 rows x 128 elements
   static constexpr int kVTile = 32768;
-  static constexpr int kKStages = 3, kVStages = 2;
+  static constexpr int kKStages = 2, kVStages = 2;
   static constexpr int kQOff = 0;                                 // two Q tiles
   static constexpr int kKOff = kQOff + 2 * kQKTile;               // K ring
   static constexpr int kVOff = kKOff + kKStages * kQKTile;        // V ring
   static constexpr int kSmem = kVOff + kVStages * kVTile + 1024;
-  static constexpr int kThreads = 352;
+  static constexpr int kThreads = 608;
   // Every kExpFmaEvery-th exponential of an off-diagonal chunk runs on the
   // FMA pipe (ex2_fma) instead of MUFU; 0 keeps all on MUFU.  A share of 1/4
   // measured no faster on the 128K layer (power-capped clocks), so it is off.
@@ -162,13 +163,15 @@ struct UnionWalk {
 };
 
 template <bool I8>
-__global__ void __launch_bounds__(352, 1)
+__global__ void __launch_bounds__(608, 1)
     k_sparse_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, AttnParams P) {
   using C = AttnCfg<I8>;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_q, bar_kfull[3], bar_kempty[3], bar_vfull[2], bar_vempty[2],
-      bar_sfull[2], bar_pfull[2], bar_odone[2];
+  __shared__ __align__(8) uint64_t bar_q, bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2],
+      bar_sfull[2], bar_pfull[2], bar_odone[2], bar_xchg[2][4];
+  __shared__ float xmax[2][2][2][128];  // [chunk parity][tile][column half][row]
+  __shared__ float xl[2][2][128];       // [tile][column half][row]
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ uint32_t chunk_bm[2][kMaxChunkWords];
@@ -186,27 +189,29 @@ __global__ void __launch_bounds__(352, 1)
   if (threadIdx.x == 0) {
     abort_sh = 0;
     mbar_init(smem_u32(&bar_q), 1);
-    for (int s = 0; s < 3; ++s) {
+    for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bar_kfull[s]), 1);
       mbar_init(smem_u32(&bar_kempty[s]), 1);
     }
+    for (int t = 0; t < 2; ++t)
+      for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&bar_xchg[t][q]), 2);
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bar_vfull[s]), 1);
       mbar_init(smem_u32(&bar_vempty[s]), 1);
       mbar_init(smem_u32(&bar_sfull[s]), 1);
-      mbar_init(smem_u32(&bar_pfull[s]), 4);
+      mbar_init(smem_u32(&bar_pfull[s]), 8);
       mbar_init(smem_u32(&bar_odone[s]), 1);
     }
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < 2 * kMaxChunkWords; i += blockDim.x) (&chunk_bm[0][0])[i] = 0u;
-  if (warp == 9) {
+  if (warp == 17) {
     tmem_alloc(smem_u32(&tmem_base_sh), 512);
     tmem_relinquish();
   }
   __syncthreads();
-  if (warp == 8 || warp == 9) {
-    const int lane64 = threadIdx.x - 256;
+  if (warp == 16 || warp == 17) {
+    const int lane64 = threadIdx.x - 512;
     build_chunk_bitmap(tl[0], per, chunk_bm[0], lane64);
     build_chunk_bitmap(tl[1], per, chunk_bm[1], lane64);
   }
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(352, 1)
   const uint32_t tmem = tmem_base_sh;
   volatile int *abort_flag = &abort_sh;
 
-  if (warp == 8) {
+  if (warp == 16) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_map(&tm_q);
@@ -229,7 +234,7 @@ __global__ void __launch_bounds__(352, 1)
         tma_load_2d(dst, &tm_q, 0, qrow, smem_u32(&bar_q));
         if (!I8) tma_load_2d(dst + 16384, &tm_q, 64, qrow, smem_u32(&bar_q));
       }
-      // K runs up to three chunks ahead of the MMA issuer; V (warp 10) has
+      // K runs up to two chunks ahead of the MMA issuer; V (warp 18) has
       // its own ring and producer, so neither waits on the other's slots.
       UnionWalk wk;
       wk.init(chunk_bm[0], chunk_bm[1], words);
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(352, 1)
         if (!I8) tma_load_2d(sk + st * C::kQKTile + 16384, &tm_k, 64, krow, smem_u32(&bar_kfull[st]));
       }
     }
-  } else if (warp == 10) {
+  } else if (warp == 18) {
     // ---------------------------------------------------------------- V producer
     if (lane == 0) {
       tma_prefetch_map(&tm_v);
@@ -261,7 +266,7 @@ __global__ void __launch_bounds__(352, 1)
         tma_load_2d(sv + st * C::kVTile + 16384, &tm_v, 64, vrow, smem_u32(&bar_vfull[st]));
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == 17) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       const uint32_t id_qk = I8 ? idesc_i8(128, 128) : idesc_bf16(128, 128, 0);
@@ -330,11 +335,19 @@ __global__ void __launch_bounds__(352, 1)
     }
   } else {
     // ---------------------------------------------------------------- softmax
-    const int t = warp >> 2;
+    // Two warps share each 32-row group of a tile: warp half ch owns keys
+    // 64ch .. 64ch+63 of every S chunk and O columns 64ch .. 64ch+63.  They
+    // exchange their partial row maxima once per chunk through shared memory
+    // (an mbarrier of count 2, waited with the usual time limit) and keep
+    // partial row sums against the same reference max, added at the end.
+    const int t = warp >> 3, ch = (warp >> 2) & 1, lq = warp & 3;
     const AttnTile &me = tl[t];
-    const int row = (warp & 3) * 32 + lane;
-    const uint32_t lane_off = ((uint32_t)((warp & 3) * 32)) << 16;
-    const uint32_t s_tm = tmem + t * 128 + lane_off, o_tm = tmem + 256 + t * 128 + lane_off;
+    const int row = lq * 32 + lane;
+    const uint32_t lane_off = ((uint32_t)(lq * 32)) << 16;
+    const uint32_t s_tm = tmem + t * 128 + ch * 64 + lane_off;    // this warp's S columns
+    const uint32_t p_tm = tmem + t * 128 + ch * 32 + lane_off;    // packed P of its 64 keys
+    const uint32_t o_tm = tmem + 256 + t * 128 + ch * 64 + lane_off;
+    const uint32_t xbar = smem_u32(&bar_xchg[t][lq]);
     float scale2 = P.scale2;
     if (I8 && me.valid) scale2 *= P.q_scale[me.h] * P.k_scale[kvh];
     float m_ref = -INFINITY, l = 0.f;
@@ -343,76 +356,67 @@ __global__ void __launch_bounds__(352, 1)
     for (int j = 0; j < L; ++j) {
       if (!mbar_wait(smem_u32(&bar_sfull[t]), j & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
-      // the whole 128-column row in one TMEM load, one wait
-      uint32_t rr[128];
-      tmem_ld128(s_tm, rr);
-      tmem_ld_wait128(rr);
-      float s[128];
+      uint32_t rr[64];
+      tmem_ld64(s_tm, rr);
+      tmem_ld_wait64(rr);
+      float s[64];
 #pragma unroll
-      for (int e = 0; e < 128; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
+      for (int e = 0; e < 64; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
       if (j == L - 1) {
-        // diagonal chunk: key e of the chunk is visible iff e <= row
+        // diagonal chunk: key 64ch+e of the chunk is visible iff it is <= row
 #pragma unroll
-        for (int e = 0; e < 128; ++e) s[e] = (e <= row) ? s[e] : -INFINITY;
+        for (int e = 0; e < 64; ++e) s[e] = (ch * 64 + e <= row) ? s[e] : -INFINITY;
       }
-      // row max as 8 independent chains, then a short tree
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = s[e];
 #pragma unroll
-      for (int c = 8; c < 128; c += 8)
+      for (int c = 8; c < 64; c += 8)
 #pragma unroll
         for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[c + e]);
-      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      const float pmx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                              fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      // exchange with the partner half (also orders both halves' S reads
+      // before either writes P over the first 64 columns of S)
+      xmax[j & 1][t][ch][row] = pmx;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+      if (!mbar_wait(xbar, j & 1, abort_flag, P.err)) { ok = false; break; }
+      tc_fence_after();
+      const float mx = fmaxf(pmx, xmax[j & 1][t][ch ^ 1][row]);
       const float rmax2 = mx * scale2;
       const bool raise = rmax2 > m_ref + 8.f;
       const float m_new = raise ? rmax2 : m_ref;
       const float alpha = raise ? ex2(m_ref - m_new) : 1.f;
       // P in bf16 (the P.V operand); the row sum adds the same rounded values
-      // so numerator and denominator use identical weights.
-      // Off the diagonal chunk every fourth exponential runs on the FMA pipe
-      // (ex2_fma), the rest on MUFU; the diagonal chunk has masked (-inf)
-      // entries and uses MUFU only, which maps them to exactly 0.
-      uint32_t pk[64];
+      uint32_t pk[32];
       float r8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
-      if (C::kExpFmaEvery > 0 && j != L - 1) {
 #pragma unroll
-        for (int e = 0; e < 128; e += 2) {
-          const float x0 = fmaf(s[e], scale2, -m_new), x1 = fmaf(s[e + 1], scale2, -m_new);
-          const bool f1 = C::kExpFmaEvery > 0 && ((e + 1) % (C::kExpFmaEvery > 0 ? C::kExpFmaEvery : 1)) == 0;
-          pk[e >> 1] = pack_bf16x2(ex2(x0), f1 ? ex2_fma(x1) : ex2(x1));
-        }
-      } else {
+      for (int e = 0; e < 64; e += 2)
+        pk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], scale2, -m_new)), ex2(fmaf(s[e + 1], scale2, -m_new)));
 #pragma unroll
-        for (int e = 0; e < 128; e += 2)
-          pk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], scale2, -m_new)), ex2(fmaf(s[e + 1], scale2, -m_new)));
-      }
-#pragma unroll
-      for (int e = 0; e < 64; ++e)
+      for (int e = 0; e < 32; ++e)
         r8[e & 7] += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
       const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l = l * alpha + rs;
       m_ref = m_new;
       // The commit that signalled S(j) also covers PV(j-1), issued before
       // QK(j): O is stable here and may be rescaled in place.
-      if (j > 0) {
-        if (__any_sync(0xffffffffu, raise)) {
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
-          for (int qq = 0; qq < 4; ++qq) {
-            uint32_t o[32];
-            tmem_ld32(o_tm + qq * 32, o);
-            tmem_ld_wait(o);
+        for (int qq = 0; qq < 2; ++qq) {
+          uint32_t o[32];
+          tmem_ld32(o_tm + qq * 32, o);
+          tmem_ld_wait(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(o_tm + qq * 32, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(o_tm + qq * 32, o);
         }
       }
-      // P over the first 64 columns of this tile's S
-      tmem_st64(s_tm, pk);
+      tmem_st32(p_tm, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -420,28 +424,34 @@ __global__ void __launch_bounds__(352, 1)
     }
     if (ok && L > 0 && mbar_wait(smem_u32(&bar_odone[t]), (L - 1) & 1, abort_flag, P.err)) {
       tc_fence_after();
-      const float inv = 1.f / l;
-      __nv_bfloat16 *orow = P.out + ((size_t)me.h * P.S + (size_t)me.qc * 128 + row) * 128;
+      // total row sum: this half's plus the partner's (exchange phase L)
+      xl[t][ch][row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xbar);
+      if (mbar_wait(xbar, L & 1, abort_flag, P.err)) {
+        const float inv = 1.f / (l + xl[t][ch ^ 1][row]);
+        __nv_bfloat16 *orow = P.out + ((size_t)me.h * P.S + (size_t)me.qc * 128 + row) * 128 + ch * 64;
 #pragma unroll 1
-      for (int qq = 0; qq < 4; ++qq) {
-        uint32_t o[32];
-        tmem_ld32(o_tm + qq * 32, o);
-        tmem_ld_wait(o);
+        for (int qq = 0; qq < 2; ++qq) {
+          uint32_t o[32];
+          tmem_ld32(o_tm + qq * 32, o);
+          tmem_ld_wait(o);
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint4 v;
-          v.x = pack_bf16x2(__uint_as_float(o[c8 * 8 + 0]) * inv, __uint_as_float(o[c8 * 8 + 1]) * inv);
-          v.y = pack_bf16x2(__uint_as_float(o[c8 * 8 + 2]) * inv, __uint_as_float(o[c8 * 8 + 3]) * inv);
-          v.z = pack_bf16x2(__uint_as_float(o[c8 * 8 + 4]) * inv, __uint_as_float(o[c8 * 8 + 5]) * inv);
-          v.w = pack_bf16x2(__uint_as_float(o[c8 * 8 + 6]) * inv, __uint_as_float(o[c8 * 8 + 7]) * inv);
-          *reinterpret_cast<uint4 *>(orow + qq * 32 + c8 * 8) = v;
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint4 v;
+            v.x = pack_bf16x2(__uint_as_float(o[c8 * 8 + 0]) * inv, __uint_as_float(o[c8 * 8 + 1]) * inv);
+            v.y = pack_bf16x2(__uint_as_float(o[c8 * 8 + 2]) * inv, __uint_as_float(o[c8 * 8 + 3]) * inv);
+            v.z = pack_bf16x2(__uint_as_float(o[c8 * 8 + 4]) * inv, __uint_as_float(o[c8 * 8 + 5]) * inv);
+            v.w = pack_bf16x2(__uint_as_float(o[c8 * 8 + 6]) * inv, __uint_as_float(o[c8 * 8 + 7]) * inv);
+            *reinterpret_cast<uint4 *>(orow + qq * 32 + c8 * 8) = v;
+          }
         }
       }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 17) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
