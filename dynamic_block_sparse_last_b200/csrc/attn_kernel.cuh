@@ -271,6 +271,11 @@ __global__ void __launch_bounds__(608, 1)
     if (lane == 0) {
       const uint32_t id_qk = I8 ? idesc_i8(128, 128) : idesc_bf16(128, 128, 0);
       const uint32_t id_pv = idesc_bf16(128, 128, 1);
+      // Shared-memory descriptors built once: a byte offset d inside an
+      // operand is the descriptor plus d >> 4 (start address field, bits 0-13).
+      const uint64_t dq0 = umma_desc_sw128(sq, 16, 1024), dq1 = umma_desc_sw128(sq + C::kQKTile, 16, 1024);
+      const uint64_t dk0 = umma_desc_sw128(sk, 16, 1024), dk1 = umma_desc_sw128(sk + C::kQKTile, 16, 1024);
+      const uint64_t dv0 = umma_desc_sw128(sv, 16384, 1024), dv1 = umma_desc_sw128(sv + C::kVTile, 16384, 1024);
       UnionWalk uw;
       uw.init(chunk_bm[0], chunk_bm[1], words);
       int npv[2] = {0, 0};
@@ -281,11 +286,11 @@ __global__ void __launch_bounds__(608, 1)
       auto issue_pv = [&](int t, int vst) -> bool {
         if (!mbar_wait(smem_u32(&bar_pfull[t]), npv[t] & 1, abort_flag, P.err)) return false;
         tc_fence_after();
-        const uint32_t vb = sv + vst * C::kVTile;
+        const uint64_t dv = vst ? dv1 : dv0;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8,
-                      umma_desc_sw128(vb + kk * 2048, 16384, 1024), id_pv, (npv[t] > 0 || kk > 0));
+          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), id_pv,
+                      (npv[t] > 0 || kk > 0));
         tc_commit(smem_u32(&bar_odone[t]));
         ++npv[t];
         return true;
@@ -307,19 +312,17 @@ __global__ void __launch_bounds__(608, 1)
               tc_fence_after();
               kwaited = true;
             }
-            const uint32_t qb = sq + t * C::kQKTile, kb = sk + st * C::kQKTile;
+            const uint64_t dq = t ? dq1 : dq0, dk = st ? dk1 : dk0;
             const uint32_t d_tmem = tmem + t * 128;
             if (I8) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)
-                mma_i8_ss(d_tmem, umma_desc_sw128(qb + kk * 32, 16, 1024),
-                          umma_desc_sw128(kb + kk * 32, 16, 1024), id_qk, kk > 0);
+                mma_i8_ss(d_tmem, dq + (uint64_t)((kk * 32) >> 4), dk + (uint64_t)((kk * 32) >> 4), id_qk, kk > 0);
             } else {
 #pragma unroll
               for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_bf16_ss(d_tmem, umma_desc_sw128(qb + off, 16, 1024),
-                            umma_desc_sw128(kb + off, 16, 1024), id_qk, kk > 0);
+                const uint64_t off = (uint64_t)(((kk >> 2) * 16384 + (kk & 3) * 32) >> 4);
+                mma_bf16_ss(d_tmem, dq + off, dk + off, id_qk, kk > 0);
               }
             }
             tc_commit(smem_u32(&bar_sfull[t]));
@@ -367,15 +370,15 @@ __global__ void __launch_bounds__(608, 1)
 #pragma unroll
         for (int e = 0; e < 64; ++e) s[e] = (ch * 64 + e <= row) ? s[e] : -INFINITY;
       }
+      // row max: eight chains of three-input max, then a short tree
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = s[e];
 #pragma unroll
-      for (int c = 8; c < 64; c += 8)
+      for (int c = 8; c < 64; c += 16)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[c + e]);
-      const float pmx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                              fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
+      const float pmx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       // exchange with the partner half (also orders both halves' S reads
       // before either writes P over the first 64 columns of S)
       xmax[j & 1][t][ch][row] = pmx;
@@ -394,12 +397,33 @@ __global__ void __launch_bounds__(608, 1)
       float r8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) r8[e] = 0.f;
+      // Off the diagonal chunk every kExpFmaEvery-th exponential may run on
+      // the FMA pipe (ex2_fma); the diagonal chunk has masked (-inf) entries
+      // and uses MUFU only, which maps them to exactly 0.
+      if (C::kExpFmaEvery > 0 && j != L - 1) {
 #pragma unroll
-      for (int e = 0; e < 64; e += 2)
-        pk[e >> 1] = pack_bf16x2(ex2(fmaf(s[e], scale2, -m_new)), ex2(fmaf(s[e + 1], scale2, -m_new)));
+        for (int e = 0; e < 64; e += 2) {
+          const float x0 = fmaf(s[e], scale2, -m_new), x1 = fmaf(s[e + 1], scale2, -m_new);
+          const bool f1 = ((e + 1) % (C::kExpFmaEvery > 0 ? C::kExpFmaEvery : 1)) == 0;
+          pk[e >> 1] = pack_bf16x2(ex2(x0), f1 ? ex2_fma(x1) : ex2(x1));
+        }
+      } else {
+        // exponent arguments two at a time (packed fp32 FMA), then MUFU ex2
+        const uint64_t sc2 = f2_pack(scale2, scale2), nm2 = f2_pack(-m_new, -m_new);
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+          pk[e >> 1] = pack_bf16x2(ex2(x0), ex2(x1));
+        }
+      }
+      // row sum of the rounded P, two at a time (packed fp32 add)
+      uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int e = 0; e < 32; ++e)
-        r8[e & 7] += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+        a2[e & 3] = f2_add(a2[e & 3], f2_pack(__uint_as_float(pk[e] << 16), __uint_as_float(pk[e] & 0xFFFF0000u)));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f2_unpack(a2[e], r8[2 * e], r8[2 * e + 1]);
       const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l = l * alpha + rs;
       m_ref = m_new;
