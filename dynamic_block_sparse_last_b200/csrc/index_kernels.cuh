@@ -782,14 +782,17 @@ __device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const floa
       float f_hi = 0.f;
       while (hi - lo > 1u && c_lo - c_hi > 1) {
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        float f = 0.f;
-        int cnt = 0;
+        // four independent accumulation chains
+        float f4[4] = {0.f, 0.f, 0.f, 0.f};
+        int c4[4] = {0, 0, 0, 0};
 #pragma unroll
         for (int i = 0; i < NL; ++i) {
           const bool ge = (lane + 32 * i < r) && __float_as_uint(v[i]) >= mid;
-          f += ge ? v[i] : 0.f;
-          cnt += ge ? 1 : 0;
+          f4[i & 3] += ge ? v[i] : 0.f;
+          c4[i & 3] += ge ? 1 : 0;
         }
+        float f = (f4[0] + f4[1]) + (f4[2] + f4[3]);
+        int cnt = (c4[0] + c4[1]) + (c4[2] + c4[3]);
 #pragma unroll
         for (int s = 16; s > 0; s >>= 1) {
           f += __shfl_xor_sync(0xffffffffu, f, s);

@@ -1,0 +1,79 @@
+"""Host-side logic without a GPU: the parity comparator's acceptance rules and
+the benchmark's clock-sample parsing and traffic-record bookkeeping."""
+import json
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+from tests import parity  # noqa: E402
+
+
+def row(w):
+    w = np.asarray(w, dtype=np.float64)
+    return w / w.sum()
+
+
+def test_equal_sets_pass_without_tolerance():
+    ok, tol, _ = parity.compare_row([0, 3], [0, 3], row([5, 1, 1, 4]), [0.5, 0.3, 0.8], 0.75, 3)
+    assert ok and tol == 0
+
+
+def test_near_cut_swap_is_tolerated_and_counted():
+    w = row([0.300000, 0.3000001, 0.1, 0.2999999])
+    # oracle kept block 1 (score just above block 0's); the GPU kept block 0
+    info = [w[1], w[3], w[3] + w[1]]
+    ok, tol, _ = parity.compare_row([0, 3], [1, 3], w, info, 0.5, 3)
+    assert ok and tol == 2
+
+
+def test_far_mismatch_is_rejected():
+    w = row([0.5, 0.05, 0.05, 0.4])
+    info = [w[0], w[3], w[3] + w[0]]
+    ok, _, msg = parity.compare_row([1, 3], [0, 3], w, info, 0.8, 3)
+    assert not ok and "differs" in msg
+
+
+def test_missing_diagonal_and_unsorted_lists_are_rejected():
+    w = row([1, 1, 1])
+    assert not parity.compare_row([0, 1], [0, 1, 2], w, [-1, 1, 1], 0.5, 2)[0]
+    assert not parity.compare_row([2, 0], [0, 2], w, [-1, 1, 1], 0.5, 2)[0]
+
+
+def test_gamma_one_requires_the_full_row():
+    w = row([1, 1, 1])
+    assert not parity.compare_row([0, 2], [0, 1, 2], w, [-1, 1, 1], 1.0, 2)[0]
+    assert parity.compare_row([0, 1, 2], [0, 1, 2], w, [-1, 1, 1], 1.0, 2)[0]
+
+
+def test_one_extra_block_allowed_only_when_oracle_barely_crossed_gamma():
+    w = row([0.2, 0.1, 0.7])
+    # oracle: diag 0.7 + block 0 0.2 = 0.9 reaches gamma exactly; the GPU took block 1 too
+    info = [w[0], w[2], w[2] + w[0]]
+    assert parity.compare_row([0, 1, 2], [0, 2], w, info, 0.9, 2)[0]
+    assert not parity.compare_row([0, 1, 2], [0, 2], w, info, 0.85, 2)[0]
+
+
+def test_clock_sampler_parses_reasons_and_median():
+    import bench
+    cs = bench.ClockSampler(0)
+    cs.proc = type("P", (), {"terminate": lambda self: None, "wait": lambda self, timeout=None: 0})()
+    cs.lines = ["1800, 1965, 900.1, 0x4, Not Active, Not Active, Not Active, Active",
+                "1750, 1965, 950.2, 0x4, Not Active, Not Active, Not Active, Active",
+                "1900, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+                "garbage"]
+    out = cs.stop()
+    assert out["sm_mhz"] == 1800 and out["sm_max_mhz"] == 1965 and out["reasons"] == ["sw_power_cap"]
+
+
+def test_traffic_record_is_dropped_when_the_kernel_source_changes(tmp_path, monkeypatch):
+    import bench
+    rec = json.load(open(os.path.join(ROOT, "profiles", "attn_traffic.json")))
+    assert set(rec) >= {"dram_bytes_per_launch", "kernel_src_sha256", "command"}
+    fake = tmp_path / "attn.cuh"
+    fake.write_text("// another kernel\n")
+    monkeypatch.setattr(bench, "ATTN_SRC", str(fake))
+    assert bench.attn_traffic_record() is None
