@@ -12,7 +12,10 @@
 //   b = 128, g == 1:    two neighbouring query tiles of one head
 // The CTA walks the union of the two tiles' chunk lists (ascending 128-key
 // chunks); a chunk only one tile needs is computed for that tile only.
-// CTAs are numbered heavy first (descending query position).
+// CTAs are numbered KV-head-major (all CTAs of one KV head together, so its
+// K and V stay in L2 while they run; the GPU analogue of the article's
+// KV-block-major schedule, section 3.2) and heavy first (descending query
+// position) within a KV head.
 //
 // Warp roles (608 threads):
 //   warps 0-7 / 8-15 softmax, correction and epilogue of tile 0 / tile 1:
@@ -76,26 +79,29 @@ struct AttnTile {
   const int *list;
 };
 
-// The two query tiles of CTA `pair`, heavy pairs first.
+// The two query tiles of CTA `pair`: KV-head-major, heavy pairs first within a head.
 __device__ inline void attn_pair_tiles(const AttnParams &P, int pair, AttnTile (&t)[2]) {
   const int nq = P.S / 128, g = P.g;
   int h0, h1, q0, q1, v1;
+  // KV-head-major: all CTAs of one KV head (its K/V fit in L2), heavy first within it
   if (P.b == 256) {
-    const int rr = P.n - 1 - pair / P.Hq;
-    h0 = h1 = pair % P.Hq;
+    const int per_kv = g * P.n, kvh = pair / per_kv, rem = pair % per_kv;
+    const int rr = P.n - 1 - rem / g;
+    h0 = h1 = kvh * g + rem % g;
     q0 = 2 * rr;
     q1 = 2 * rr + 1;
     v1 = 1;
   } else if (g >= 2) {
-    const int hp = (g + 1) / 2, per_qc = P.Hkv * hp;
-    const int qc = nq - 1 - pair / per_qc, rem = pair % per_qc;
-    h0 = (rem / hp) * g + 2 * (rem % hp);
+    const int hp = (g + 1) / 2, per_kv = hp * nq, kvh = pair / per_kv, rem = pair % per_kv;
+    const int qc = nq - 1 - rem / hp, k = rem % hp;
+    h0 = kvh * g + 2 * k;
     h1 = h0 + 1;
-    v1 = (2 * (rem % hp) + 1) < g;
+    v1 = (2 * k + 1) < g;
     q0 = q1 = qc;
   } else {
-    const int m = (nq + 1) / 2 - 1 - pair / P.Hq;
-    h0 = h1 = pair % P.Hq;
+    const int per_kv = (nq + 1) / 2, h = pair / per_kv;
+    const int m = per_kv - 1 - pair % per_kv;
+    h0 = h1 = h;
     q0 = 2 * m;
     q1 = 2 * m + 1;
     v1 = q1 < nq;
