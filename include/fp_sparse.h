@@ -24,6 +24,12 @@
  * NULL = legacy default stream) unless stated; the caller keeps every buffer
  * alive until the stream has passed the call.
  *
+ * Batches: B sequences of equal length S are one call with the tensors
+ * stacked sequence-major, i.e. q[B*Hq][S][d], k and v [B*Hkv][S][d], passing
+ * B*Hq and B*Hkv as the head counts (query head b*Hq + h then reads KV head
+ * b*Hkv + h/(Hq/Hkv), as it should).  Every step works per head, so the result
+ * equals B separate calls.
+ *
  * Errors: functions return FP_OK (0) or an FP_ERR_* code; nothing aborts the
  * process.  Argument errors are detected on the host before any launch.  A
  * device-side bounded wait that gives up records FP_ERR_TIMEOUT in a sticky
@@ -141,9 +147,10 @@ int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int H
  *
  * Scratch: a fixed 32 MiB array inside the library (a file-scope device
  * array; every GPU that loads the library keeps it until process exit).  A
- * problem needs at most 12*Hq*S + 128*Hq*b + 8*Hq*(S/128) + 4*Hkv*S +
- * 512*Hkv*(S/b) bytes of it plus 2 KiB of alignment; e.g. S=32768 with
- * Hq=32, Hkv=8 fits, and so does S=131072 with Hq=16, Hkv=4.
+ * problem needs at most 12*Hq*C*b + 128*Hq*b + 8*Hq*C + 512*Hkv*C +
+ * 512*Hkv*n bytes of it, with C = ceil(S/128) and n = ceil(S/b), plus 2 KiB
+ * of alignment; e.g. S=32768 with Hq=32, Hkv=8, b=128 fits, and so does
+ * S=131072 with Hq=16, Hkv=4, b=128.
  * Larger problems are rejected with FP_ERR_ARG before anything is launched.
  * The first call on a device looks up the array's device address (set-up,
  * once per device, with that device current); make that first call before

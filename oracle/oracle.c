@@ -23,8 +23,9 @@
  * tie order, ">= gamma", int8 scale) are the written conventions of the
  * package design notes; each function below states the one it uses.
  *
- * Notation: n = S/b blocks, g = Hq/Hkv, query head h reads KV head h/g,
- * tensors are [H][S][d] row-major, the "last block" is rows (n-1)b .. S-1.
+ * Notation: n = ceil(S/b) blocks (the last one holds S - (n-1)b tokens when
+ * b does not divide S), g = Hq/Hkv, query head h reads KV head h/g, tensors
+ * are [H][S][d] row-major, the "last block" is rows (n-1)b .. S-1.
  */
 #include <math.h>
 #include <stdint.h>
@@ -101,19 +102,22 @@ static double logit(const orc_problem *P, int h, int p, int j)
     return dot_bf(qr, kr, P->d) * inv;
 }
 
+static int nblocks(const orc_problem *P) { return (P->S + P->b - 1) / P->b; }
+
 /* S1+S2 ([FP] 2.1, 3.1): score the last query block of head h against every
- * causal key, softmax each row over j <= p, and pool the probabilities
- *   vhat[c] = (1/b) sum_i sum_{j in block c} A_ij                (vertical)
- *   shat[o] = (1/b) sum_i sum_{j : floor((p_i - j)/b) = o} A_ij  (slash)
+ * causal key, softmax each row over j <= p, and pool the probabilities over
+ * the block's L = S - (n-1)b rows
+ *   vhat[c] = (1/L) sum_i sum_{j in block c} A_ij                (vertical)
+ *   shat[o] = (1/L) sum_i sum_{j : floor((p_i - j)/b) = o} A_ij  (slash)
  * Returns max |sum_j A_ij - 1| over the block's rows. */
 double orc_last_block_stats(const orc_problem *P, int h, double *vhat, double *shat)
 {
-    int S = P->S, b = P->b, n = S / b;
-    int p0 = (n - 1) * b;
+    int S = P->S, b = P->b, n = nblocks(P);
+    int p0 = (n - 1) * b, rows = S - p0;
     double *s = (double *)malloc(sizeof(double) * (size_t)S);
     double worst = 0.0;
     for (int c = 0; c < n; ++c) { vhat[c] = 0.0; shat[c] = 0.0; }
-    for (int i = 0; i < b; ++i) {
+    for (int i = 0; i < rows; ++i) {
         int p = p0 + i;
         double mx = -INFINITY, z = 0.0, rs = 0.0;
         for (int j = 0; j <= p; ++j) {
@@ -129,30 +133,32 @@ double orc_last_block_stats(const orc_problem *P, int h, double *vhat, double *s
         }
         if (fabs(rs - 1.0) > worst) worst = fabs(rs - 1.0);
     }
-    for (int c = 0; c < n; ++c) { vhat[c] /= b; shat[c] /= b; }
+    for (int c = 0; c < n; ++c) { vhat[c] /= rows; shat[c] /= rows; }
     free(s);
     return worst;
 }
 
 /* Block means of the rows of head `head` of Q (which = 0) or K (which = 1):
- * out[c][t] = (1/b) sum_{p in block c} x[p][t].  For int8 problems the exact
- * integer column sum is scaled by the head's scale. */
+ * out[c][t] = mean over the rows p of block c (all b of them, or the
+ * S - (n-1)b of a partial last block) of x[p][t].  For int8 problems the
+ * exact integer column sum is scaled by the head's scale. */
 void orc_block_means(const orc_problem *P, int which, int head, double *out)
 {
-    int S = P->S, b = P->b, d = P->d, n = S / b;
+    int S = P->S, b = P->b, d = P->d, n = nblocks(P);
     for (int c = 0; c < n; ++c) {
+        int hi = (c + 1) * b < S ? (c + 1) * b : S, cnt = hi - c * b;
         for (int t = 0; t < d; ++t) {
             if (P->qk_int8) {
                 const int8_t *x = (which == 0 ? P->q8 : P->k8) + (size_t)head * S * d;
                 int64_t acc = 0;
-                for (int p = c * b; p < (c + 1) * b; ++p) acc += x[(size_t)p * d + t];
+                for (int p = c * b; p < hi; ++p) acc += x[(size_t)p * d + t];
                 double sc = which == 0 ? P->q_scale[head] : P->k_scale[head];
-                out[(size_t)c * d + t] = (double)acc * sc / b;
+                out[(size_t)c * d + t] = (double)acc * sc / cnt;
             } else {
                 const uint16_t *x = (which == 0 ? P->q : P->k) + (size_t)head * S * d;
                 double acc = 0.0;
-                for (int p = c * b; p < (c + 1) * b; ++p) acc += bf(x[(size_t)p * d + t]);
-                out[(size_t)c * d + t] = acc / b;
+                for (int p = c * b; p < hi; ++p) acc += bf(x[(size_t)p * d + t]);
+                out[(size_t)c * d + t] = acc / cnt;
             }
         }
     }
@@ -266,7 +272,7 @@ double orc_build_index_head(const orc_problem *P, int h, double gamma, double ta
                             double *vhat, double *shat, double *pest, double *jsd, int32_t *pattern,
                             int32_t *counts, int32_t *cols, double *scores, double *info)
 {
-    int S = P->S, b = P->b, d = P->d, n = S / b, kvh = h / (P->Hq / P->Hkv);
+    int b = P->b, d = P->d, n = nblocks(P), kvh = h / (P->Hq / P->Hkv);
     double worst = orc_last_block_stats(P, h, vhat, shat);
     double *kbar = (double *)malloc(sizeof(double) * (size_t)n * d);
     double *qbar = (double *)malloc(sizeof(double) * (size_t)n * d);
@@ -303,7 +309,7 @@ void orc_attn_rows(const orc_problem *P, int h, int p_lo, int p_hi, const int32_
         int m = 0;
         double mx = -INFINITY, z = 0.0;
         for (int e = 0; e < nblocks; ++e)
-            for (int j = blocks[e] * b; j < (blocks[e] + 1) * b; ++j)
+            for (int j = blocks[e] * b; j < (blocks[e] + 1) * b && j < S; ++j)
                 if (j <= p) { js[m] = j; s[m] = logit(P, h, p, j); if (s[m] > mx) mx = s[m]; ++m; }
         for (int e = 0; e < m; ++e) { s[e] = exp(s[e] - mx); z += s[e]; }
         double *o = out + (size_t)(p - p_lo) * d;

@@ -103,7 +103,7 @@ class OracleProblem:
         Hq, S, d = q.shape
         Hkv = k.shape[0]
         self.S, self.Hq, self.Hkv, self.d, self.b = S, Hq, Hkv, d, b
-        self.n = S // b
+        self.n = (S + b - 1) // b
         self.int8 = q8 is not None
         self._keep = []
 

@@ -177,3 +177,22 @@ def test_full_size_layers(fp, name, ntiles):
             fp.fp_debug_qk_tile_i8(q8, k8, w.S, w.Hq, w.Hkv, w.d, h, p0, j0, t)
             torch.cuda.synchronize()
             assert np.array_equal(t.cpu().numpy(), P.qk_int_tile(h, p0, j0, 128, 128))
+
+
+def test_batched_sequences_equal_separate_calls(fp):
+    """B sequences of equal length run as one call with B*Hq / B*Hkv heads
+    (stacked sequence-major) and give bit-identical index and output."""
+    ws = [synth.Workload(f"seq{i}", S=2048, Hq=4, Hkv=2, b=128, seed=30 + i) for i in range(2)]
+    xs = [synth.make_inputs(w) for w in ws]
+    single = [run_gpu(fp, x, w) for x, w in zip(xs, ws)]
+    xb = {key: torch.cat([x[key] for x in xs], 0) for key in ("q", "k", "v")}
+    wb = synth.Workload("batch2", S=2048, Hq=8, Hkv=4, b=128, seed=0)
+    exp_b, out_b, _ = run_gpu(fp, xb, wb)
+    n = wb.S // wb.b
+    for i, (exp, out, _) in enumerate(single):
+        assert torch.equal(out_b[4 * i: 4 * i + 4], out)
+        assert np.array_equal(exp_b["pattern"][4 * i: 4 * i + 4], exp["pattern"])
+        for h in range(4):
+            rows_b = parity.gpu_rows(exp_b, 4 * i + h, n)
+            rows_s = parity.gpu_rows(exp, h, n)
+            assert all(np.array_equal(a, c) for a, c in zip(rows_b, rows_s))

@@ -165,12 +165,15 @@ def test_qa_scores_match_scipy_softmax():
 
 # ---------------------------------------------------------------- last-block statistics
 
-@pytest.mark.parametrize("S,b,d,int8", [(16, 4, 8, False), (24, 8, 16, False), (32, 8, 8, True)])
+@pytest.mark.parametrize("S,b,d,int8", [(16, 4, 8, False), (24, 8, 16, False), (32, 8, 8, True),
+                                         (18, 4, 8, False), (29, 8, 16, True)])
 def test_last_block_stats_against_full_attention_matrix(S, b, d, int8):
     """vhat / shat from the full causal softmax matrix (torch fp64), pooled
-    by block columns and by torch.diagonal sums."""
+    by block columns and by torch.diagonal sums; S not a multiple of b gives a
+    partial last block whose rows are averaged."""
     P, (q, k, v, q8, k8, qs, ks) = rand_problem(S, 2, 1, d, b, seed=S + b, int8=int8, scale=2.0)
-    n = S // b
+    n = -(-S // b)
+    rows_last = S - (n - 1) * b
     for h in range(2):
         if int8:
             logits = (q8[h].double() @ k8[0].double().T) * (float(qs[h]) * float(ks[0])) / math.sqrt(d)
@@ -179,12 +182,12 @@ def test_last_block_stats_against_full_attention_matrix(S, b, d, int8):
         mask = torch.ones(S, S, dtype=torch.bool).tril()
         A = torch.softmax(logits.masked_fill(~mask, float("-inf")), dim=-1)
         last = A[(n - 1) * b:]
-        vref = last.reshape(b, n, b).sum(dim=(0, 2)) / b
+        vref = torch.stack([last[:, c * b:(c + 1) * b].sum() for c in range(n)]) / rows_last
         sref = torch.zeros(n, dtype=torch.float64)
         for delta in range(S):
             diag = torch.diagonal(A, offset=-delta)            # entries (p, p - delta)
             rows = torch.arange(delta, S)
-            sref[delta // b] += diag[rows >= (n - 1) * b].sum() / b
+            sref[delta // b] += diag[rows >= (n - 1) * b].sum() / rows_last
         vh, sh, err = P.last_block_stats(h)
         assert err < 1e-12
         assert np.allclose(vh, vref.numpy(), atol=1e-14)
@@ -226,6 +229,14 @@ def test_single_block_is_query_aware_with_zero_divergence():
     assert out["pattern"] == orc.VS
 
 
+def test_block_means_of_a_partial_last_block():
+    P, (q, k, *_r) = rand_problem(S=40, Hq=1, Hkv=1, d=8, b=16, seed=5)
+    km = P.block_means("k", 0)
+    assert km.shape == (3, 8)
+    assert np.allclose(km[2], k[0, 32:40].double().mean(0).numpy(), atol=1e-15)
+    assert np.allclose(km[0], k[0, 0:16].double().mean(0).numpy(), atol=1e-15)
+
+
 def test_block_means_match_torch():
     P, (q, k, v, q8, k8, qs, ks) = rand_problem(S=64, Hq=2, Hkv=1, d=16, b=16, seed=2, int8=True)
     qb = P.block_means("q", 1)
@@ -251,21 +262,23 @@ def sdpa_ref(q, k, v, h, g, mask=None, int8=None):
     return A @ v[h // g].double()
 
 
-@pytest.mark.parametrize("int8", [False, True])
-def test_gamma_one_equals_dense_causal_attention(int8):
-    S, b, d = 48, 8, 16
+@pytest.mark.parametrize("int8,S", [(False, 48), (True, 48), (False, 45), (True, 51)])
+def test_gamma_one_equals_dense_causal_attention(int8, S):
+    b, d = 8, 16
     P, (q, k, v, q8, k8, qs, ks) = rand_problem(S, 4, 2, d, b, seed=11, int8=int8, scale=1.5)
     for h in range(4):
         idx = P.build_index_head(h, 1.0, 0.1)
         assert all(list(r) == list(range(i + 1)) for i, r in enumerate(idx["rows"]))
-        got = np.concatenate([P.attn_rows(h, r * b, (r + 1) * b, idx["rows"][r]) for r in range(S // b)])
+        nb = -(-S // b)
+        got = np.concatenate([P.attn_rows(h, r * b, min((r + 1) * b, S), idx["rows"][r]) for r in range(nb)])
         ref = sdpa_ref(q, k, v, h, 2, int8=(q8, k8, qs, ks) if int8 else None)
         assert np.allclose(got, ref.numpy(), atol=1e-12)
     if not int8:
         sd = torch.nn.functional.scaled_dot_product_attention(
             q.double()[None], k.double().repeat_interleave(2, 0)[None], v.double().repeat_interleave(2, 0)[None],
             is_causal=True)[0]
-        got = np.concatenate([P.attn_rows(1, r * b, (r + 1) * b, list(range(r + 1))) for r in range(S // b)])
+        nb = -(-S // b)
+        got = np.concatenate([P.attn_rows(1, r * b, min((r + 1) * b, S), list(range(r + 1))) for r in range(nb)])
         assert np.allclose(got, sd[1].numpy(), atol=1e-12)
 
 
