@@ -12,6 +12,10 @@
 //   b = 128, g == 1:    two neighbouring query tiles of one head
 // The CTA walks the union of the two tiles' chunk lists (ascending 128-key
 // chunks); a chunk only one tile needs is computed for that tile only.
+// When 128 does not divide S the last query tile and the last key chunk run
+// past S: the tensor maps read whatever follows (the next head's rows, or
+// zeros past the end of the tensor), the causal mask keeps those keys away
+// from every real row, and rows at or past S are not stored.
 // CTAs are numbered KV-head-major (all CTAs of one KV head together, so its
 // K and V stay in L2 while they run; the GPU analogue of the article's
 // KV-block-major schedule, section 3.2) and heavy first (descending query
@@ -68,8 +72,8 @@ struct AttnCfg {
 
 // Number of CTAs (tile pairs) for a layer shape.
 __host__ __device__ inline int attn_pairs(int Hq, int Hkv, int S, int b) {
-  const int nq = S / 128, g = Hq / Hkv;
-  if (b == 256) return Hq * (S / b);
+  const int nq = (S + 127) / 128, g = Hq / Hkv;
+  if (b == 256) return Hq * ((S + b - 1) / b);
   if (g >= 2) return Hkv * ((g + 1) / 2) * nq;
   return Hq * ((nq + 1) / 2);
 }
@@ -81,7 +85,7 @@ struct AttnTile {
 
 // The two query tiles of CTA `pair`: KV-head-major, heavy pairs first within a head.
 __device__ inline void attn_pair_tiles(const AttnParams &P, int pair, AttnTile (&t)[2]) {
-  const int nq = P.S / 128, g = P.g;
+  const int nq = (P.S + 127) / 128, g = P.g;
   int h0, h1, q0, q1, v1;
   // KV-head-major: all CTAs of one KV head (its K/V fit in L2), heavy first within it
   if (P.b == 256) {
@@ -90,7 +94,7 @@ __device__ inline void attn_pair_tiles(const AttnParams &P, int pair, AttnTile (
     h0 = h1 = kvh * g + rem % g;
     q0 = 2 * rr;
     q1 = 2 * rr + 1;
-    v1 = 1;
+    v1 = q1 < nq;  // a partial last block may have a single tile
   } else if (g >= 2) {
     const int hp = (g + 1) / 2, per_kv = hp * nq, kvh = pair / per_kv, rem = pair % per_kv;
     const int qc = nq - 1 - rem / hp, k = rem % hp;
@@ -460,6 +464,7 @@ __global__ void __launch_bounds__(608, 1)
       if (lane == 0) mbar_arrive(xbar);
       if (mbar_wait(xbar, L & 1, abort_flag, P.err)) {
         const float inv = 1.f / (l + xl[t][ch ^ 1][row]);
+        const bool store = me.qc * 128 + row < P.S;  // rows past S belong to the next head
         __nv_bfloat16 *orow = P.out + ((size_t)me.h * P.S + (size_t)me.qc * 128 + row) * 128 + ch * 64;
 #pragma unroll 1
         for (int qq = 0; qq < 2; ++qq) {
@@ -473,7 +478,7 @@ __global__ void __launch_bounds__(608, 1)
             v.y = pack_bf16x2(__uint_as_float(o[c8 * 8 + 2]) * inv, __uint_as_float(o[c8 * 8 + 3]) * inv);
             v.z = pack_bf16x2(__uint_as_float(o[c8 * 8 + 4]) * inv, __uint_as_float(o[c8 * 8 + 5]) * inv);
             v.w = pack_bf16x2(__uint_as_float(o[c8 * 8 + 6]) * inv, __uint_as_float(o[c8 * 8 + 7]) * inv);
-            *reinterpret_cast<uint4 *>(orow + qq * 32 + c8 * 8) = v;
+            if (store) *reinterpret_cast<uint4 *>(orow + qq * 32 + c8 * 8) = v;
           }
         }
       }

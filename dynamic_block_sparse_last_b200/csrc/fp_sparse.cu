@@ -94,7 +94,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 bool shape_ok(int S, int Hq, int Hkv, int d, int b) {
   if (d != 128) return false;
   if (b != 128 && b != 256) return false;
-  if (S <= 0 || S % b != 0 || S / b > kSelMaxN) return false;
+  if (S <= 0 || (S + b - 1) / b > kSelMaxN) return false;
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return false;
   if ((int64_t)Hq * S > (int64_t)INT32_MAX || (int64_t)Hkv * S > (int64_t)INT32_MAX) return false;
   return true;
@@ -132,6 +132,69 @@ int set_smem_attrs() {
   return FP_OK;
 }
 
+// Shape, inputs and scratch of the pattern-statistics launches (steps 1-3 of
+// fp_build_index), shared by the index build and the allocation-free call.
+struct StatsJob {
+  int S, Hq, Hkv, d, b, n, nch, g, R2, chunks_per_part;
+  const void *q, *k;
+  const float *q_scale, *k_scale;  // int8 only
+  float tau;
+  float *pm, *plo, *phi, *partM, *partL, *LOc, *HIc, *ksum, *kbar;
+  float *vhat, *shat, *pest, *jsd;
+  int *pattern;
+};
+
+// k_score_last, k_row_stats, k_block_mass, k_kbar and k_pattern on `st`.
+template <bool I8>
+int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
+  int rc;
+  CUtensorMap tq, tk;
+  if (!make_map(&tq, J.q, I8, (uint64_t)J.Hq * J.S) || !make_map(&tk, J.k, I8, (uint64_t)J.Hkv * J.S))
+    return FP_ERR_CUDA;
+  const int nlast = J.S - (J.n - 1) * J.b;  // rows of the (possibly partial) last block
+  const int tiles_per_head = (nlast + 127) / 128;
+  const int tiles_per_group = J.g * tiles_per_head;
+  const int tgroups = (tiles_per_group + 3) / 4;
+  int R = sm_count() / (tgroups * J.Hkv);
+  if (R < 1) R = 1;
+  if (R > J.nch) R = J.nch;
+  const int cpc = (J.nch + R - 1) / R;
+  R = (J.nch + cpc - 1) / cpc;
+  ScoreParams sp;
+  sp.S = J.S; sp.Hq = J.Hq; sp.Hkv = J.Hkv; sp.b = J.b; sp.n = J.n; sp.nch = J.nch; sp.g = J.g;
+  sp.nlast = nlast;
+  sp.tiles_per_head = tiles_per_head;
+  sp.tiles_per_group = tiles_per_group;
+  sp.chunks_per_cta = cpc;
+  sp.scale2 = kLog2e / sqrtf((float)J.d);
+  sp.q_scale = J.q_scale;
+  sp.k_scale = J.k_scale;
+  sp.pm = J.pm; sp.plo = J.plo; sp.phi = J.phi; sp.ksum = J.ksum;
+  sp.err = err;
+  k_score_last<I8><<<dim3(R, tgroups, J.Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
+  if ((rc = launch_status())) return rc;
+  k_row_stats<<<dim3(J.Hq, J.R2), J.b, 0, st>>>(J.pm, J.plo, J.phi, J.nch, J.b, nlast, J.chunks_per_part,
+                                                J.partM, J.partL);
+  if ((rc = launch_status())) return rc;
+  const size_t red_bytes = (size_t)(J.b / 32) * J.chunks_per_part * 2 * sizeof(float);
+  k_block_mass<<<dim3(J.Hq, J.R2), J.b, red_bytes, st>>>(J.pm, J.plo, J.phi, J.partM, J.partL, J.nch, J.b,
+                                                         nlast, J.chunks_per_part, J.LOc, J.HIc);
+  if ((rc = launch_status())) return rc;
+  k_kbar<<<dim3(J.n, J.Hkv), 128, 0, st>>>(J.ksum, I8 ? J.k_scale : nullptr, J.S, J.nch, J.b, J.n, J.kbar);
+  if ((rc = launch_status())) return rc;
+  k_pattern<I8><<<J.Hq, 1024, 0, st>>>(J.q, J.q_scale, J.LOc, J.HIc, J.kbar, J.S, J.g, J.b, J.n, J.nch,
+                                       1.0f / sqrtf((float)J.d), J.tau, J.vhat, J.shat, J.pest, J.jsd,
+                                       J.pattern);
+  return launch_status();
+}
+
+// Row-part split of the per-row reductions: at most 16 parts over the chunks.
+void row_parts(int nch, int &R2, int &chunks_per_part) {
+  R2 = nch < 16 ? nch : 16;
+  chunks_per_part = (nch + R2 - 1) / R2;
+  R2 = (nch + chunks_per_part - 1) / chunks_per_part;
+}
+
 template <bool I8>
 int build_index_impl(const void *q, const void *k, float gamma, float tau, const float *q_scale,
                      const float *k_scale, fp_index *I, cudaStream_t st) {
@@ -139,43 +202,15 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   if (rc) return rc;
   int *err = device_error_word();
   if (!err) return FP_ERR_CUDA;
-  CUtensorMap tq, tk;
-  if (!make_map(&tq, q, I8, (uint64_t)I->Hq * I->S) || !make_map(&tk, k, I8, (uint64_t)I->Hkv * I->S))
-    return FP_ERR_CUDA;
-  const int tiles_per_group = I->g * (I->b / 128);
-  const int tgroups = (tiles_per_group + 3) / 4;
-  int R = sm_count() / (tgroups * I->Hkv);
-  if (R < 1) R = 1;
-  if (R > I->nch) R = I->nch;
-  int cpc = (I->nch + R - 1) / R;
-  R = (I->nch + cpc - 1) / cpc;
-  ScoreParams sp;
-  sp.S = I->S; sp.Hq = I->Hq; sp.Hkv = I->Hkv; sp.b = I->b; sp.n = I->n; sp.nch = I->nch; sp.g = I->g;
-  sp.tiles_per_group = tiles_per_group;
-  sp.chunks_per_cta = cpc;
-  sp.scale2 = kLog2e / sqrtf((float)I->d);
-  sp.q_scale = q_scale;
-  sp.k_scale = k_scale;
-  sp.pm = I->pm; sp.plo = I->plo; sp.phi = I->phi; sp.ksum = I->ksum;
-  sp.err = err;
-  k_score_last<I8><<<dim3(R, tgroups, I->Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
-  if ((rc = launch_status())) return rc;
-
-  k_row_stats<<<dim3(I->Hq, I->R2), I->b, 0, st>>>(I->pm, I->plo, I->phi, I->nch, I->b,
-                                                   I->chunks_per_part, I->partM, I->partL);
-  if ((rc = launch_status())) return rc;
-  const size_t red_bytes = (size_t)(I->b / 32) * I->chunks_per_part * 2 * sizeof(float);
-  k_block_mass<<<dim3(I->Hq, I->R2), I->b, red_bytes, st>>>(I->pm, I->plo, I->phi, I->partM, I->partL,
-                                                            I->nch, I->b, I->chunks_per_part, I->LOc,
-                                                            I->HIc);
-  if ((rc = launch_status())) return rc;
-  k_kbar<<<dim3(I->n, I->Hkv), 128, 0, st>>>(I->ksum, I8 ? k_scale : nullptr, I->nch, I->b, I->n, I->kbar);
-  if ((rc = launch_status())) return rc;
+  StatsJob J;
+  J.S = I->S; J.Hq = I->Hq; J.Hkv = I->Hkv; J.d = I->d; J.b = I->b; J.n = I->n; J.nch = I->nch; J.g = I->g;
+  J.R2 = I->R2; J.chunks_per_part = I->chunks_per_part;
+  J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
+  J.pm = I->pm; J.plo = I->plo; J.phi = I->phi; J.partM = I->partM; J.partL = I->partL;
+  J.LOc = I->LOc; J.HIc = I->HIc; J.ksum = I->ksum; J.kbar = I->kbar;
+  J.vhat = I->vhat; J.shat = I->shat; J.pest = I->pest; J.jsd = I->jsd; J.pattern = I->pattern;
+  if ((rc = launch_pattern_stats<I8>(J, err, st))) return rc;
   const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
-  k_pattern<I8><<<I->Hq, 1024, 0, st>>>(q, q_scale, I->LOc, I->HIc, I->kbar, I->S, I->g, I->b, I->n,
-                                        I->nch, inv_sqrt_d, tau, I->vhat, I->shat, I->pest, I->jsd,
-                                        I->pattern);
-  if ((rc = launch_status())) return rc;
   k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->b, I->n, I->qbar);
   if ((rc = launch_status())) return rc;
   const int nt = (I->n + kLgTile - 1) / kLgTile;
@@ -223,10 +258,8 @@ int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out) {
   fp_index *I = static_cast<fp_index *>(calloc(1, sizeof(fp_index)));
   if (!I) return FP_ERR_CUDA;
   I->S = S; I->Hq = Hq; I->Hkv = Hkv; I->d = d; I->b = b;
-  I->n = S / b; I->nch = S / 128; I->g = Hq / Hkv;
-  I->R2 = I->nch < 16 ? I->nch : 16;
-  I->chunks_per_part = (I->nch + I->R2 - 1) / I->R2;
-  I->R2 = (I->nch + I->chunks_per_part - 1) / I->chunks_per_part;
+  I->n = (S + b - 1) / b; I->nch = (S + 127) / 128; I->g = Hq / Hkv;
+  row_parts(I->nch, I->R2, I->chunks_per_part);
   cudaGetDevice(&I->device);
   const size_t n = I->n, nch = I->nch, bb = b;
   const size_t tri = n * (n + 1) / 2;
@@ -451,10 +484,9 @@ template <bool I8>
 int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int d, int b, float tau,
                        const float *q_scale, const float *k_scale, float *vhat, float *shat, float *pest,
                        float *jsd, int32_t *pattern, cudaStream_t st) {
-  const int n = S / b, nch = S / 128, g = Hq / Hkv;
-  int R2 = nch < 16 ? nch : 16;
-  const int cpp = (nch + R2 - 1) / R2;
-  R2 = (nch + cpp - 1) / cpp;
+  const int n = (S + b - 1) / b, nch = (S + 127) / 128;
+  int R2, cpp;
+  row_parts(nch, R2, cpp);
   const size_t e_part = (size_t)Hq * nch * b, e_rs = (size_t)Hq * R2 * b, e_blk = (size_t)Hq * nch;
   const size_t e_ksum = (size_t)Hkv * nch * 128, e_kbar = (size_t)Hkv * n * 128;
   const size_t need = 3 * round256(e_part * 4) + 2 * round256(e_rs * 4) + 2 * round256(e_blk * 4) +
@@ -472,36 +504,14 @@ int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int
   float *LOc = carve<float>(cur, e_blk), *HIc = carve<float>(cur, e_blk);
   float *ksum = carve<float>(cur, e_ksum), *kbar = carve<float>(cur, e_kbar);
 
-  CUtensorMap tq, tk;
-  if (!make_map(&tq, q, I8, (uint64_t)Hq * S) || !make_map(&tk, k, I8, (uint64_t)Hkv * S)) return FP_ERR_CUDA;
-  const int tiles_per_group = g * (b / 128);
-  const int tgroups = (tiles_per_group + 3) / 4;
-  int R = sm_count() / (tgroups * Hkv);
-  if (R < 1) R = 1;
-  if (R > nch) R = nch;
-  const int cpc = (nch + R - 1) / R;
-  R = (nch + cpc - 1) / cpc;
-  ScoreParams sp;
-  sp.S = S; sp.Hq = Hq; sp.Hkv = Hkv; sp.b = b; sp.n = n; sp.nch = nch; sp.g = g;
-  sp.tiles_per_group = tiles_per_group;
-  sp.chunks_per_cta = cpc;
-  sp.scale2 = kLog2e / sqrtf((float)d);
-  sp.q_scale = q_scale;
-  sp.k_scale = k_scale;
-  sp.pm = pm; sp.plo = plo; sp.phi = phi; sp.ksum = ksum;
-  sp.err = err;
-  k_score_last<I8><<<dim3(R, tgroups, Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
-  if ((rc = launch_status())) return rc;
-  k_row_stats<<<dim3(Hq, R2), b, 0, st>>>(pm, plo, phi, nch, b, cpp, partM, partL);
-  if ((rc = launch_status())) return rc;
-  k_block_mass<<<dim3(Hq, R2), b, (size_t)(b / 32) * cpp * 2 * sizeof(float), st>>>(pm, plo, phi, partM, partL,
-                                                                                    nch, b, cpp, LOc, HIc);
-  if ((rc = launch_status())) return rc;
-  k_kbar<<<dim3(n, Hkv), 128, 0, st>>>(ksum, I8 ? k_scale : nullptr, nch, b, n, kbar);
-  if ((rc = launch_status())) return rc;
-  k_pattern<I8><<<Hq, 1024, 0, st>>>(q, q_scale, LOc, HIc, kbar, S, g, b, n, nch, 1.0f / sqrtf((float)d), tau,
-                                     vhat, shat, pest, jsd, pattern);
-  return launch_status();
+  StatsJob J;
+  J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.d = d; J.b = b; J.n = n; J.nch = nch; J.g = Hq / Hkv;
+  J.R2 = R2; J.chunks_per_part = cpp;
+  J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
+  J.pm = pm; J.plo = plo; J.phi = phi; J.partM = partM; J.partL = partL;
+  J.LOc = LOc; J.HIc = HIc; J.ksum = ksum; J.kbar = kbar;
+  J.vhat = vhat; J.shat = shat; J.pest = pest; J.jsd = jsd; J.pattern = pattern;
+  return launch_pattern_stats<I8>(J, err, st);
 }
 
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }

@@ -33,7 +33,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 //
 // CTA = (KV head, group of up to 4 row tiles of 128 query rows of the last
 // block, range of 128-key chunks).  A "tile" is (query head of the group,
-// 128-row slice of the b-row last block).  Warps:
+// 128-row slice of the last block; ceil(nlast/128) slices for its nlast =
+// S - (n-1)b rows, which is fewer than b when b does not divide S).  Rows of
+// a slice past nlast are computed but not stored: every reader of the
+// per-row partials stops at nlast.  Keys at or past S only meet the last
+// block, where the causal mask already hides them from its real rows.
+// Warps:
 //   0..15  statistics: warpgroup t owns tile t; thread = one query row
 //   16     TMA producer     17  MMA issuer + TMEM owner
 //   18     K column sums for the block means (only CTAs of tile group 0)
@@ -42,7 +47,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ---------------------------------------------------------------------------
 struct ScoreParams {
   int S, Hq, Hkv, b, n, nch, g;
-  int tiles_per_group;  // g * b / 128
+  int nlast;            // rows of the last block, S - (n-1)b
+  int tiles_per_head;   // ceil(nlast / 128)
+  int tiles_per_group;  // g * tiles_per_head
   int chunks_per_cta;
   float scale2;          // log2(e)/sqrt(d) (bf16); int8: multiplied by per-head scales
   const float *q_scale;  // int8 only
@@ -82,7 +89,7 @@ __global__ void __launch_bounds__(608, 1)
   const int U = ch1 - ch0;
   const bool do_ksum = (blockIdx.y == 0);
   const int n_ksum_warps = do_ksum ? 1 : 0;
-  const int tiles_per_head = P.b / 128;
+  const int tiles_per_head = P.tiles_per_head;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const uint32_t q_smem = base;                                // 4 tiles
@@ -195,10 +202,11 @@ __global__ void __launch_bounds__(608, 1)
           if (!mbar_wait(smem_u32(&bar_kfull[st]), (u / C::kStages) & 1, abort_flag, P.err)) break;
           const uint8_t *tile = k_gen + st * C::kTileBytes;
           float* out = P.ksum + ((size_t)kvh * P.nch + (ch0 + u)) * 128;
+          const int nrows = min(128, P.S - (ch0 + u) * 128);  // keys of the chunk inside [0, S)
           if (I8) {
             // one 128-byte row per key; lane owns bytes 4*lane .. 4*lane+3
             int acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;
-            for (int r = 0; r < 128; ++r) {
+            for (int r = 0; r < nrows; ++r) {
               const int phys = (((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) << 2);
               const uint32_t w = *reinterpret_cast<const uint32_t *>(tile + r * 128 + phys);
               acc0 += (int)(int8_t)(w & 0xff);
@@ -213,7 +221,7 @@ __global__ void __launch_bounds__(608, 1)
           } else {
             // lane owns columns 2*lane, 2*lane+1 of each 64-column half
             float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
-            for (int r = 0; r < 128; ++r) {
+            for (int r = 0; r < nrows; ++r) {
               const int phys = (((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) << 2);
               const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(tile + r * 128 + phys));
               const float2 e = __bfloat1622float2(
@@ -315,10 +323,12 @@ __global__ void __launch_bounds__(608, 1)
           const float m2 = m * scale2;
           const float lo = (lo4[0] + lo4[1]) + (lo4[2] + lo4[3]);
           const float hi = (hi4[0] + hi4[1]) + (hi4[2] + hi4[3]);
-          const size_t o = ((size_t)hh * P.nch + ch) * P.b + i;
-          P.pm[o] = m2;
-          P.plo[o] = lo;
-          P.phi[o] = hi;
+          if (i < P.nlast) {
+            const size_t o = ((size_t)hh * P.nch + ch) * P.b + i;
+            P.pm[o] = m2;
+            P.plo[o] = lo;
+            P.phi[o] = hi;
+          }
         }
       }
     }
@@ -333,13 +343,14 @@ __global__ void __launch_bounds__(608, 1)
 
 // ---------------------------------------------------------------------------
 // k_row_stats: grid (Hq, R2), block b threads.  Row i's running max M and
-// sum L = sum_chunks (lo + hi) 2^(m - M) over the CTA's chunk range.
+// sum L = sum_chunks (lo + hi) 2^(m - M) over the CTA's chunk range; rows at
+// or past nlast (absent from a partial last block) get M = -inf, L = 0.
 // ---------------------------------------------------------------------------
 __global__ void k_row_stats(const float *__restrict__ pm, const float *__restrict__ plo,
-                            const float *__restrict__ phi, int nch, int b, int chunks_per_part,
+                            const float *__restrict__ phi, int nch, int b, int nlast, int chunks_per_part,
                             float *__restrict__ partM, float *__restrict__ partL) {
   const int h = blockIdx.x, part = blockIdx.y, R2 = gridDim.y, i = threadIdx.x;
-  const int c0 = part * chunks_per_part, c1 = min(nch, c0 + chunks_per_part);
+  const int c0 = part * chunks_per_part, c1 = i < nlast ? min(nch, c0 + chunks_per_part) : c0;
   float M = -INFINITY, L = 0.f;
   for (int ch = c0; ch < c1; ch += 4) {
     // four chunks' loads in flight, then the running combine in order
@@ -375,8 +386,8 @@ __global__ void k_row_stats(const float *__restrict__ pm, const float *__restric
 // ---------------------------------------------------------------------------
 __global__ void k_block_mass(const float *__restrict__ pm, const float *__restrict__ plo,
                              const float *__restrict__ phi, const float *__restrict__ partM,
-                             const float *__restrict__ partL, int nch, int b, int chunks_per_part,
-                             float *__restrict__ LOc, float *__restrict__ HIc) {
+                             const float *__restrict__ partL, int nch, int b, int nlast,
+                             int chunks_per_part, float *__restrict__ LOc, float *__restrict__ HIc) {
   extern __shared__ float red[];  // [nwarps][chunks_per_part][2]
   const int h = blockIdx.x, part = blockIdx.y, R2 = gridDim.y, i = threadIdx.x;
   const int warp = i >> 5, lane = i & 31, nw = blockDim.x >> 5;
@@ -394,7 +405,7 @@ __global__ void k_block_mass(const float *__restrict__ pm, const float *__restri
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const size_t o = ((size_t)h * nch + ch + u) * b + i;
-      const bool in = ch + u < c1;
+      const bool in = i < nlast && ch + u < c1;  // rows past nlast hold no partials
       const float m = in ? pm[o] : -INFINITY;
       const float w = (m == -INFINITY) ? 0.f : ex2(m - M) * invL;
       a[u] = in ? plo[o] * w : 0.f;
@@ -431,23 +442,26 @@ __global__ void k_block_mass(const float *__restrict__ pm, const float *__restri
 }
 
 // ---------------------------------------------------------------------------
-// k_kbar: grid (n, Hkv), block 128: kbar[kvh][c][t] = (1/b) sum of K rows of
-// block c; for int8 keys the exact integer sum times k_scale[kvh].
+// k_kbar: grid (n, Hkv), block 128: kbar[kvh][c][t] = mean of the K rows of
+// block c (b rows, or S - (n-1)b for a partial last block); for int8 keys the
+// exact integer sum times k_scale[kvh].
 // ---------------------------------------------------------------------------
-__global__ void k_kbar(const float *__restrict__ ksum, const float *__restrict__ k_scale, int nch, int b,
-                       int n, float *__restrict__ kbar) {
+__global__ void k_kbar(const float *__restrict__ ksum, const float *__restrict__ k_scale, int S, int nch,
+                       int b, int n, float *__restrict__ kbar) {
   const int c = blockIdx.x, kvh = blockIdx.y, t = threadIdx.x;
-  const int per = b / 128;
+  const int per = b / 128, rows = min(b, S - c * b);
   float s = 0.f;
-  for (int k = 0; k < per; ++k) s += ksum[((size_t)kvh * nch + c * per + k) * 128 + t];
+  for (int k = 0; k < per && c * per + k < nch; ++k) s += ksum[((size_t)kvh * nch + c * per + k) * 128 + t];
   if (k_scale) s *= k_scale[kvh];
-  kbar[((size_t)kvh * n + c) * 128 + t] = s / (float)b;
+  kbar[((size_t)kvh * n + c) * 128 + t] = s / (float)rows;
 }
 
 // ---------------------------------------------------------------------------
-// k_pattern: grid (Hq), block 1024.  vhat[c] = (LO[c] + HI[c]) / b,
-// shat[o] = (LO[n-1-o] + HI[n-2-o]) / b, P_est = softmax_c(qbar_last . kbar_c
-// / sqrt(d)), JSD(vhat, P_est) (natural log), pattern = QA iff JSD < tau.
+// k_pattern: grid (Hq), block 1024.  With nlast = S - (n-1)b rows in the
+// last block: vhat[c] = (LO[c] + HI[c]) / nlast, shat[o] = (LO[n-1-o] +
+// HI[n-2-o]) / nlast, P_est = softmax_c(qbar_last . kbar_c / sqrt(d)) with
+// qbar_last the mean of those nlast rows, JSD(vhat, P_est) (natural log),
+// pattern = QA iff JSD < tau.
 // ---------------------------------------------------------------------------
 template <bool I8>
 __global__ void __launch_bounds__(1024)
@@ -460,16 +474,16 @@ __global__ void __launch_bounds__(1024)
   __shared__ float part[1024 / 32];
   __shared__ float lo_s[1024], hi_s[1024];
   const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int kvh = h / g, per = b / 128;
+  const int kvh = h / g, per = b / 128, nlast = S - (n - 1) * b;
   // block masses
   for (int c = tid; c < n; c += blockDim.x) {
     float a = 0.f, e = 0.f;
-    for (int k = 0; k < per; ++k) {
+    for (int k = 0; k < per && c * per + k < nch; ++k) {
       a += LOc[(size_t)h * nch + c * per + k];
       e += HIc[(size_t)h * nch + c * per + k];
     }
-    lo_s[c] = a / (float)b;
-    hi_s[c] = e / (float)b;
+    lo_s[c] = a / (float)nlast;
+    hi_s[c] = e / (float)nlast;
   }
   // mean of the last block's query rows
   if (tid < 128) {
@@ -477,13 +491,13 @@ __global__ void __launch_bounds__(1024)
     if (I8) {
       const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
       int acc = 0;
-      for (int r = 0; r < b; ++r) acc += q8[base + (size_t)r * 128];
-      qb[tid] = (float)acc * q_scale[h] / (float)b;
+      for (int r = 0; r < nlast; ++r) acc += q8[base + (size_t)r * 128];
+      qb[tid] = (float)acc * q_scale[h] / (float)nlast;
     } else {
       const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(q);
       float acc = 0.f;
-      for (int r = 0; r < b; ++r) acc += __bfloat162float(qh[base + (size_t)r * 128]);
-      qb[tid] = acc / (float)b;
+      for (int r = 0; r < nlast; ++r) acc += __bfloat162float(qh[base + (size_t)r * 128]);
+      qb[tid] = acc / (float)nlast;
     }
   }
   __syncthreads();
@@ -549,8 +563,9 @@ __global__ void __launch_bounds__(1024)
 }
 
 // ---------------------------------------------------------------------------
-// k_qbar: grid (n, Hq), block 256: qbar[h][r][t] = (1/b) sum of Q rows of
-// block r, only for heads whose pattern is query-aware (others exit).
+// k_qbar: grid (n, Hq), block 256: qbar[h][r][t] = mean of the Q rows of
+// block r (b rows, or S - (n-1)b for a partial last block), only for heads
+// whose pattern is query-aware (others exit).
 // ---------------------------------------------------------------------------
 template <bool I8>
 __global__ void __launch_bounds__(256)
@@ -560,6 +575,7 @@ __global__ void __launch_bounds__(256)
   if (pattern[h] != 1) return;
   __shared__ float red[16][128];
   const size_t row0 = (size_t)h * S + (size_t)r * b;
+  const int rows = min(b, S - r * b);
   if (I8) {
     // 8 threads per 128-byte row, 32 rows per pass; thread owns 16 columns
     const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
@@ -567,7 +583,7 @@ __global__ void __launch_bounds__(256)
     int acc[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) acc[e] = 0;
-    for (int p = rr; p < b; p += 32) {
+    for (int p = rr; p < rows; p += 32) {
       const int4 v = *reinterpret_cast<const int4 *>(q8 + (row0 + p) * 128 + c16 * 16);
       const int w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -590,7 +606,7 @@ __global__ void __launch_bounds__(256)
     if (tid < 128) {
       float s = 0.f;
       for (int w = 0; w < 8; ++w) s += red[w][tid];
-      qbar[((size_t)h * n + r) * 128 + tid] = s * q_scale[h] / (float)b;
+      qbar[((size_t)h * n + r) * 128 + tid] = s * q_scale[h] / (float)rows;
     }
   } else {
     // 16 threads per 256-byte row, 16 rows per pass; thread owns 8 columns
@@ -600,7 +616,7 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll 4
-    for (int p = rr; p < b; p += 16) {
+    for (int p = rr; p < rows; p += 16) {
       const uint4 v = *reinterpret_cast<const uint4 *>(qh + (row0 + p) * 128 + c8 * 8);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
@@ -621,7 +637,7 @@ __global__ void __launch_bounds__(256)
     if (tid < 128) {
       float s = 0.f;
       for (int w = 0; w < 8; ++w) s += red[w][tid];
-      qbar[((size_t)h * n + r) * 128 + tid] = s / (float)b;
+      qbar[((size_t)h * n + r) * 128 + tid] = s / (float)rows;
     }
   }
 }

@@ -97,7 +97,7 @@ class Index:
     def __init__(self, handle, S, Hq, Hkv, d, b):
         self.handle = handle
         self.S, self.Hq, self.Hkv, self.d, self.b = S, Hq, Hkv, d, b
-        self.n = S // b
+        self.n = (S + b - 1) // b
 
     def free(self):
         if self.handle:

@@ -18,9 +18,13 @@
  *
  * Conventions (all arguments): batch 1, tensors head-major and contiguous,
  * q[Hq][S][d], k[Hkv][S][d], v[Hkv][S][d], out[Hq][S][d]; query head h reads
- * KV head h / (Hq/Hkv).  Supported: d = 128, b in {128, 256}, S a multiple of
- * b with S/b <= 1024 blocks, Hq a multiple of Hkv.  Device pointers must be
- * 16-byte aligned.  All calls are asynchronous on `stream` (a cudaStream_t,
+ * KV head h / (Hq/Hkv).  Supported: d = 128, b in {128, 256}, any S >= 1 with
+ * n = ceil(S/b) <= 1024 blocks, Hq a multiple of Hkv.  When b does not divide
+ * S the last block is partial: it holds the S - (n-1)b rows (n-1)b .. S-1,
+ * the statistics of steps 1-2 below average over those rows and every block
+ * mean is taken over the rows the block actually has (the articles only
+ * treat whole blocks; this is the reading that keeps every other step
+ * unchanged).  Device pointers must be 16-byte aligned.  All calls are asynchronous on `stream` (a cudaStream_t,
  * NULL = legacy default stream) unless stated; the caller keeps every buffer
  * alive until the stream has passed the call.
  *
@@ -130,7 +134,7 @@ int fp_debug_wait_timeout(int timeout_us, void *stream);
 /* Test hook for the int8 score tiles: computes the exact int32 tile
  * out[i][t] = q8[h][p0 + i] . k8[h/g][j0 + t] for i, t in [0, 128) with the
  * same tensor-core path the int8 kernels use, into device out[128][128].
- * p0, j0 multiples of 128 inside [0, S). */
+ * S a multiple of 128; p0, j0 multiples of 128 inside [0, S). */
 int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int Hkv, int d, int h,
                         int p0, int j0, int32_t *out, void *stream);
 

@@ -38,7 +38,7 @@ def test_strerror(fp):
     assert "timed out" in fp.fp_strerror(fp.FP_ERR_TIMEOUT)
 
 
-@pytest.mark.parametrize("S,Hq,Hkv,d,b", [(1000, 4, 2, 128, 128), (1024, 4, 3, 128, 128), (1024, 4, 2, 64, 128),
+@pytest.mark.parametrize("S,Hq,Hkv,d,b", [(131073, 4, 2, 128, 128), (1024, 4, 3, 128, 128), (1024, 4, 2, 64, 128),
                                            (1024, 4, 2, 128, 64), (0, 4, 2, 128, 128), (262144, 4, 2, 128, 128),
                                            (1024, 0, 2, 128, 128)])
 def test_create_rejects_unsupported_shapes(fp, S, Hq, Hkv, d, b):

@@ -52,29 +52,35 @@ def oracle_problem(x, w):
     return orc.OracleProblem(x["q"], x["k"], x["v"], w.b)
 
 
+def nblocks(S, b):
+    return -(-S // b)
+
+
 def check_index(P, exp, w):
+    n = nblocks(w.S, w.b)
     heads = parity.run_parallel(lambda h: P.build_index_head(h, w.gamma, w.tau), range(w.Hq))
-    stats = parity.compare_index(exp, heads, w.S // w.b, w.gamma, w.tau,
+    stats = parity.compare_index(exp, heads, n, w.gamma, w.tau,
                                  oracle_forced=lambda h, pat: P.build_index_head(h, w.gamma, w.tau, pat))
     print(f"[{w.name}] index: {stats}; patterns {exp['pattern'].tolist()}; "
-          f"density {exp['nnz'] / (w.Hq * (w.S // w.b) * (w.S // w.b + 1) / 2):.4f}")
+          f"density {exp['nnz'] / (w.Hq * n * (n + 1) / 2):.4f}")
     return heads, stats
 
 
 def check_tiles(P, exp, out, w, tiles):
-    n = w.S // w.b
+    """Query tiles (h, qc) of 128 rows; the last one stops at S."""
+    n = nblocks(w.S, w.b)
 
     def one(t):
         h, qc = t
         r = qc * 128 // w.b
         rows = parity.gpu_rows(exp, h, n)[r]
-        ref = P.attn_rows(h, qc * 128, qc * 128 + 128, rows)
+        ref = P.attn_rows(h, qc * 128, min(qc * 128 + 128, w.S), rows)
         return ref
 
     refs = parity.run_parallel(one, tiles)
     worst_max, sum_mean = 0.0, 0.0
     for (h, qc), ref in zip(tiles, refs):
-        got = out[h, qc * 128: qc * 128 + 128].float().cpu().numpy()
+        got = out[h, qc * 128: min(qc * 128 + 128, w.S)].float().cpu().numpy()
         mx, mean = parity.compare_tile(got, ref)
         assert mx <= parity.OUT_MAX_ABS and mean <= parity.OUT_MEAN_ABS, (h, qc, mx, mean)
         worst_max = max(worst_max, mx)
@@ -94,6 +100,14 @@ SMALL = [
     synth.Workload("two_blocks_tau0", S=256, Hq=2, Hkv=1, b=128, tau=0.0, seed=12),
     synth.Workload("int8_small", S=2048, Hq=4, Hkv=2, b=128, int8=True, seed=9),
     synth.Workload("int8_b256", S=2048, Hq=4, Hkv=1, b=256, gamma=0.95, int8=True, seed=10),
+    # lengths that b (and 128) do not divide: a partial last block
+    synth.Workload("ragged_b128", S=1000, Hq=4, Hkv=2, b=128, seed=16),
+    synth.Workload("ragged_b256_short_tail", S=1300, Hq=6, Hkv=2, b=256, seed=17),
+    synth.Workload("ragged_b256_long_tail", S=1500, Hq=4, Hkv=1, b=256, gamma=0.95, seed=18),
+    synth.Workload("ragged_one_row_tail", S=129, Hq=2, Hkv=1, b=128, seed=19),
+    synth.Workload("ragged_single_block", S=77, Hq=2, Hkv=2, b=256, seed=20),
+    synth.Workload("ragged_int8", S=2000, Hq=4, Hkv=2, b=128, int8=True, seed=21),
+    synth.Workload("ragged_int8_b256", S=1800, Hq=4, Hkv=2, b=256, gamma=0.95, int8=True, seed=22),
 ]
 
 
@@ -103,7 +117,7 @@ def test_small_layers_full_parity(fp, w):
     exp, out, idx = run_gpu(fp, x, w)
     P = oracle_problem(x, w)
     check_index(P, exp, w)
-    tiles = [(h, qc) for h in range(w.Hq) for qc in range(w.S // 128)]
+    tiles = [(h, qc) for h in range(w.Hq) for qc in range(nblocks(w.S, 128))]
     check_tiles(P, exp, out, w, tiles)
 
 
@@ -111,7 +125,9 @@ DENSE = [synth.Workload("dense", S=2048, Hq=8, Hkv=2, b=128, gamma=1.0, seed=13)
          synth.Workload("sweep_gen_b128", S=4096, Hq=32, Hkv=8, b=128, gamma=1.0, n_vertical=64, n_topics=32,
                         seed=2),
          synth.Workload("sweep_gen_b256", S=4096, Hq=32, Hkv=8, b=256, gamma=1.0, n_vertical=64, n_topics=32,
-                        seed=2)]
+                        seed=2),
+         synth.Workload("dense_ragged_b128", S=1234, Hq=8, Hkv=2, b=128, gamma=1.0, seed=23),
+         synth.Workload("dense_ragged_b256", S=1234, Hq=8, Hkv=2, b=256, gamma=1.0, seed=23)]
 
 
 @pytest.mark.parametrize("w", DENSE, ids=[w.name for w in DENSE])
@@ -120,7 +136,7 @@ def test_gamma_one_matches_dense_sdpa(fp, w):
     (checked against torch SDPA in fp32 on the GPU)."""
     x = synth.make_inputs(w)
     exp, out, idx = run_gpu(fp, x, w)
-    n = w.S // w.b
+    n = nblocks(w.S, w.b)
     g = w.Hq // w.Hkv
     assert exp["nnz"] == w.Hq * n * (n + 1) // 2
     q, k, v = (x[t].cuda().float() for t in ("q", "k", "v"))
@@ -155,7 +171,7 @@ def test_bounded_wait_reports_timeout_and_context_survives(fp):
 
 def sampled_tiles(w, count, seed):
     rng = random.Random(seed)
-    nq = w.S // 128
+    nq = nblocks(w.S, 128)
     tiles = {(h, nq - 1) for h in range(0, w.Hq, max(1, w.Hq // 4))}      # longest rows
     while len(tiles) < count:
         tiles.add((rng.randrange(w.Hq), rng.randrange(nq)))

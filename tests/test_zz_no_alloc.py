@@ -29,7 +29,7 @@ def reference_stats(fp, x, w, qq, kk, qs, ks, dt):
 
 
 def noalloc_stats(fp, w, qq, kk, qs, ks, dt):
-    n = w.S // w.b
+    n = -(-w.S // w.b)
     dev = qq.device
     vhat = torch.full((w.Hq, n), float("nan"), device=dev)
     shat = torch.full((w.Hq, n), float("nan"), device=dev)
@@ -57,6 +57,7 @@ def test_noalloc_statistics_match_build_index_on_consecutive_calls():
     cases = [synth.WORKLOADS["tiny"],
              synth.Workload("noalloc_b256_int8", S=8192, Hq=8, Hkv=2, b=256, int8=True, seed=21),
              synth.Workload("noalloc_llama3b_shape", S=32768, Hq=32, Hkv=8, b=128, seed=22),
+             synth.Workload("noalloc_ragged", S=1500, Hq=4, Hkv=2, b=256, seed=24),
              synth.WORKLOADS["tiny"]]
     for w in cases:      # consecutive calls share (and overwrite) the fixed scratch
         x, qq, kk, qs, ks, dt = inputs(fp, w)
