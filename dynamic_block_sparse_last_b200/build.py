@@ -9,9 +9,9 @@ import sys
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
-SRC = os.path.join(PKG, "csrc", "fp_sparse.cu")
-DEPS = [os.path.join(PKG, "csrc", f) for f in ("fp_sparse.cu", "ptx.cuh", "index_kernels.cuh", "attn_kernel.cuh")] \
-    + [os.path.join(ROOT, "include", "fp_sparse.h")]
+SRCS = [os.path.join(PKG, "csrc", f) for f in ("fp_sparse.cu", "fp_prefill.cpp")]
+DEPS = SRCS + [os.path.join(PKG, "csrc", f) for f in ("ptx.cuh", "index_kernels.cuh", "attn_kernel.cuh")] \
+    + [os.path.join(ROOT, "include", f) for f in ("fp_sparse.h", "fp_prefill.h")]
 LIB = os.path.join(PKG, "_lib", "libfpsparse.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc" if os.path.exists("/usr/local/cuda/bin/nvcc") else "nvcc")
 
@@ -23,7 +23,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         return LIB
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [NVCC, "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
-           "-Xcompiler", "-fPIC", "-shared", "-I" + os.path.join(ROOT, "include"), SRC, "-o", tmp]
+           "-Xcompiler", "-fPIC", "-shared", "-I" + os.path.join(ROOT, "include"), *SRCS, "-o", tmp]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)

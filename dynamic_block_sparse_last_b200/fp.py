@@ -20,7 +20,9 @@ FP_PATTERN_VS, FP_PATTERN_QA = 0, 1
 
 SYMBOLS = ("fp_index_create", "fp_index_free", "fp_build_index", "fp_sparse_attn", "fp_index_info",
            "fp_index_nnz", "fp_index_export", "fp_get_device_error", "fp_debug_wait_timeout",
-           "fp_debug_qk_tile_i8", "fp_pattern_stats_noalloc", "fp_strerror")
+           "fp_debug_qk_tile_i8", "fp_pattern_stats_noalloc", "fp_strerror",
+           "fp_prefill_create", "fp_prefill_free", "fp_prefill_enqueue", "fp_prefill_wait", "fp_prefill_run",
+           "fp_prefill_group_index")
 
 
 class FpError(RuntimeError):
@@ -49,8 +51,15 @@ def _load():
     L.fp_pattern_stats_noalloc.argtypes = [vp, vp, i, i, i, i, i, f, i, vp, vp, vp, vp, vp, vp, vp, vp]
     L.fp_strerror.argtypes = [i]
     L.fp_strerror.restype = ctypes.c_char_p
+    L.fp_prefill_create.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(vp)]
+    L.fp_prefill_free.argtypes = [vp]
+    L.fp_prefill_free.restype = None
+    L.fp_prefill_run.argtypes = [vp, vp, vp, vp, vp, vp, f, f, vp, vp]
+    L.fp_prefill_enqueue.argtypes = [vp, vp, vp, vp, vp, vp, f, f, vp, vp]
+    L.fp_prefill_wait.argtypes = [vp, vp]
+    L.fp_prefill_group_index.argtypes = [vp, i, ctypes.POINTER(vp)]
     for s in SYMBOLS:
-        if s != "fp_index_free" and s != "fp_strerror":
+        if s not in ("fp_index_free", "fp_strerror", "fp_prefill_free"):
             getattr(L, s).restype = i
     return L
 
@@ -183,3 +192,52 @@ def fp_pattern_stats_noalloc(q, k, S, Hq, Hkv, d, b, tau, qk_dtype, q_scale, k_s
     _check(_lib.fp_pattern_stats_noalloc(_ptr(q), _ptr(k), S, Hq, Hkv, d, b, float(tau), int(qk_dtype),
                                          _ptr(q_scale), _ptr(k_scale), _ptr(vhat), _ptr(shat), _ptr(pest),
                                          _ptr(jsd), _ptr(pattern), _stream(stream)), "fp_pattern_stats_noalloc")
+
+
+class Prefill:
+    """Owns one fp_prefill pipeline (include/fp_prefill.h): device copies of a
+    layer and one index per KV-head group, for host-to-host runs."""
+
+    def __init__(self, S, Hq, Hkv, d, b, qk_dtype=FP_QK_BF16, groups=0):
+        h = ctypes.c_void_p()
+        _check(_lib.fp_prefill_create(S, Hq, Hkv, d, b, int(qk_dtype), int(groups), ctypes.byref(h)),
+               "fp_prefill_create")
+        self.handle = h.value
+        self.S, self.Hq, self.Hkv, self.d, self.b, self.qk_dtype = S, Hq, Hkv, d, b, qk_dtype
+        self.groups = groups if groups else Hkv
+
+    def run(self, h_q, h_k, h_v, h_q_scale, h_k_scale, gamma, tau, h_out, stream=None):
+        """Host tensors in, host tensor out (pinned for overlap); asynchronous on `stream`."""
+        _check(_lib.fp_prefill_run(self.handle, _ptr(h_q), _ptr(h_k), _ptr(h_v), _ptr(h_q_scale),
+                                   _ptr(h_k_scale), float(gamma), float(tau), _ptr(h_out), _stream(stream)),
+               "fp_prefill_run")
+
+    def enqueue(self, h_q, h_k, h_v, h_q_scale, h_k_scale, gamma, tau, h_out, stream=None):
+        """Queues a run; consecutive runs overlap.  h_out is ready after wait()."""
+        _check(_lib.fp_prefill_enqueue(self.handle, _ptr(h_q), _ptr(h_k), _ptr(h_v), _ptr(h_q_scale),
+                                       _ptr(h_k_scale), float(gamma), float(tau), _ptr(h_out), _stream(stream)),
+               "fp_prefill_enqueue")
+
+    def wait(self, stream=None):
+        """Makes `stream` wait for the outputs of every queued run."""
+        _check(_lib.fp_prefill_wait(self.handle, _stream(stream)), "fp_prefill_wait")
+
+    def group_index(self, group):
+        """The fp_index of KV-head group `group` of the last run (owned by the pipeline)."""
+        h = ctypes.c_void_p()
+        _check(_lib.fp_prefill_group_index(self.handle, int(group), ctypes.byref(h)), "fp_prefill_group_index")
+        hkv = self.Hkv // self.groups if self.groups <= self.Hkv else 1
+        idx = Index(h.value, self.S, self.Hq // self.groups, hkv, self.d, self.b)
+        idx.free = lambda: None  # owned by the pipeline
+        return idx
+
+    def free(self):
+        if self.handle:
+            _lib.fp_prefill_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass

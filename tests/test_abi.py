@@ -1,6 +1,6 @@
 """The C ABI library without a GPU: it loads, exports every function that
-include/fp_sparse.h declares, and rejects bad arguments on the host before
-any CUDA call."""
+include/*.h declares, and rejects bad arguments on the host before any CUDA
+call."""
 import ctypes
 import os
 import re
@@ -19,14 +19,18 @@ def fp():
 
 
 def declared_functions():
-    src = open(os.path.join(ROOT, "include", "fp_sparse.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(fp_[a-z0-9_]+)\s*\(", src)))
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            src = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, f)).read(), flags=re.S)
+            names |= set(re.findall(r"\b(fp_[a-z0-9_]+)\s*\(", src))
+    return sorted(names)
 
 
 def test_every_declared_symbol_is_exported(fp):
     names = declared_functions()
-    assert "fp_build_index" in names and "fp_sparse_attn" in names
+    assert "fp_build_index" in names and "fp_sparse_attn" in names and "fp_prefill_run" in names
     lib = ctypes.CDLL(fp.library_path())
     for name in names:
         assert hasattr(lib, name), name
@@ -60,3 +64,22 @@ def test_calls_reject_null_and_misaligned_pointers(fp):
 
 def test_index_info_rejects_null(fp):
     assert fp.lib().fp_index_info(None, None, None, None, None, None, None) == fp.FP_ERR_ARG
+
+
+@pytest.mark.parametrize("S,Hq,Hkv,d,b,dt,groups", [(1024, 4, 2, 128, 128, 0, 3), (1024, 4, 2, 128, 128, 0, -1),
+                                                   (1024, 4, 2, 128, 128, 0, 6), (1024, 6, 2, 128, 128, 0, 4),
+                                                   (1024, 4, 2, 128, 128, 2, 0),
+                                                   (1024, 4, 2, 64, 128, 0, 0), (131073, 4, 2, 128, 128, 0, 0)])
+def test_prefill_create_rejects_bad_arguments(fp, S, Hq, Hkv, d, b, dt, groups):
+    h = ctypes.c_void_p()
+    assert fp.lib().fp_prefill_create(S, Hq, Hkv, d, b, dt, groups, ctypes.byref(h)) == fp.FP_ERR_ARG
+    assert h.value is None
+
+
+def test_prefill_run_rejects_null_before_any_cuda_call(fp):
+    L = fp.lib()
+    assert L.fp_prefill_run(None, 16, 16, 16, None, None, 0.9, 0.1, 16, None) == fp.FP_ERR_ARG
+    assert L.fp_prefill_enqueue(None, 16, 16, 16, None, None, 0.9, 0.1, 16, None) == fp.FP_ERR_ARG
+    assert L.fp_prefill_wait(None, None) == fp.FP_ERR_ARG
+    assert L.fp_prefill_group_index(None, 0, None) == fp.FP_ERR_ARG
+    L.fp_prefill_free(None)
