@@ -13,9 +13,10 @@
 // The CTA walks the union of the two tiles' chunk lists (ascending 128-key
 // chunks); a chunk only one tile needs is computed for that tile only.
 // When 128 does not divide S the last query tile and the last key chunk run
-// past S: the tensor maps read whatever follows (the next head's rows, or
-// zeros past the end of the tensor), the causal mask keeps those keys away
-// from every real row, and rows at or past S are not stored.
+// past S: the tensor maps read whatever follows (the next head's or the next
+// packed sequence's rows, or zeros past the end of the tensor), the causal
+// mask keeps those keys away from every real row, and rows at or past S are
+// not stored.
 // CTAs are numbered KV-head-major (all CTAs of one KV head together, so its
 // K and V stay in L2 while they run; the GPU analogue of the article's
 // KV-block-major schedule, section 3.2) and heavy first (descending query
@@ -46,6 +47,7 @@ namespace fpk {
 
 struct AttnParams {
   int S, Hq, Hkv, b, n, g;
+  int ld;             // rows from one head to the next (S, or more for packed sequences)
   const int *counts;  // [Hq][n]
   const int *cols;    // padded lists, row (h, r) at h*n(n+1)/2 + r(r+1)/2
   const float *q_scale, *k_scale;  // int8 only
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(608, 1)
       const int nt = tl[1].valid ? 2 : 1;
       mbar_expect_tx(smem_u32(&bar_q), nt * C::kQKTile);
       for (int t = 0; t < nt; ++t) {
-        const int qrow = tl[t].h * P.S + tl[t].qc * 128;
+        const int qrow = tl[t].h * P.ld + tl[t].qc * 128;
         const uint32_t dst = sq + t * C::kQKTile;
         tma_load_2d(dst, &tm_q, 0, qrow, smem_u32(&bar_q));
         if (!I8) tma_load_2d(dst + 16384, &tm_q, 64, qrow, smem_u32(&bar_q));
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(608, 1)
       wk.init(chunk_bm[0], chunk_bm[1], words);
       int kc, mask;
       for (int u = 0; wk.next(kc, mask); ++u) {
-        const int st = u % C::kKStages, krow = kvh * P.S + kc * 128;
+        const int st = u % C::kKStages, krow = kvh * P.ld + kc * 128;
         if (u >= C::kKStages &&
             !mbar_wait(smem_u32(&bar_kempty[st]), ((u / C::kKStages) - 1) & 1, abort_flag, P.err))
           break;
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(608, 1)
       wv.init(chunk_bm[0], chunk_bm[1], words);
       int kc, mask;
       for (int u = 0; wv.next(kc, mask); ++u) {
-        const int st = u % C::kVStages, vrow = kvh * P.S + kc * 128;
+        const int st = u % C::kVStages, vrow = kvh * P.ld + kc * 128;
         if (u >= C::kVStages &&
             !mbar_wait(smem_u32(&bar_vempty[st]), ((u / C::kVStages) - 1) & 1, abort_flag, P.err))
           break;
@@ -464,8 +466,8 @@ __global__ void __launch_bounds__(608, 1)
       if (lane == 0) mbar_arrive(xbar);
       if (mbar_wait(xbar, L & 1, abort_flag, P.err)) {
         const float inv = 1.f / (l + xl[t][ch ^ 1][row]);
-        const bool store = me.qc * 128 + row < P.S;  // rows past S belong to the next head
-        __nv_bfloat16 *orow = P.out + ((size_t)me.h * P.S + (size_t)me.qc * 128 + row) * 128 + ch * 64;
+        const bool store = me.qc * 128 + row < P.S;  // rows past S belong to a neighbour
+        __nv_bfloat16 *orow = P.out + ((size_t)me.h * P.ld + (size_t)me.qc * 128 + row) * 128 + ch * 64;
 #pragma unroll 1
         for (int qq = 0; qq < 2; ++qq) {
           uint32_t o[32];

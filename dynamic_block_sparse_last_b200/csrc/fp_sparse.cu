@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <new>
 #include <vector>
 
 #include "attn_kernel.cuh"
@@ -23,6 +24,7 @@ static __device__ int g_fp_dev_error;
 
 struct fp_index {
   int S, Hq, Hkv, d, b, n, nch, g;
+  int ld;                  // rows from one head to the next in q, k, v, out (S, or T when packed)
   int device;
   int built;
   int qk_dtype;
@@ -74,7 +76,9 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D map over a [rows][128] tensor: boxes of 128 rows x 128 bytes
-// (64 bf16 or 128 int8 columns), 128-byte swizzle.
+// (64 bf16 or 128 int8 columns), 128-byte swizzle.  For H heads of S rows
+// spaced ld rows apart the map covers (H-1)*ld + S rows from the first head's
+// first row, so no box reads past the last head's last row.
 bool make_map(CUtensorMap *m, const void *ptr, bool i8, uint64_t rows) {
   auto enc = encode_fn();
   if (!enc) return false;
@@ -88,6 +92,8 @@ bool make_map(CUtensorMap *m, const void *ptr, bool i8, uint64_t rows) {
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+uint64_t map_rows(int H, int ld, int S) { return (uint64_t)(H - 1) * (uint64_t)ld + (uint64_t)S; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -136,6 +142,7 @@ int set_smem_attrs() {
 // fp_build_index), shared by the index build and the allocation-free call.
 struct StatsJob {
   int S, Hq, Hkv, d, b, n, nch, g, R2, chunks_per_part;
+  int ld;  // rows from one head to the next
   const void *q, *k;
   const float *q_scale, *k_scale;  // int8 only
   float tau;
@@ -149,7 +156,7 @@ template <bool I8>
 int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   int rc;
   CUtensorMap tq, tk;
-  if (!make_map(&tq, J.q, I8, (uint64_t)J.Hq * J.S) || !make_map(&tk, J.k, I8, (uint64_t)J.Hkv * J.S))
+  if (!make_map(&tq, J.q, I8, map_rows(J.Hq, J.ld, J.S)) || !make_map(&tk, J.k, I8, map_rows(J.Hkv, J.ld, J.S)))
     return FP_ERR_CUDA;
   const int nlast = J.S - (J.n - 1) * J.b;  // rows of the (possibly partial) last block
   const int tiles_per_head = (nlast + 127) / 128;
@@ -162,6 +169,7 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   R = (J.nch + cpc - 1) / cpc;
   ScoreParams sp;
   sp.S = J.S; sp.Hq = J.Hq; sp.Hkv = J.Hkv; sp.b = J.b; sp.n = J.n; sp.nch = J.nch; sp.g = J.g;
+  sp.ld = J.ld;
   sp.nlast = nlast;
   sp.tiles_per_head = tiles_per_head;
   sp.tiles_per_group = tiles_per_group;
@@ -182,7 +190,7 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   if ((rc = launch_status())) return rc;
   k_kbar<<<dim3(J.n, J.Hkv), 128, 0, st>>>(J.ksum, I8 ? J.k_scale : nullptr, J.S, J.nch, J.b, J.n, J.kbar);
   if ((rc = launch_status())) return rc;
-  k_pattern<I8><<<J.Hq, 1024, 0, st>>>(J.q, J.q_scale, J.LOc, J.HIc, J.kbar, J.S, J.g, J.b, J.n, J.nch,
+  k_pattern<I8><<<J.Hq, 1024, 0, st>>>(J.q, J.q_scale, J.LOc, J.HIc, J.kbar, J.S, J.ld, J.g, J.b, J.n, J.nch,
                                        1.0f / sqrtf((float)J.d), J.tau, J.vhat, J.shat, J.pest, J.jsd,
                                        J.pattern);
   return launch_status();
@@ -204,14 +212,14 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   if (!err) return FP_ERR_CUDA;
   StatsJob J;
   J.S = I->S; J.Hq = I->Hq; J.Hkv = I->Hkv; J.d = I->d; J.b = I->b; J.n = I->n; J.nch = I->nch; J.g = I->g;
-  J.R2 = I->R2; J.chunks_per_part = I->chunks_per_part;
+  J.R2 = I->R2; J.chunks_per_part = I->chunks_per_part; J.ld = I->ld;
   J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
   J.pm = I->pm; J.plo = I->plo; J.phi = I->phi; J.partM = I->partM; J.partL = I->partL;
   J.LOc = I->LOc; J.HIc = I->HIc; J.ksum = I->ksum; J.kbar = I->kbar;
   J.vhat = I->vhat; J.shat = I->shat; J.pest = I->pest; J.jsd = I->jsd; J.pattern = I->pattern;
   if ((rc = launch_pattern_stats<I8>(J, err, st))) return rc;
   const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
-  k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->b, I->n, I->qbar);
+  k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->ld, I->b, I->n, I->qbar);
   if ((rc = launch_status())) return rc;
   const int nt = (I->n + kLgTile - 1) / kLgTile;
   k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, I->qbar, I->kbar, I->g, I->n,
@@ -230,11 +238,11 @@ int attn_impl(const void *q, const void *k, const void *v, const float *q_scale,
   int *err = device_error_word();
   if (!err) return FP_ERR_CUDA;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, I8, (uint64_t)I->Hq * I->S) || !make_map(&tk, k, I8, (uint64_t)I->Hkv * I->S) ||
-      !make_map(&tv, v, false, (uint64_t)I->Hkv * I->S))
+  if (!make_map(&tq, q, I8, map_rows(I->Hq, I->ld, I->S)) || !make_map(&tk, k, I8, map_rows(I->Hkv, I->ld, I->S)) ||
+      !make_map(&tv, v, false, map_rows(I->Hkv, I->ld, I->S)))
     return FP_ERR_CUDA;
   AttnParams ap;
-  ap.S = I->S; ap.Hq = I->Hq; ap.Hkv = I->Hkv; ap.b = I->b; ap.n = I->n; ap.g = I->g;
+  ap.S = I->S; ap.Hq = I->Hq; ap.Hkv = I->Hkv; ap.b = I->b; ap.n = I->n; ap.g = I->g; ap.ld = I->ld;
   ap.counts = I->counts;
   ap.cols = I->cols;
   ap.q_scale = q_scale;
@@ -251,13 +259,18 @@ int attn_impl(const void *q, const void *k, const void *v, const float *q_scale,
 
 extern "C" {
 
-int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out) {
+}  // extern "C"
+
+namespace {
+
+// Index for one sequence of S rows per head, heads ld rows apart.
+int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   if (!out) return FP_ERR_ARG;
   *out = nullptr;
-  if (!shape_ok(S, Hq, Hkv, d, b)) return FP_ERR_ARG;
+  if (!shape_ok(S, Hq, Hkv, d, b) || ld < S || (int64_t)Hq * ld > (int64_t)INT32_MAX) return FP_ERR_ARG;
   fp_index *I = static_cast<fp_index *>(calloc(1, sizeof(fp_index)));
   if (!I) return FP_ERR_CUDA;
-  I->S = S; I->Hq = Hq; I->Hkv = Hkv; I->d = d; I->b = b;
+  I->S = S; I->Hq = Hq; I->Hkv = Hkv; I->d = d; I->b = b; I->ld = ld;
   I->n = (S + b - 1) / b; I->nch = (S + 127) / 128; I->g = Hq / Hkv;
   row_parts(I->nch, I->R2, I->chunks_per_part);
   cudaGetDevice(&I->device);
@@ -305,6 +318,14 @@ int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out) {
   return FP_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out) {
+  return index_create(S, S, Hq, Hkv, d, b, out);
+}
+
 void fp_index_free(fp_index *I) {
   if (!I) return;
   cudaDeviceSynchronize();
@@ -318,6 +339,7 @@ int fp_build_index(const void *q, const void *k, int S, int Hq, int Hkv, int d, 
   if (!idx || !q || !k) return FP_ERR_ARG;
   if (!shape_ok(S, Hq, Hkv, d, b)) return FP_ERR_ARG;
   if (S != idx->S || Hq != idx->Hq || Hkv != idx->Hkv || d != idx->d || b != idx->b) return FP_ERR_STATE;
+  if (idx->ld != idx->S) return FP_ERR_STATE;  // an index of a packed set: fp_varlen_* calls only
   if (!(gamma > 0.f && gamma <= 1.f) || !(tau >= 0.f) || std::isnan(gamma) || std::isnan(tau)) return FP_ERR_ARG;
   if (qk_dtype != FP_QK_BF16 && qk_dtype != FP_QK_INT8) return FP_ERR_ARG;
   if (qk_dtype == FP_QK_INT8 && (!q_scale || !k_scale)) return FP_ERR_ARG;
@@ -336,7 +358,7 @@ int fp_build_index(const void *q, const void *k, int S, int Hq, int Hkv, int d, 
 int fp_sparse_attn(const void *q, const void *k, const void *v, const float *q_scale, const float *k_scale,
                    const fp_index *idx, void *out, void *stream) {
   if (!idx || !q || !k || !v || !out) return FP_ERR_ARG;
-  if (!idx->built) return FP_ERR_STATE;
+  if (!idx->built || idx->ld != idx->S) return FP_ERR_STATE;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FP_ERR_ARG;
   if (idx->qk_dtype == FP_QK_INT8 && (!q_scale || !k_scale)) return FP_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -506,7 +528,7 @@ int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int
 
   StatsJob J;
   J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.d = d; J.b = b; J.n = n; J.nch = nch; J.g = Hq / Hkv;
-  J.R2 = R2; J.chunks_per_part = cpp;
+  J.R2 = R2; J.chunks_per_part = cpp; J.ld = S;
   J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
   J.pm = pm; J.plo = plo; J.phi = phi; J.partM = partM; J.partL = partL;
   J.LOc = LOc; J.HIc = HIc; J.ksum = ksum; J.kbar = kbar;
@@ -548,6 +570,117 @@ const char *fp_strerror(int code) {
     case FP_ERR_STATE: return "index not built or built for another shape";
     default: return "unknown error";
   }
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Packed variable-length sequences: one index per sequence over strided views
+// of the packed [H][T][d] tensors (heads T rows apart, sequence s at rows
+// cu_seqlens[s] .. cu_seqlens[s+1]-1 of every head).
+// ---------------------------------------------------------------------------
+struct fp_varlen {
+  int nseq, T, Hq, Hkv, d, b;
+  std::vector<int> cu;              // nseq + 1 offsets
+  std::vector<fp_index *> idx;      // nullptr for empty sequences
+  int built, qk_dtype;
+};
+
+extern "C" {
+
+void fp_varlen_free(fp_varlen *V) {
+  if (!V) return;
+  for (fp_index *I : V->idx) fp_index_free(I);
+  delete V;
+}
+
+int fp_varlen_create(const int32_t *cu_seqlens, int nseq, int Hq, int Hkv, int d, int b, fp_varlen **out) {
+  if (!out) return FP_ERR_ARG;
+  *out = nullptr;
+  if (!cu_seqlens || nseq <= 0 || cu_seqlens[0] != 0) return FP_ERR_ARG;
+  for (int s = 0; s < nseq; ++s) {
+    const int len = cu_seqlens[s + 1] - cu_seqlens[s];
+    if (len < 0 || (len > 0 && !shape_ok(len, Hq, Hkv, d, b))) return FP_ERR_ARG;
+  }
+  const int T = cu_seqlens[nseq];
+  if (T <= 0 || !shape_ok(1, Hq, Hkv, d, b) || (int64_t)Hq * T > (int64_t)INT32_MAX) return FP_ERR_ARG;
+  fp_varlen *V = new (std::nothrow) fp_varlen();
+  if (!V) return FP_ERR_CUDA;
+  V->nseq = nseq; V->T = T; V->Hq = Hq; V->Hkv = Hkv; V->d = d; V->b = b;
+  V->cu.assign(cu_seqlens, cu_seqlens + nseq + 1);
+  V->idx.assign(nseq, nullptr);
+  V->built = 0;
+  V->qk_dtype = FP_QK_BF16;
+  for (int s = 0; s < nseq; ++s) {
+    const int len = V->cu[s + 1] - V->cu[s];
+    if (len == 0) continue;
+    const int rc = index_create(len, T, Hq, Hkv, d, b, &V->idx[s]);
+    if (rc) {
+      fp_varlen_free(V);
+      return rc;
+    }
+  }
+  *out = V;
+  return FP_OK;
+}
+
+int fp_varlen_build_index(fp_varlen *V, const void *q, const void *k, float gamma, float tau, int qk_dtype,
+                          const float *q_scale, const float *k_scale, void *stream) {
+  if (!V || !q || !k) return FP_ERR_ARG;
+  if (!(gamma > 0.f && gamma <= 1.f) || !(tau >= 0.f) || std::isnan(gamma) || std::isnan(tau)) return FP_ERR_ARG;
+  if (qk_dtype != FP_QK_BF16 && qk_dtype != FP_QK_INT8) return FP_ERR_ARG;
+  const bool i8 = qk_dtype == FP_QK_INT8;
+  if (i8 && (!q_scale || !k_scale)) return FP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k)) return FP_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t elt = i8 ? 1 : 2;
+  V->built = 0;
+  for (int s = 0; s < V->nseq; ++s) {
+    fp_index *I = V->idx[s];
+    if (!I) continue;
+    const size_t off = (size_t)V->cu[s] * V->d * elt;  // bytes to the sequence's first row in head 0
+    const void *qs = static_cast<const char *>(q) + off, *ks = static_cast<const char *>(k) + off;
+    I->built = 0;
+    const int rc = i8 ? build_index_impl<true>(qs, ks, gamma, tau, q_scale + (size_t)s * V->Hq,
+                                               k_scale + (size_t)s * V->Hkv, I, st)
+                      : build_index_impl<false>(qs, ks, gamma, tau, nullptr, nullptr, I, st);
+    if (rc) return rc;
+    I->built = 1;
+    I->qk_dtype = qk_dtype;
+  }
+  V->built = 1;
+  V->qk_dtype = qk_dtype;
+  return FP_OK;
+}
+
+int fp_varlen_sparse_attn(const fp_varlen *V, const void *q, const void *k, const void *v, const float *q_scale,
+                          const float *k_scale, void *out, void *stream) {
+  if (!V || !q || !k || !v || !out) return FP_ERR_ARG;
+  if (!V->built) return FP_ERR_STATE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return FP_ERR_ARG;
+  const bool i8 = V->qk_dtype == FP_QK_INT8;
+  if (i8 && (!q_scale || !k_scale)) return FP_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t elt = i8 ? 1 : 2;
+  for (int s = 0; s < V->nseq; ++s) {
+    const fp_index *I = V->idx[s];
+    if (!I) continue;
+    const size_t row = (size_t)V->cu[s] * V->d;
+    const void *qs = static_cast<const char *>(q) + row * elt, *ks = static_cast<const char *>(k) + row * elt;
+    const void *vs = static_cast<const char *>(v) + row * 2;
+    void *os = static_cast<char *>(out) + row * 2;
+    const int rc = i8 ? attn_impl<true>(qs, ks, vs, q_scale + (size_t)s * V->Hq, k_scale + (size_t)s * V->Hkv, I,
+                                        os, st)
+                      : attn_impl<false>(qs, ks, vs, nullptr, nullptr, I, os, st);
+    if (rc) return rc;
+  }
+  return FP_OK;
+}
+
+int fp_varlen_index(const fp_varlen *V, int seq, const fp_index **out) {
+  if (!V || !out || seq < 0 || seq >= V->nseq) return FP_ERR_ARG;
+  *out = V->idx[seq];
+  return FP_OK;
 }
 
 }  // extern "C"

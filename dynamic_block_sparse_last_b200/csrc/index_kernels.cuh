@@ -47,6 +47,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ---------------------------------------------------------------------------
 struct ScoreParams {
   int S, Hq, Hkv, b, n, nch, g;
+  int ld;               // rows from one head to the next (S, or more for packed sequences)
   int nlast;            // rows of the last block, S - (n-1)b
   int tiles_per_head;   // ceil(nlast / 128)
   int tiles_per_group;  // g * tiles_per_head
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(608, 1)
         for (int t = 0; t < T; ++t) {
           const int tile = tg0 + t;
           const int hh = kvh * P.g + tile / tiles_per_head;
-          const int row = hh * P.S + (P.n - 1) * P.b + (tile % tiles_per_head) * 128;
+          const int row = hh * P.ld + (P.n - 1) * P.b + (tile % tiles_per_head) * 128;
           const uint32_t dst = q_smem + t * C::kTileBytes;
           if (I8) {
             tma_load_2d(dst, &tm_q, 0, row, smem_u32(&bar_q));
@@ -145,7 +146,7 @@ __global__ void __launch_bounds__(608, 1)
               !mbar_wait(smem_u32(&bar_kempty[st]), ((u / C::kStages) - 1) & 1, abort_flag, P.err))
             break;
           const uint32_t dst = k_smem + st * C::kTileBytes;
-          const int row = kvh * P.S + (ch0 + u) * 128;
+          const int row = kvh * P.ld + (ch0 + u) * 128;
           mbar_expect_tx(smem_u32(&bar_kfull[st]), C::kTileBytes);
           tma_load_2d(dst, &tm_k, 0, row, smem_u32(&bar_kfull[st]));
           if (!I8) tma_load_2d(dst + 16384, &tm_k, 64, row, smem_u32(&bar_kfull[st]));
@@ -467,7 +468,7 @@ template <bool I8>
 __global__ void __launch_bounds__(1024)
     k_pattern(const void *__restrict__ q, const float *__restrict__ q_scale,
               const float *__restrict__ LOc, const float *__restrict__ HIc,
-              const float *__restrict__ kbar, int S, int g, int b, int n, int nch, float inv_sqrt_d,
+              const float *__restrict__ kbar, int S, int ld, int g, int b, int n, int nch, float inv_sqrt_d,
               float tau, float *__restrict__ vhat, float *__restrict__ shat,
               float *__restrict__ pest, float *__restrict__ jsd, int *__restrict__ pattern) {
   __shared__ float qb[128];
@@ -487,7 +488,7 @@ __global__ void __launch_bounds__(1024)
   }
   // mean of the last block's query rows
   if (tid < 128) {
-    const size_t base = ((size_t)h * S + (size_t)(n - 1) * b) * 128 + tid;
+    const size_t base = ((size_t)h * ld + (size_t)(n - 1) * b) * 128 + tid;
     if (I8) {
       const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
       int acc = 0;
@@ -570,11 +571,11 @@ __global__ void __launch_bounds__(1024)
 template <bool I8>
 __global__ void __launch_bounds__(256)
     k_qbar(const void *__restrict__ q, const float *__restrict__ q_scale,
-           const int *__restrict__ pattern, int S, int b, int n, float *__restrict__ qbar) {
+           const int *__restrict__ pattern, int S, int ld, int b, int n, float *__restrict__ qbar) {
   const int r = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
   if (pattern[h] != 1) return;
   __shared__ float red[16][128];
-  const size_t row0 = (size_t)h * S + (size_t)r * b;
+  const size_t row0 = (size_t)h * ld + (size_t)r * b;
   const int rows = min(b, S - r * b);
   if (I8) {
     // 8 threads per 128-byte row, 32 rows per pass; thread owns 16 columns

@@ -22,7 +22,8 @@ SYMBOLS = ("fp_index_create", "fp_index_free", "fp_build_index", "fp_sparse_attn
            "fp_index_nnz", "fp_index_export", "fp_get_device_error", "fp_debug_wait_timeout",
            "fp_debug_qk_tile_i8", "fp_pattern_stats_noalloc", "fp_strerror",
            "fp_prefill_create", "fp_prefill_free", "fp_prefill_enqueue", "fp_prefill_wait", "fp_prefill_run",
-           "fp_prefill_group_index")
+           "fp_prefill_group_index", "fp_varlen_create", "fp_varlen_free", "fp_varlen_build_index",
+           "fp_varlen_sparse_attn", "fp_varlen_index")
 
 
 class FpError(RuntimeError):
@@ -58,8 +59,14 @@ def _load():
     L.fp_prefill_enqueue.argtypes = [vp, vp, vp, vp, vp, vp, f, f, vp, vp]
     L.fp_prefill_wait.argtypes = [vp, vp]
     L.fp_prefill_group_index.argtypes = [vp, i, ctypes.POINTER(vp)]
+    L.fp_varlen_create.argtypes = [vp, i, i, i, i, i, ctypes.POINTER(vp)]
+    L.fp_varlen_free.argtypes = [vp]
+    L.fp_varlen_free.restype = None
+    L.fp_varlen_build_index.argtypes = [vp, vp, vp, f, f, i, vp, vp, vp]
+    L.fp_varlen_sparse_attn.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp]
+    L.fp_varlen_index.argtypes = [vp, i, ctypes.POINTER(vp)]
     for s in SYMBOLS:
-        if s not in ("fp_index_free", "fp_strerror", "fp_prefill_free"):
+        if s not in ("fp_index_free", "fp_strerror", "fp_prefill_free", "fp_varlen_free"):
             getattr(L, s).restype = i
     return L
 
@@ -234,6 +241,49 @@ class Prefill:
     def free(self):
         if self.handle:
             _lib.fp_prefill_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+class Varlen:
+    """Owns one fp_varlen set (include/fp_sparse.h): one index per packed
+    sequence; cu_seqlens is a host sequence of nseq + 1 offsets."""
+
+    def __init__(self, cu_seqlens, Hq, Hkv, d, b):
+        import numpy as np
+        cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int32))
+        h = ctypes.c_void_p()
+        _check(_lib.fp_varlen_create(cu.ctypes.data, len(cu) - 1, Hq, Hkv, d, b, ctypes.byref(h)),
+               "fp_varlen_create")
+        self.handle = h.value
+        self.cu, self.Hq, self.Hkv, self.d, self.b = [int(c) for c in cu], Hq, Hkv, d, b
+
+    def build_index(self, q, k, gamma, tau, qk_dtype, q_scale=None, k_scale=None, stream=None):
+        _check(_lib.fp_varlen_build_index(self.handle, _ptr(q), _ptr(k), float(gamma), float(tau), int(qk_dtype),
+                                          _ptr(q_scale), _ptr(k_scale), _stream(stream)), "fp_varlen_build_index")
+
+    def sparse_attn(self, q, k, v, out, q_scale=None, k_scale=None, stream=None):
+        _check(_lib.fp_varlen_sparse_attn(self.handle, _ptr(q), _ptr(k), _ptr(v), _ptr(q_scale), _ptr(k_scale),
+                                          _ptr(out), _stream(stream)), "fp_varlen_sparse_attn")
+
+    def index(self, seq):
+        """The Index of sequence `seq` (owned by the set), or None when it is empty."""
+        h = ctypes.c_void_p()
+        _check(_lib.fp_varlen_index(self.handle, int(seq), ctypes.byref(h)), "fp_varlen_index")
+        if not h.value:
+            return None
+        idx = Index(h.value, self.cu[seq + 1] - self.cu[seq], self.Hq, self.Hkv, self.d, self.b)
+        idx.free = lambda: None  # owned by the set
+        return idx
+
+    def free(self):
+        if self.handle:
+            _lib.fp_varlen_free(self.handle)
             self.handle = None
 
     def __del__(self):

@@ -169,6 +169,43 @@ int fp_pattern_stats_noalloc(const void *q, const void *k, int S, int Hq, int Hk
                              float *vhat, float *shat, float *pest, float *jsd, int32_t *pattern,
                              void *stream);
 
+/* ---- Packed sequences of different lengths ------------------------------
+ * nseq sequences packed head-major: q[Hq][T][d], k and v [Hkv][T][d],
+ * out [Hq][T][d], with sequence s at rows cu_seqlens[s] .. cu_seqlens[s+1]-1
+ * of every head and T = cu_seqlens[nseq].  Every sequence is its own
+ * problem (its own last block, statistics, pattern and block lists; causal
+ * within the sequence, never across sequences), with the same supported
+ * shapes as above for its length (lengths of 0 are allowed and skipped).
+ * The articles treat one sequence at a time; this is that operation applied
+ * to each sequence of a packed batch. */
+typedef struct fp_varlen fp_varlen;
+
+/* Allocates one index per non-empty sequence on the current device.
+ * cu_seqlens: HOST int32[nseq + 1], cu_seqlens[0] = 0, non-decreasing.
+ * Returns FP_ERR_ARG for bad offsets or shapes, FP_ERR_CUDA if allocation
+ * fails. */
+int fp_varlen_create(const int32_t *cu_seqlens, int nseq, int Hq, int Hkv, int d, int b, fp_varlen **out);
+
+/* Frees the set and its indexes (NULL is ignored); synchronises the device. */
+void fp_varlen_free(fp_varlen *set);
+
+/* fp_build_index for every sequence, queued in order on `stream`.  q, k:
+ * packed device tensors as above (bf16 or int8); for FP_QK_INT8 the device
+ * scales are per sequence and head: q_scale[nseq][Hq], k_scale[nseq][Hkv]. */
+int fp_varlen_build_index(fp_varlen *set, const void *q, const void *k, float gamma, float tau, int qk_dtype,
+                          const float *q_scale, const float *k_scale, void *stream);
+
+/* fp_sparse_attn for every sequence over its own block lists; writes the
+ * packed out [Hq][T][d] bf16.  Returns FP_ERR_STATE before a build. */
+int fp_varlen_sparse_attn(const fp_varlen *set, const void *q, const void *k, const void *v, const float *q_scale,
+                          const float *k_scale, void *out, void *stream);
+
+/* Index of sequence `seq` (NULL for an empty sequence), owned by the set, for
+ * fp_index_export / fp_index_nnz / fp_index_info (its S is the sequence
+ * length).  fp_build_index and fp_sparse_attn refuse it with FP_ERR_STATE,
+ * since its rows are spaced for the packed layout. */
+int fp_varlen_index(const fp_varlen *set, int seq, const fp_index **out);
+
 /* Static message for an FP_* code. */
 const char *fp_strerror(int code);
 

@@ -83,3 +83,22 @@ def test_prefill_run_rejects_null_before_any_cuda_call(fp):
     assert L.fp_prefill_wait(None, None) == fp.FP_ERR_ARG
     assert L.fp_prefill_group_index(None, 0, None) == fp.FP_ERR_ARG
     L.fp_prefill_free(None)
+
+
+def test_varlen_create_rejects_bad_offsets(fp):
+    L = fp.lib()
+    h = ctypes.c_void_p()
+    for cu, nseq, b in [([1, 100], 1, 128), ([0, 100, 50], 2, 128), ([0, 100], 0, 128), ([0, 131073], 1, 128),
+                        ([0, 0], 1, 128), ([0, 100], 1, 64)]:
+        arr = (ctypes.c_int32 * len(cu))(*cu)
+        assert L.fp_varlen_create(arr, nseq, 4, 2, 128, b, ctypes.byref(h)) == fp.FP_ERR_ARG, cu
+        assert h.value is None
+    assert L.fp_varlen_create(None, 1, 4, 2, 128, 128, ctypes.byref(h)) == fp.FP_ERR_ARG
+
+
+def test_varlen_calls_reject_null(fp):
+    L = fp.lib()
+    assert L.fp_varlen_build_index(None, 16, 16, 0.9, 0.1, 0, None, None, None) == fp.FP_ERR_ARG
+    assert L.fp_varlen_sparse_attn(None, 16, 16, 16, None, None, 16, None) == fp.FP_ERR_ARG
+    assert L.fp_varlen_index(None, 0, None) == fp.FP_ERR_ARG
+    L.fp_varlen_free(None)
