@@ -161,7 +161,7 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   const int nlast = J.S - (J.n - 1) * J.b;  // rows of the (possibly partial) last block
   const int tiles_per_head = (nlast + 127) / 128;
   const int tiles_per_group = J.g * tiles_per_head;
-  const int tgroups = (tiles_per_group + 3) / 4;
+  const int tgroups = (tiles_per_group + ScoreCfg<I8>::kTiles - 1) / ScoreCfg<I8>::kTiles;
   int R = sm_count() / (tgroups * J.Hkv);
   if (R < 1) R = 1;
   if (R > J.nch) R = J.nch;

@@ -40,8 +40,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 // block, where the causal mask already hides them from its real rows.
 // Warps:
 //   0..15  statistics: warpgroup t owns tile t; thread = one query row
-//   16     TMA producer     17  MMA issuer + TMEM owner
-//   18     K column sums for the block means (only CTAs of tile group 0)
+//   16     TMA producer
+//   17..20 MMA issuers, one per tile (warp 17 also owns TMEM): each tile's
+//          chain (score a 64-key half, drain it, score the next) runs on its
+//          own, so a slow tile never holds back the others
+//   21, 22 K column sums for the block means, one 64-column half each (only
+//          CTAs of tile group 0)
 // TMEM: tile t's 128x128 fp32 score tile at columns [128t, 128t+128), filled
 // and drained as two 64-key halves with their own barriers.
 // ---------------------------------------------------------------------------
@@ -64,14 +68,16 @@ template <bool I8>
 struct ScoreCfg {
   static constexpr int kStages = I8 ? 4 : 3;
   static constexpr int kTileBytes = I8 ? 16384 : 32768;  // 128 rows x 128 elements
-  static constexpr int kThreads = 608;
-  static constexpr int kSmem = 4 * kTileBytes + kStages * kTileBytes + 1024;
-  // warps 0-15 statistics, 16 producer, 17 MMA, 18 K column sums
-  static_assert(kThreads == 19 * 32, "k_score_last warp roles need exactly 19 warps");
+  static constexpr int kTiles = 4;       // row tiles per CTA
+  static constexpr int kSumWarps = 2;
+  static constexpr int kThreads = (17 + kTiles + kSumWarps) * 32;
+  static constexpr int kSmem = kTiles * kTileBytes + kStages * kTileBytes + 1024;
+  // warps 0-15 statistics, 16 producer, 17-20 MMA issuers, 21-22 K column sums
+  static_assert(kThreads == 736, "k_score_last warp roles need exactly 23 warps");
 };
 
 template <bool I8>
-__global__ void __launch_bounds__(608, 1)
+__global__ void __launch_bounds__(736, 1)
     k_score_last(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  ScoreParams P) {
   using C = ScoreCfg<I8>;
@@ -89,7 +95,7 @@ __global__ void __launch_bounds__(608, 1)
   const int ch1 = min(P.nch, ch0 + P.chunks_per_cta);
   const int U = ch1 - ch0;
   const bool do_ksum = (blockIdx.y == 0);
-  const int n_ksum_warps = do_ksum ? 1 : 0;
+  const int n_ksum_warps = do_ksum ? C::kSumWarps : 0;
   const int tiles_per_head = P.tiles_per_head;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -102,7 +108,7 @@ __global__ void __launch_bounds__(608, 1)
     mbar_init(smem_u32(&bar_q), 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(smem_u32(&bar_kfull[s]), 1);
-      mbar_init(smem_u32(&bar_kempty[s]), 1 + n_ksum_warps);
+      mbar_init(smem_u32(&bar_kempty[s]), T + n_ksum_warps);
     }
     for (int t = 0; t < 4; ++t)
       for (int hf = 0; hf < 2; ++hf) {
@@ -152,90 +158,96 @@ __global__ void __launch_bounds__(608, 1)
           if (!I8) tma_load_2d(dst + 16384, &tm_k, 64, row, smem_u32(&bar_kfull[st]));
         }
       }
-    } else if (warp == 17) {
-      // ------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
-        // Each 128-key chunk is scored as two 64-key halves, all tiles' first
-        // halves before the second ones, so a statistics warpgroup works on
-        // one half while the tensor pipe fills the other.
+    } else if (warp >= 17 && warp < 17 + C::kTiles) {
+      // ------------------------------------------------------------ MMA issuers
+      // Warp 17 + t scores tile t: each 128-key chunk as two 64-key halves,
+      // a half once the statistics warps have drained it from the previous
+      // chunk.  Every issuer commits its own MMAs (a commit tracks the
+      // issuing thread's operations) to the K stage's empty barrier.
+      const int t = warp - 17;
+      if (lane == 0 && t < T) {
         const uint32_t idesc = I8 ? idesc_i8(128, 64) : idesc_bf16(128, 64, 0);
+        const uint32_t qb = q_smem + t * C::kTileBytes;
         bool ok = mbar_wait(smem_u32(&bar_q), 0, abort_flag, P.err);
         for (int u = 0; ok && u < U; ++u) {
           const int st = u % C::kStages;
           if (!mbar_wait(smem_u32(&bar_kfull[st]), (u / C::kStages) & 1, abort_flag, P.err)) break;
           const uint32_t kb = k_smem + st * C::kTileBytes;
-          for (int hf = 0; hf < 2 && ok; ++hf) {
-            for (int t = 0; t < T; ++t) {
-              if (u > 0 && !mbar_wait(smem_u32(&bar_sfree[t][hf]), (u - 1) & 1, abort_flag, P.err)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              const uint32_t qb = q_smem + t * C::kTileBytes;
-              const uint32_t d_tmem = tmem + t * 128 + hf * 64;
-              const uint32_t kh = kb + hf * 8192;  // key rows 64*hf .. 64*hf+63
-              if (I8) {
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                  mma_i8_ss(d_tmem, umma_desc_sw128(qb + kk * 32, 16, 1024),
-                            umma_desc_sw128(kh + kk * 32, 16, 1024), idesc, kk > 0);
-              } else {
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                  const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                  mma_bf16_ss(d_tmem, umma_desc_sw128(qb + off, 16, 1024),
-                              umma_desc_sw128(kh + off, 16, 1024), idesc, kk > 0);
-                }
-              }
-              tc_commit(smem_u32(&bar_sfull[t][hf]));
+          for (int hf = 0; hf < 2; ++hf) {
+            if (u > 0 && !mbar_wait(smem_u32(&bar_sfree[t][hf]), (u - 1) & 1, abort_flag, P.err)) {
+              ok = false;
+              break;
             }
+            tc_fence_after();
+            const uint32_t d_tmem = tmem + t * 128 + hf * 64;
+            const uint32_t kh = kb + hf * 8192;  // key rows 64*hf .. 64*hf+63
+            if (I8) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_i8_ss(d_tmem, umma_desc_sw128(qb + kk * 32, 16, 1024), umma_desc_sw128(kh + kk * 32, 16, 1024),
+                          idesc, kk > 0);
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                mma_bf16_ss(d_tmem, umma_desc_sw128(qb + off, 16, 1024), umma_desc_sw128(kh + off, 16, 1024), idesc,
+                            kk > 0);
+              }
+            }
+            tc_commit(smem_u32(&bar_sfull[t][hf]));
           }
           if (!ok) break;
           tc_commit(smem_u32(&bar_kempty[st]));
         }
       }
-    } else if (warp >= 18) {
+    } else if (warp >= 17 + C::kTiles) {
       // ------------------------------------------------------------ K column sums
-      const int kw = warp - 18;
-      if (kw < n_ksum_warps) {
+      // warp 21 + kh sums key columns 64kh .. 64kh+63 over the chunk's keys
+      // inside [0, S)
+      const int kh = warp - 17 - C::kTiles;
+      if (kh < n_ksum_warps) {
         for (int u = 0; u < U; ++u) {
           const int st = u % C::kStages;
           if (!mbar_wait(smem_u32(&bar_kfull[st]), (u / C::kStages) & 1, abort_flag, P.err)) break;
           const uint8_t *tile = k_gen + st * C::kTileBytes;
-          float* out = P.ksum + ((size_t)kvh * P.nch + (ch0 + u)) * 128;
-          const int nrows = min(128, P.S - (ch0 + u) * 128);  // keys of the chunk inside [0, S)
+          float *out = P.ksum + ((size_t)kvh * P.nch + (ch0 + u)) * 128 + kh * 64;
+          const int nrows = min(128, P.S - (ch0 + u) * 128);
           if (I8) {
-            // one 128-byte row per key; lane owns bytes 4*lane .. 4*lane+3
-            int acc0 = 0, acc1 = 0, acc2 = 0, acc3 = 0;
+            // one 128-byte row per key; lane owns bytes 64kh + 2lane, +1
+            const int c16 = 4 * kh + (lane >> 3), within = (2 * lane) & 15;
+            int acc0 = 0, acc1 = 0;
+#pragma unroll 4
             for (int r = 0; r < nrows; ++r) {
-              const int phys = (((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) << 2);
-              const uint32_t w = *reinterpret_cast<const uint32_t *>(tile + r * 128 + phys);
+              const int phys = ((c16 ^ (r & 7)) << 4) | within;
+              const uint32_t w = *reinterpret_cast<const uint16_t *>(tile + r * 128 + phys);
               acc0 += (int)(int8_t)(w & 0xff);
               acc1 += (int)(int8_t)((w >> 8) & 0xff);
-              acc2 += (int)(int8_t)((w >> 16) & 0xff);
-              acc3 += (int)(int8_t)(w >> 24);
             }
-            out[4 * lane + 0] = (float)acc0;
-            out[4 * lane + 1] = (float)acc1;
-            out[4 * lane + 2] = (float)acc2;
-            out[4 * lane + 3] = (float)acc3;
+            out[2 * lane] = (float)acc0;
+            out[2 * lane + 1] = (float)acc1;
           } else {
-            // lane owns columns 2*lane, 2*lane+1 of each 64-column half
-            float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
-            for (int r = 0; r < nrows; ++r) {
-              const int phys = (((lane >> 2) ^ (r & 7)) << 4) | ((lane & 3) << 2);
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(tile + r * 128 + phys));
-              const float2 e = __bfloat1622float2(
-                  *reinterpret_cast<const __nv_bfloat162 *>(tile + 16384 + r * 128 + phys));
-              a0 += f.x;
-              a1 += f.y;
-              c0 += e.x;
-              c1 += e.y;
+            // 64-column half kh (a 16 KB swizzled block); lane owns columns
+            // 2lane, 2lane+1: the bf16 pair widened by bit moves and added as
+            // one packed fp32 pair, even and odd rows in separate chains
+            const uint8_t *hsrc = tile + kh * 16384;
+            uint64_t ae = 0ull, ao = 0ull;
+            const int c16 = lane >> 2, within = (lane & 3) << 2;
+            auto row_pair = [&](int r) -> uint64_t {
+              const uint32_t w = *reinterpret_cast<const uint32_t *>(hsrc + r * 128 + (((c16 ^ (r & 7)) << 4) | within));
+              return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+            };
+            int r = 0;
+#pragma unroll 2
+            for (; r + 1 < nrows; r += 2) {
+              ae = f2_add(ae, row_pair(r));
+              ao = f2_add(ao, row_pair(r + 1));
             }
-            out[2 * lane] = a0;
-            out[2 * lane + 1] = a1;
-            out[64 + 2 * lane] = c0;
-            out[64 + 2 * lane + 1] = c1;
+            if (r < nrows) ae = f2_add(ae, row_pair(r));
+            float x0, x1, y0, y1;
+            f2_unpack(ae, x0, x1);
+            f2_unpack(ao, y0, y1);
+            out[2 * lane] = x0 + y0;
+            out[2 * lane + 1] = x1 + y1;
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bar_kempty[st]));
