@@ -90,14 +90,20 @@ def sweep_workloads():
     return out
 
 
+def rope_tables(S: int, d: int, theta: float = ROPE_THETA):
+    """cos/sin of the rotary angles p * theta^(-2i/d), p in [0, S), i in [0, d/2),
+    evaluated in float64 and rounded to float32: two [S][d/2] tensors."""
+    half = d // 2
+    inv = theta ** (-torch.arange(0, half, dtype=torch.float64) * 2.0 / d)
+    ang = torch.arange(S, dtype=torch.float64)[:, None] * inv[None, :]
+    return torch.cos(ang).to(torch.float32), torch.sin(ang).to(torch.float32)
+
+
 def rope_(x: torch.Tensor, theta: float = ROPE_THETA) -> torch.Tensor:
     """In-place rotate-half rotary embedding of x[H][S][d] (fp32), positions 0..S-1."""
     H, S, d = x.shape
     half = d // 2
-    inv = theta ** (-torch.arange(0, half, dtype=torch.float64) * 2.0 / d)
-    ang = torch.arange(S, dtype=torch.float64)[:, None] * inv[None, :]
-    cos = torch.cos(ang).to(torch.float32)
-    sin = torch.sin(ang).to(torch.float32)
+    cos, sin = rope_tables(S, d, theta)
     for h in range(H):
         x1 = x[h, :, :half].clone()
         x2 = x[h, :, half:].clone()
@@ -173,3 +179,26 @@ def make_inputs(w: Workload):
 def dense_equiv_flops(S: int, Hq: int, d: int) -> float:
     """Causal dense attention FLOPs, 4*Hq*S^2*d/2 (two GEMMs over the lower triangle)."""
     return 2.0 * Hq * d * float(S) * float(S)
+
+
+def make_prerope_inputs(w: Workload) -> dict:
+    """Q and K before the rotary embedding (as a projection's epilogue sees
+    them), V, and the rotary tables: q_in [Hq][S][d], k_in [Hkv][S][d] and v
+    bf16 (N(0,1), with the topic structure of the query-aware heads), cos/sin
+    [S][d/2] float32.  Seeded like make_inputs."""
+    S, Hq, Hkv, d = w.S, w.Hq, w.Hkv, w.d
+    g = Hq // Hkv
+    gen = torch.Generator().manual_seed(10_000 + w.seed)
+    q = torch.randn((Hq, S, d), generator=gen, dtype=torch.float32)
+    k = torch.randn((Hkv, S, d), generator=gen, dtype=torch.float32)
+    v = torch.randn((Hkv, S, d), generator=gen, dtype=torch.float32)
+    for kv in range(Hkv):
+        topic = torch.randint(0, w.n_topics, (S,), generator=gen)
+        cent = torch.randn((w.n_topics, d), generator=gen, dtype=torch.float32)
+        k[kv] += 2.0 * cent[topic]
+        for h in range(kv * g, kv * g + g):
+            if h % 2:
+                q[h] += 2.0 * cent[topic]
+    cos, sin = rope_tables(S, d)
+    return {"q_in": q.to(torch.bfloat16), "k_in": k.to(torch.bfloat16), "v": v.to(torch.bfloat16),
+            "cos": cos, "sin": sin}

@@ -332,3 +332,52 @@ void orc_qk_int_tile(const orc_problem *P, int h, int p0, int j0, int rows, int 
         for (int t = 0; t < cols; ++t)
             out[(size_t)i * cols + t] = (int32_t)orc_qk_int(P, h, p0 + i, j0 + t);
 }
+
+/* ------------------------------------------------------------------------
+ * Rotary embedding with block pooling: the epilogue of the projection step
+ * that produces Q and K ([FP] 1.1: Q = X W_q, K = X W_k), followed by the
+ * block means the index generation uses ([FP] 2.1 block pooling; [MV] 1.1
+ * block-level estimate).  Rotate-half convention: for i < d/2, with c =
+ * cos[p][i], s = sin[p][i] (the caller's tables),
+ *   out[p][i]       = x[p][i] c - x[p][i + d/2] s
+ *   out[p][i + d/2] = x[p][i + d/2] c + x[p][i] s,
+ * each rounded to the nearest bf16 (ties to even), as the stored tensor is
+ * bf16; means[c][t] = mean over the rows of block c (b of them, or S-(n-1)b
+ * for a partial last block) of the rounded out[p][t].
+ * x: H*S*d doubles (bf16 values); cos, sin: S*(d/2) doubles; out: H*S*d;
+ * means: H*n*d with n = ceil(S/b). */
+
+/* Nearest bf16 (8 significant bits, ties to even) of a finite double. */
+static double round_bf16(double x)
+{
+    if (x == 0.0 || !isfinite(x)) return x;
+    int e;
+    double m = frexp(x, &e);            /* x = m 2^e, 0.5 <= |m| < 1 */
+    double r = nearbyint(ldexp(m, 8));  /* 128 <= |r| <= 256, ties to even */
+    return ldexp(r, e - 8);
+}
+
+void orc_rope_pool(const double *x, const double *cosT, const double *sinT, int H, int S, int d, int b,
+                   double *out, double *means)
+{
+    int half = d / 2, n = (S + b - 1) / b;
+    for (int h = 0; h < H; ++h) {
+        for (int p = 0; p < S; ++p) {
+            const double *xr = x + ((size_t)h * S + p) * d;
+            double *orow = out + ((size_t)h * S + p) * d;
+            for (int i = 0; i < half; ++i) {
+                double c = cosT[(size_t)p * half + i], sn = sinT[(size_t)p * half + i];
+                orow[i] = round_bf16(xr[i] * c - xr[i + half] * sn);
+                orow[i + half] = round_bf16(xr[i + half] * c + xr[i] * sn);
+            }
+        }
+        for (int c = 0; c < n; ++c) {
+            int lo = c * b, hi = (c + 1) * b < S ? (c + 1) * b : S;
+            for (int t = 0; t < d; ++t) {
+                double acc = 0.0;
+                for (int p = lo; p < hi; ++p) acc += out[((size_t)h * S + p) * d + t];
+                means[((size_t)h * n + c) * d + t] = acc / (hi - lo);
+            }
+        }
+    }
+}

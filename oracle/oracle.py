@@ -58,6 +58,8 @@ def lib():
         L.orc_last_block_stats.argtypes = [pp, ctypes.c_int, dp, dp]
         L.orc_last_block_stats.restype = ctypes.c_double
         L.orc_block_means.argtypes = [pp, ctypes.c_int, ctypes.c_int, dp]
+        L.orc_rope_pool.argtypes = [dp, dp, dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, dp, dp]
+        L.orc_rope_pool.restype = None
         L.orc_block_means.restype = None
         L.orc_pest.argtypes = [dp, dp, ctypes.c_int, ctypes.c_int, dp]
         L.orc_pest.restype = None
@@ -201,3 +203,20 @@ def select(w, r, gamma):
     info = np.zeros(3)
     cnt = lib().orc_select(_dp(w), int(r), float(gamma), _ip(sel), _dp(info))
     return sel[:cnt].copy(), info
+
+
+def rope_pool(x, cos, sin, b):
+    """Rotary embedding (rotate-half, the caller's cos/sin tables [S][d/2])
+    of x [H][S][d], each output rounded to bf16, and the block means of the
+    rounded rows.  Returns (out [H][S][d] float64, means [H][n][d])."""
+    def f64(t):  # values (not bit patterns) as float64
+        if isinstance(t, torch.Tensor):
+            return t.detach().cpu().to(torch.float64).contiguous().numpy()
+        return np.ascontiguousarray(t, dtype=np.float64)
+    x, cos, sin = f64(x), f64(cos), f64(sin)
+    H, S, d = x.shape
+    n = (S + b - 1) // b
+    out = np.zeros_like(x)
+    means = np.zeros((H, n, d))
+    lib().orc_rope_pool(_dp(x), _dp(cos), _dp(sin), H, S, d, b, _dp(out), _dp(means))
+    return out, means

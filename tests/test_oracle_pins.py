@@ -19,6 +19,7 @@ import torch
 from scipy.spatial.distance import jensenshannon
 from scipy.special import softmax as sp_softmax
 
+from dynamic_block_sparse_last_b200 import synth
 from oracle import oracle as orc
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -332,3 +333,72 @@ def test_golden_tiny_index_regression():
         assert abs(out["jsd"] - gh["jsd"]) < 1e-12
         assert np.allclose(out["vhat"], gh["vhat"], atol=1e-14)
         assert [list(map(int, r)) for r in out["rows"]] == gh["rows"]
+
+
+# ---------------------------------------------------------------------------
+# Rotary embedding + block pooling (the projection epilogue, [FP] 1.1 / 2.1)
+# ---------------------------------------------------------------------------
+
+def _bf16_grid(shape, seed):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(shape, generator=g).to(torch.bfloat16)
+
+
+def test_rope_exact_turns():
+    """cos = 0, sin = 1 is a quarter turn (x_i -> -x_{i+d/2}, x_{i+d/2} -> x_i);
+    cos = -1, sin = 0 a half turn; both exact in bf16."""
+    x = _bf16_grid((2, 5, 128), 1)
+    xf = x.double().numpy()
+    zero, one = np.zeros((5, 64)), np.ones((5, 64))
+    out, _ = orc.rope_pool(x, zero, one, 4)
+    assert np.array_equal(out[..., :64], -xf[..., 64:]) and np.array_equal(out[..., 64:], xf[..., :64])
+    out, _ = orc.rope_pool(x, -one, zero, 4)
+    assert np.array_equal(out, -xf)
+
+
+def test_rope_equals_complex_rotation():
+    """The pair (x_i, x_{i+d/2}) rotates as the complex number x_i + i x_{i+d/2}
+    multiplied by cos + i sin (numpy complex128), then rounded to bf16."""
+    w = synth.Workload("rope", S=200, Hq=2, Hkv=1, b=64, seed=3)
+    x = synth.make_prerope_inputs(w)
+    out, _ = orc.rope_pool(x["q_in"], x["cos"], x["sin"], 64)
+    xf = x["q_in"].double().numpy()
+    z = (xf[..., :64] + 1j * xf[..., 64:]) * (x["cos"].double().numpy() + 1j * x["sin"].double().numpy())[None]
+    ref = torch.from_numpy(np.concatenate([z.real, z.imag], -1)).to(torch.bfloat16).double().numpy()
+    diff = np.abs(out - ref)
+    assert (diff == 0).mean() > 0.999
+    assert np.all(diff <= 2.0 ** -7 * np.abs(ref) + 1e-30)
+
+
+def test_rope_relative_position_property():
+    """<R_p q, R_j k> depends on p - j only: the same q, k placed at (p, j) and
+    (p + t, j + t) give the same logit up to bf16 rounding of the outputs."""
+    S = 256
+    cos, sin = synth.rope_tables(S, 128)
+    q0 = _bf16_grid((128,), 5).double()
+    k0 = _bf16_grid((128,), 6).double()
+    x = torch.zeros(2, S, 128, dtype=torch.float64)
+    for p in (10, 40, 200):
+        x[0, p] = q0
+    for j in (3, 33, 193):
+        x[1, j] = k0
+    out, _ = orc.rope_pool(x, cos, sin, 64)
+    dots = [float(out[0, p] @ out[1, j]) for p, j in ((10, 3), (40, 33), (200, 193))]
+    scale = float(q0.norm() * k0.norm())
+    assert max(dots) - min(dots) <= 2e-2 * scale
+    assert abs(float(out[0, 10] @ out[1, 3]) - float(out[0, 10] @ out[1, 33])) > 1e-3 * scale  # not trivially equal
+
+
+def test_rope_pair_norms_and_block_means():
+    """Each rotated pair keeps its length (to bf16 rounding); the means are the
+    column means of the rounded rows over each block, the last one partial."""
+    w = synth.Workload("rope2", S=300, Hq=3, Hkv=1, b=128, seed=4)
+    x = synth.make_prerope_inputs(w)
+    out, means = orc.rope_pool(x["q_in"], x["cos"], x["sin"], 128)
+    xf = x["q_in"].double().numpy()
+    n_in = np.hypot(xf[..., :64], xf[..., 64:])
+    n_out = np.hypot(out[..., :64], out[..., 64:])
+    assert np.all(np.abs(n_out - n_in) <= 2.0 ** -7 * n_in + 1e-12)
+    assert means.shape == (3, 3, 128)
+    for c, (lo, hi) in enumerate(((0, 128), (128, 256), (256, 300))):
+        assert np.allclose(means[:, c], out[:, lo:hi].mean(1), rtol=0, atol=1e-13)
