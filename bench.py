@@ -399,6 +399,59 @@ def run_sweep(args):
     return 0
 
 
+def run_rope_pool(args):
+    """The rotary-embedding epilogue with block pooling (fp_rope_pool) at the
+    workload's shape against HBM, and the index build on its means
+    (fp_build_index_pooled) beside the one that pools Q and K itself.  One JSON
+    line; not the headline."""
+    from dynamic_block_sparse_last_b200 import fp
+    dev = torch.device("cuda", 0)
+    w = synth.WORKLOADS[args.workload]
+    x = synth.make_prerope_inputs(w)
+    q_in, k_in = x["q_in"].to(dev), x["k_in"].to(dev)
+    cos, sin = x["cos"].to(dev), x["sin"].to(dev)
+    n = (w.S + w.b - 1) // w.b
+    q, k = torch.empty_like(q_in), torch.empty_like(k_in)
+    qbar = torch.empty(w.Hq, n, w.d, device=dev)
+    kbar = torch.empty(w.Hkv, n, w.d, device=dev)
+    idx = fp.fp_index_create(w.S, w.Hq, w.Hkv, w.d, w.b)
+
+    def rope():
+        fp.fp_rope_pool(q_in, k_in, cos, sin, w.S, w.Hq, w.Hkv, w.d, w.b, q, k, qbar, kbar)
+
+    def build():
+        fp.fp_build_index(q, k, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, fp.FP_QK_BF16, None, None, idx)
+
+    def build_pooled():
+        fp.fp_build_index_pooled(q, k, qbar, kbar, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, idx)
+
+    res = {}
+    for name, fn in (("rope_pool", rope), ("index", build), ("index_pooled", build_pooled)):
+        for _ in range(max(3, args.warmup)):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for e0, e1 in ev:
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        res[name] = float(np.median([e0.elapsed_time(e1) for e0, e1 in ev]))
+    assert fp.fp_get_device_error() == fp.FP_OK
+    peaks = load_peaks()
+    # algorithmic bytes: every Q and K element read and written once (bf16),
+    # the cos/sin tables read once, the means written
+    nbytes = (w.Hq + w.Hkv) * w.S * w.d * 4 + w.S * (w.d // 2) * 4 * 2 + (w.Hq + w.Hkv) * n * w.d * 4
+    gbs = nbytes / (res["rope_pool"] / 1e3) / 1e9
+    print(json.dumps({"metric": "rotary epilogue with block pooling (GB/s) and index build on its means (ms)",
+                      "config": {"workload": w.name, "S": w.S, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "b": w.b},
+                      "steps": args.steps, "rope_pool_ms": res["rope_pool"], "rope_pool_bytes": nbytes,
+                      "rope_pool_gbs": gbs, "rope_pool_frac_of_hbm": gbs / peaks["hbm_gbs"],
+                      "hbm_peak_gbs": peaks["hbm_gbs"], "index_ms": res["index"],
+                      "index_pooled_ms": res["index_pooled"], "gpu": torch.cuda.get_device_name(dev)}), flush=True)
+    idx.free()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -410,11 +463,15 @@ def main():
     ap.add_argument("--e2e-groups", type=int, default=0,
                     help="KV-head groups of the host-to-host pipeline (0 = one KV head per group)")
     ap.add_argument("--sweep", action="store_true", help="S x b x gamma sweep (one line per point)")
+    ap.add_argument("--rope-pool", action="store_true",
+                    help="time the rotary epilogue with block pooling and the index build on its means")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.sweep:
         return run_sweep(args)
+    if args.rope_pool:
+        return run_rope_pool(args)
     w = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

@@ -16,6 +16,7 @@
 #include "attn_kernel.cuh"
 #include "fp_sparse.h"
 #include "index_kernels.cuh"
+#include "rope_pool.cuh"
 
 using namespace fpk;
 
@@ -149,6 +150,7 @@ struct StatsJob {
   float *pm, *plo, *phi, *partM, *partL, *LOc, *HIc, *ksum, *kbar;
   float *vhat, *shat, *pest, *jsd;
   int *pattern;
+  const float *ext_kbar;  // K block means given by the caller (then ksum/kbar are not computed), or null
 };
 
 // k_score_last, k_row_stats, k_block_mass, k_kbar and k_pattern on `st`.
@@ -177,7 +179,7 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   sp.scale2 = kLog2e / sqrtf((float)J.d);
   sp.q_scale = J.q_scale;
   sp.k_scale = J.k_scale;
-  sp.pm = J.pm; sp.plo = J.plo; sp.phi = J.phi; sp.ksum = J.ksum;
+  sp.pm = J.pm; sp.plo = J.plo; sp.phi = J.phi; sp.ksum = J.ext_kbar ? nullptr : J.ksum;
   sp.err = err;
   k_score_last<I8><<<dim3(R, tgroups, J.Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
   if ((rc = launch_status())) return rc;
@@ -188,9 +190,13 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   k_block_mass<<<dim3(J.Hq, J.R2), J.b, red_bytes, st>>>(J.pm, J.plo, J.phi, J.partM, J.partL, J.nch, J.b,
                                                          nlast, J.chunks_per_part, J.LOc, J.HIc);
   if ((rc = launch_status())) return rc;
-  k_kbar<<<dim3(J.n, J.Hkv), 128, 0, st>>>(J.ksum, I8 ? J.k_scale : nullptr, J.S, J.nch, J.b, J.n, J.kbar);
-  if ((rc = launch_status())) return rc;
-  k_pattern<I8><<<J.Hq, 1024, 0, st>>>(J.q, J.q_scale, J.LOc, J.HIc, J.kbar, J.S, J.ld, J.g, J.b, J.n, J.nch,
+  const float *kbar = J.ext_kbar;
+  if (!kbar) {
+    k_kbar<<<dim3(J.n, J.Hkv), 128, 0, st>>>(J.ksum, I8 ? J.k_scale : nullptr, J.S, J.nch, J.b, J.n, J.kbar);
+    if ((rc = launch_status())) return rc;
+    kbar = J.kbar;
+  }
+  k_pattern<I8><<<J.Hq, 1024, 0, st>>>(J.q, J.q_scale, J.LOc, J.HIc, kbar, J.S, J.ld, J.g, J.b, J.n, J.nch,
                                        1.0f / sqrtf((float)J.d), J.tau, J.vhat, J.shat, J.pest, J.jsd,
                                        J.pattern);
   return launch_status();
@@ -203,9 +209,13 @@ void row_parts(int nch, int &R2, int &chunks_per_part) {
   R2 = (nch + chunks_per_part - 1) / chunks_per_part;
 }
 
+// ext_qbar / ext_kbar: block means of Q [Hq][n][128] and K [Hkv][n][128]
+// computed by the caller (fp_rope_pool); when given, the index build does not
+// pool Q or K itself.
 template <bool I8>
 int build_index_impl(const void *q, const void *k, float gamma, float tau, const float *q_scale,
-                     const float *k_scale, fp_index *I, cudaStream_t st) {
+                     const float *k_scale, fp_index *I, cudaStream_t st, const float *ext_qbar = nullptr,
+                     const float *ext_kbar = nullptr) {
   int rc = set_smem_attrs<I8>();
   if (rc) return rc;
   int *err = device_error_word();
@@ -217,12 +227,17 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   J.pm = I->pm; J.plo = I->plo; J.phi = I->phi; J.partM = I->partM; J.partL = I->partL;
   J.LOc = I->LOc; J.HIc = I->HIc; J.ksum = I->ksum; J.kbar = I->kbar;
   J.vhat = I->vhat; J.shat = I->shat; J.pest = I->pest; J.jsd = I->jsd; J.pattern = I->pattern;
+  J.ext_kbar = ext_kbar;
   if ((rc = launch_pattern_stats<I8>(J, err, st))) return rc;
   const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
-  k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->ld, I->b, I->n, I->qbar);
-  if ((rc = launch_status())) return rc;
+  const float *qbar = ext_qbar, *kbar = ext_kbar ? ext_kbar : I->kbar;
+  if (!qbar) {
+    k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->ld, I->b, I->n, I->qbar);
+    if ((rc = launch_status())) return rc;
+    qbar = I->qbar;
+  }
   const int nt = (I->n + kLgTile - 1) / kLgTile;
-  k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, I->qbar, I->kbar, I->g, I->n,
+  k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, qbar, kbar, I->g, I->n,
                                                                inv_sqrt_d, I->zlog);
   if ((rc = launch_status())) return rc;
   k_cut<<<(I->Hq * I->n + 7) / 8, 256, 0, st>>>(I->pattern, I->vhat, I->shat, I->zlog, I->Hq, I->n, gamma,
@@ -528,7 +543,7 @@ int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int
 
   StatsJob J;
   J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.d = d; J.b = b; J.n = n; J.nch = nch; J.g = Hq / Hkv;
-  J.R2 = R2; J.chunks_per_part = cpp; J.ld = S;
+  J.R2 = R2; J.chunks_per_part = cpp; J.ld = S; J.ext_kbar = nullptr;
   J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
   J.pm = pm; J.plo = plo; J.phi = phi; J.partM = partM; J.partL = partL;
   J.LOc = LOc; J.HIc = HIc; J.ksum = ksum; J.kbar = kbar;
@@ -681,6 +696,46 @@ int fp_varlen_index(const fp_varlen *V, int seq, const fp_index **out) {
   if (!V || !out || seq < 0 || seq >= V->nseq) return FP_ERR_ARG;
   *out = V->idx[seq];
   return FP_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Rotary-embedding epilogue with block pooling, and the index build that
+// takes its block means.
+// ---------------------------------------------------------------------------
+extern "C" {
+
+int fp_rope_pool(const void *q_in, const void *k_in, const float *rope_cos, const float *rope_sin, int S, int Hq,
+                 int Hkv, int d, int b, void *q_out, void *k_out, float *qbar, float *kbar, void *stream) {
+  if (!q_in || !k_in || !rope_cos || !rope_sin || !q_out || !k_out || !qbar || !kbar) return FP_ERR_ARG;
+  if (!shape_ok(S, Hq, Hkv, d, b)) return FP_ERR_ARG;
+  if (!aligned16(q_in) || !aligned16(k_in) || !aligned16(rope_cos) || !aligned16(rope_sin) || !aligned16(q_out) ||
+      !aligned16(k_out) || !aligned16(qbar) || !aligned16(kbar))
+    return FP_ERR_ARG;
+  const int n = (S + b - 1) / b;
+  k_rope_pool<<<dim3(n, Hq + Hkv), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16 *>(q_in), static_cast<const __nv_bfloat16 *>(k_in), rope_cos, rope_sin, S, Hq, b,
+      n, static_cast<__nv_bfloat16 *>(q_out), static_cast<__nv_bfloat16 *>(k_out), qbar, kbar);
+  return launch_status();
+}
+
+int fp_build_index_pooled(const void *q, const void *k, const float *qbar, const float *kbar, int S, int Hq, int Hkv,
+                          int d, int b, float gamma, float tau, fp_index *idx, void *stream) {
+  if (!idx || !q || !k || !qbar || !kbar) return FP_ERR_ARG;
+  if (!shape_ok(S, Hq, Hkv, d, b)) return FP_ERR_ARG;
+  if (S != idx->S || Hq != idx->Hq || Hkv != idx->Hkv || d != idx->d || b != idx->b) return FP_ERR_STATE;
+  if (idx->ld != idx->S) return FP_ERR_STATE;
+  if (!(gamma > 0.f && gamma <= 1.f) || !(tau >= 0.f) || std::isnan(gamma) || std::isnan(tau)) return FP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(qbar) || !aligned16(kbar)) return FP_ERR_ARG;
+  idx->built = 0;
+  const int rc = build_index_impl<false>(q, k, gamma, tau, nullptr, nullptr, idx, static_cast<cudaStream_t>(stream),
+                                         qbar, kbar);
+  if (rc == FP_OK) {
+    idx->built = 1;
+    idx->qk_dtype = FP_QK_BF16;
+  }
+  return rc;
 }
 
 }  // extern "C"

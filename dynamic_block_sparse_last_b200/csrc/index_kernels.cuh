@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(736, 1)
   const int ch0 = blockIdx.x * P.chunks_per_cta;
   const int ch1 = min(P.nch, ch0 + P.chunks_per_cta);
   const int U = ch1 - ch0;
-  const bool do_ksum = (blockIdx.y == 0);
+  const bool do_ksum = (blockIdx.y == 0) && P.ksum != nullptr;  // null: the caller gave the K means
   const int n_ksum_warps = do_ksum ? C::kSumWarps : 0;
   const int tiles_per_head = P.tiles_per_head;
 

@@ -23,7 +23,7 @@ SYMBOLS = ("fp_index_create", "fp_index_free", "fp_build_index", "fp_sparse_attn
            "fp_debug_qk_tile_i8", "fp_pattern_stats_noalloc", "fp_strerror",
            "fp_prefill_create", "fp_prefill_free", "fp_prefill_enqueue", "fp_prefill_wait", "fp_prefill_run",
            "fp_prefill_group_index", "fp_varlen_create", "fp_varlen_free", "fp_varlen_build_index",
-           "fp_varlen_sparse_attn", "fp_varlen_index")
+           "fp_varlen_sparse_attn", "fp_varlen_index", "fp_rope_pool", "fp_build_index_pooled")
 
 
 class FpError(RuntimeError):
@@ -59,6 +59,8 @@ def _load():
     L.fp_prefill_enqueue.argtypes = [vp, vp, vp, vp, vp, vp, f, f, vp, vp]
     L.fp_prefill_wait.argtypes = [vp, vp]
     L.fp_prefill_group_index.argtypes = [vp, i, ctypes.POINTER(vp)]
+    L.fp_rope_pool.argtypes = [vp, vp, vp, vp, i, i, i, i, i, vp, vp, vp, vp, vp]
+    L.fp_build_index_pooled.argtypes = [vp, vp, vp, vp, i, i, i, i, i, f, f, vp, vp]
     L.fp_varlen_create.argtypes = [vp, i, i, i, i, i, ctypes.POINTER(vp)]
     L.fp_varlen_free.argtypes = [vp]
     L.fp_varlen_free.restype = None
@@ -145,6 +147,17 @@ def fp_build_index(q, k, S, Hq, Hkv, d, b, gamma, tau, qk_dtype, q_scale, k_scal
 def fp_sparse_attn(q, k, v, q_scale, k_scale, idx: Index, out, stream=None):
     _check(_lib.fp_sparse_attn(_ptr(q), _ptr(k), _ptr(v), _ptr(q_scale), _ptr(k_scale), idx.handle,
                                _ptr(out), _stream(stream)), "fp_sparse_attn")
+
+
+def fp_rope_pool(q_in, k_in, rope_cos, rope_sin, S, Hq, Hkv, d, b, q_out, k_out, qbar, kbar, stream=None):
+    """Rotary embedding of bf16 q_in/k_in into q_out/k_out (may alias) plus block means."""
+    _check(_lib.fp_rope_pool(_ptr(q_in), _ptr(k_in), _ptr(rope_cos), _ptr(rope_sin), S, Hq, Hkv, d, b, _ptr(q_out),
+                             _ptr(k_out), _ptr(qbar), _ptr(kbar), _stream(stream)), "fp_rope_pool")
+
+
+def fp_build_index_pooled(q, k, qbar, kbar, S, Hq, Hkv, d, b, gamma, tau, idx: Index, stream=None):
+    _check(_lib.fp_build_index_pooled(_ptr(q), _ptr(k), _ptr(qbar), _ptr(kbar), S, Hq, Hkv, d, b, float(gamma),
+                                      float(tau), idx.handle, _stream(stream)), "fp_build_index_pooled")
 
 
 def fp_index_info(idx: Index):

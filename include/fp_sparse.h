@@ -169,6 +169,33 @@ int fp_pattern_stats_noalloc(const void *q, const void *k, int S, int Hq, int Hk
                              float *vhat, float *shat, float *pest, float *jsd, int32_t *pattern,
                              void *stream);
 
+/* ---- Rotary-embedding epilogue with block pooling ----------------------
+ * The projection step before the path (first article, section 1.1: Q = X W_q,
+ * K = X W_k) ends with the rotary embedding; fp_rope_pool is that epilogue and
+ * also emits the block means the index generation uses (section 2.1 block
+ * pooling), so the index build need not read Q again to pool it.
+ *
+ * q_in [Hq][S][d], k_in [Hkv][S][d]: device bf16 before the rotation;
+ * rope_cos, rope_sin: device fp32 [S][d/2] tables (cos and sin of the angle of
+ * position p and frequency i); q_out, k_out: device bf16, same layouts (may be
+ * q_in / k_in themselves); qbar [Hq][n][d], kbar [Hkv][n][d]: device fp32,
+ * n = ceil(S/b).  Rotate-half convention: for i < d/2
+ *   out[p][i] = x[p][i] cos[p][i] - x[p][i+d/2] sin[p][i],
+ *   out[p][i+d/2] = x[p][i+d/2] cos[p][i] + x[p][i] sin[p][i],
+ * computed in fp32 and stored as bf16 (nearest, ties to even); the means are
+ * over the stored values of each block's rows.  Shapes as for fp_index_create;
+ * all pointers 16-byte aligned; asynchronous on `stream`. */
+int fp_rope_pool(const void *q_in, const void *k_in, const float *rope_cos, const float *rope_sin, int S, int Hq,
+                 int Hkv, int d, int b, void *q_out, void *k_out, float *qbar, float *kbar, void *stream);
+
+/* fp_build_index (bf16 q and k) with the block means supplied by the caller,
+ * e.g. by fp_rope_pool: qbar [Hq][n][d] and kbar [Hkv][n][d] device fp32 must
+ * be the block means of q and k.  The index pass then skips its own Q and K
+ * pooling; the result is the one fp_build_index gives up to the summation
+ * order of those means. */
+int fp_build_index_pooled(const void *q, const void *k, const float *qbar, const float *kbar, int S, int Hq, int Hkv,
+                          int d, int b, float gamma, float tau, fp_index *idx, void *stream);
+
 /* ---- Packed sequences of different lengths ------------------------------
  * nseq sequences packed head-major: q[Hq][T][d], k and v [Hkv][T][d],
  * out [Hq][T][d], with sequence s at rows cu_seqlens[s] .. cu_seqlens[s+1]-1

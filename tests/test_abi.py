@@ -102,3 +102,11 @@ def test_varlen_calls_reject_null(fp):
     assert L.fp_varlen_sparse_attn(None, 16, 16, 16, None, None, 16, None) == fp.FP_ERR_ARG
     assert L.fp_varlen_index(None, 0, None) == fp.FP_ERR_ARG
     L.fp_varlen_free(None)
+
+
+def test_rope_pool_calls_reject_null(fp):
+    L = fp.lib()
+    assert L.fp_rope_pool(None, 16, 16, 16, 1024, 4, 2, 128, 128, 16, 16, 16, 16, None) == fp.FP_ERR_ARG
+    assert L.fp_rope_pool(16, 16, 16, 16, 1024, 4, 2, 64, 128, 16, 16, 16, 16, None) == fp.FP_ERR_ARG  # d
+    assert L.fp_rope_pool(16, 16, 8, 16, 1024, 4, 2, 128, 128, 16, 16, 16, 16, None) == fp.FP_ERR_ARG  # align
+    assert L.fp_build_index_pooled(16, 16, None, 16, 1024, 4, 2, 128, 128, 0.9, 0.1, None, None) == fp.FP_ERR_ARG
