@@ -714,7 +714,7 @@ int fp_rope_pool(const void *q_in, const void *k_in, const float *rope_cos, cons
       !aligned16(k_out) || !aligned16(qbar) || !aligned16(kbar))
     return FP_ERR_ARG;
   const int n = (S + b - 1) / b;
-  k_rope_pool<<<dim3(n, Hq + Hkv), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  k_rope_pool<<<dim3(Hq + Hkv, n), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16 *>(q_in), static_cast<const __nv_bfloat16 *>(k_in), rope_cos, rope_sin, S, Hq, b,
       n, static_cast<__nv_bfloat16 *>(q_out), static_cast<__nv_bfloat16 *>(k_out), qbar, kbar);
   return launch_status();

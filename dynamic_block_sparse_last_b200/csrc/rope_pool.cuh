@@ -20,14 +20,16 @@
 
 namespace fpk {
 
-// grid (n, Hq + Hkv), block 256.  Thread = (row slot rs in 0..31, pair group
-// j in 0..7): dims 8j..8j+7 and 64+8j..64+8j+7 of rows rs, rs+32, ...
+// grid (Hq + Hkv, n), block 256: the heads of a block of positions are
+// neighbours in launch order, so that block's cos/sin rows come from DRAM
+// once and from L2 for the other heads.  Thread = (row slot rs in 0..31, pair
+// group j in 0..7): dims 8j..8j+7 and 64+8j..64+8j+7 of rows rs, rs+32, ...
 __global__ void __launch_bounds__(256)
     k_rope_pool(const __nv_bfloat16 *q_in, const __nv_bfloat16 *k_in,
                 const float *__restrict__ cosT, const float *__restrict__ sinT, int S, int Hq, int b, int n,
                 __nv_bfloat16 *q_out, __nv_bfloat16 *k_out, float *__restrict__ qbar, float *__restrict__ kbar) {
   __shared__ float red[8][128];
-  const int r = blockIdx.x, hh = blockIdx.y, tid = threadIdx.x;
+  const int hh = blockIdx.x, r = blockIdx.y, tid = threadIdx.x;
   const bool isq = hh < Hq;
   const int h = isq ? hh : hh - Hq;
   // in and out may be the same tensor: every element is read, then written,
@@ -40,6 +42,7 @@ __global__ void __launch_bounds__(256)
   float acc[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+#pragma unroll 4
   for (int rr = rs; rr < rows; rr += 32) {
     const size_t p = (size_t)(p0 + rr);
     const uint4 xl = *reinterpret_cast<const uint4 *>(in + p * 128 + 8 * j);
