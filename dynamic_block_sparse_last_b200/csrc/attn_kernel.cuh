@@ -8,8 +8,13 @@
 // chunk the CTA loads serves both (KV reuse across the heads of a GQA group,
 // FAST-Prefill article section 2.2):
 //   b = 256:            the two 128-row halves of one 256-row query block
-//   b = 128, g >= 2:    the same query tile of two heads of one GQA group
-//   b = 128, g == 1:    two neighbouring query tiles of one head
+//   b <= 128, g >= 2:   the same query tile of two heads of one GQA group
+//   b <= 128, g == 1:   two neighbouring query tiles of one head
+// With b = 64 a tile holds two query blocks and a chunk two key blocks: the
+// tile attends to a chunk if either of its blocks lists either key block, and
+// each softmax warp, which owns one 32-row by 64-key quadrant and so exactly
+// one (query block, key block) pair, masks the quadrant when that pair is not
+// listed.
 // The CTA walks the union of the two tiles' chunk lists (ascending 128-key
 // chunks); a chunk only one tile needs is computed for that tile only.
 // When 128 does not divide S the last query tile and the last key chunk run
@@ -81,8 +86,10 @@ __host__ __device__ inline int attn_pairs(int Hq, int Hkv, int S, int b) {
 }
 
 struct AttnTile {
-  int valid, h, qc, r, cnt, L;
+  int valid, h, qc, r, cnt;
   const int *list;
+  int cnt1;            // b = 64: the tile's second query block r + 1 (0 when past the last block)
+  const int *list1;
 };
 
 // The two query tiles of CTA `pair`: KV-head-major, heavy pairs first within a head.
@@ -113,21 +120,22 @@ __device__ inline void attn_pair_tiles(const AttnParams &P, int pair, AttnTile (
     v1 = q1 < nq;
   }
   const int hs[2] = {h0, h1}, qs[2] = {q0, q1}, vs[2] = {1, v1};
-  const int per = P.b / 128;
+  const size_t tri = (size_t)P.n * (P.n + 1) / 2;
   for (int i = 0; i < 2; ++i) {
     t[i].valid = vs[i];
     t[i].h = hs[i];
     t[i].qc = qs[i];
     t[i].r = (qs[i] * 128) / P.b;
+    t[i].cnt = t[i].cnt1 = 0;
+    t[i].list = t[i].list1 = nullptr;
     if (vs[i]) {
-      t[i].cnt = P.counts[(size_t)hs[i] * P.n + t[i].r];
-      t[i].list = P.cols + (size_t)hs[i] * ((size_t)P.n * (P.n + 1) / 2) + (size_t)t[i].r * (t[i].r + 1) / 2;
-      // the list is ascending and ends with the diagonal block r
-      t[i].L = t[i].cnt > 0 ? (t[i].cnt - 1) * per + (qs[i] % per) + 1 : 0;
-    } else {
-      t[i].cnt = 0;
-      t[i].list = nullptr;
-      t[i].L = 0;
+      const int r = t[i].r;
+      t[i].cnt = P.counts[(size_t)hs[i] * P.n + r];
+      t[i].list = P.cols + (size_t)hs[i] * tri + (size_t)r * (r + 1) / 2;
+      if (P.b < 128 && r + 1 < P.n) {
+        t[i].cnt1 = P.counts[(size_t)hs[i] * P.n + r + 1];
+        t[i].list1 = P.cols + (size_t)hs[i] * tri + (size_t)(r + 1) * (r + 2) / 2;
+      }
     }
   }
 }
@@ -137,13 +145,32 @@ __device__ inline void attn_pair_tiles(const AttnParams &P, int pair, AttnTile (
 // (coalesced loads by 64 lanes), so the producer and the MMA issuer walk the
 // union without global-memory round trips.
 constexpr int kMaxChunkWords = 64;  // 2048 chunks: S/128 <= 2048 for S/b <= 1024, b <= 256
+constexpr int kMaxBlockWords = 32;  // b = 64: 1024 key blocks, one bit each
 
-__device__ inline void build_chunk_bitmap(const AttnTile &t, int per, uint32_t *bm, int lane64) {
+// b >= 128: chunk kc is attended when its block kc*128/b is listed.  b = 64:
+// chunk kc when block 2kc or 2kc+1 is listed for either query block, and
+// blk0 / blk1 get the listed key blocks of the tile's two query blocks.
+__device__ inline void build_chunk_bitmap(const AttnTile &t, int b, uint32_t *bm, uint32_t *blk0, uint32_t *blk1,
+                                          int lane64) {
   if (!t.valid) return;
-  for (int e = lane64; e < t.cnt; e += 64) {
-    const int c = t.list[e];
-    for (int k = 0; k < per; ++k) {
-      const int kc = c * per + k;
+  if (b >= 128) {
+    const int per = b / 128;
+    for (int e = lane64; e < t.cnt; e += 64) {
+      const int c = t.list[e];
+      for (int k = 0; k < per; ++k) {
+        const int kc = c * per + k;
+        if (kc <= t.qc) atomicOr(&bm[kc >> 5], 1u << (kc & 31));
+      }
+    }
+    return;
+  }
+  for (int rb = 0; rb < 2; ++rb) {
+    const int *list = rb ? t.list1 : t.list;
+    const int cnt = rb ? t.cnt1 : t.cnt;
+    uint32_t *blk = rb ? blk1 : blk0;
+    for (int e = lane64; e < cnt; e += 64) {
+      const int c = list[e], kc = c >> 1;
+      atomicOr(&blk[c >> 5], 1u << (c & 31));
       if (kc <= t.qc) atomicOr(&bm[kc >> 5], 1u << (kc & 31));
     }
   }
@@ -187,12 +214,12 @@ __global__ void __launch_bounds__(608, 1)
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   __shared__ uint32_t chunk_bm[2][kMaxChunkWords];
+  __shared__ uint32_t block_bm[2][2][kMaxBlockWords];  // b = 64: [tile][query block][key-block bits]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   AttnTile tl[2];
   attn_pair_tiles(P, blockIdx.x, tl);
   const int kvh = tl[0].h / P.g;
-  const int per = P.b / 128;
   const int words = (max(tl[0].qc, tl[1].valid ? tl[1].qc : 0) >> 5) + 1;
 
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
@@ -217,6 +244,7 @@ __global__ void __launch_bounds__(608, 1)
     fence_mbar_init();
   }
   for (int i = threadIdx.x; i < 2 * kMaxChunkWords; i += blockDim.x) (&chunk_bm[0][0])[i] = 0u;
+  for (int i = threadIdx.x; i < 4 * kMaxBlockWords; i += blockDim.x) (&block_bm[0][0][0])[i] = 0u;
   if (warp == 17) {
     tmem_alloc(smem_u32(&tmem_base_sh), 512);
     tmem_relinquish();
@@ -224,8 +252,8 @@ __global__ void __launch_bounds__(608, 1)
   __syncthreads();
   if (warp == 16 || warp == 17) {
     const int lane64 = threadIdx.x - 512;
-    build_chunk_bitmap(tl[0], per, chunk_bm[0], lane64);
-    build_chunk_bitmap(tl[1], per, chunk_bm[1], lane64);
+    build_chunk_bitmap(tl[0], P.b, chunk_bm[0], block_bm[0][0], block_bm[0][1], lane64);
+    build_chunk_bitmap(tl[1], P.b, chunk_bm[1], block_bm[1][0], block_bm[1][1], lane64);
   }
   tc_fence_before();
   __syncthreads();
@@ -367,8 +395,17 @@ __global__ void __launch_bounds__(608, 1)
     if (I8 && me.valid) scale2 *= P.q_scale[me.h] * P.k_scale[kvh];
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
-    const int L = me.L;
+    // this tile's chunks, ascending: the entries its S tile receives
+    int L = 0;
+    if (me.valid)
+      for (int w = 0; w < words; ++w) L += __popc(chunk_bm[t][w]);
+    int wi = 0;
+    uint32_t cur = me.valid ? chunk_bm[t][0] : 0u;
+    const uint32_t *vis_bm = block_bm[t][lq >= 2 ? 1 : 0];  // b = 64: this warp's query block
     for (int j = 0; j < L; ++j) {
+      while (cur == 0u) cur = chunk_bm[t][++wi];
+      const int kc = wi * 32 + (__ffs(cur) - 1);
+      cur &= cur - 1u;
       if (!mbar_wait(smem_u32(&bar_sfull[t]), j & 1, abort_flag, P.err)) { ok = false; break; }
       tc_fence_after();
       uint32_t rr[64];
@@ -377,6 +414,14 @@ __global__ void __launch_bounds__(608, 1)
       float s[64];
 #pragma unroll
       for (int e = 0; e < 64; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
+      if (P.b < 128) {
+        // the warp's quadrant is one (query block, key block 2kc + ch) pair
+        const int kb = 2 * kc + ch;
+        if (!((vis_bm[kb >> 5] >> (kb & 31)) & 1u)) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e) s[e] = -INFINITY;
+        }
+      }
       if (j == L - 1) {
         // diagonal chunk: key 64ch+e of the chunk is visible iff it is <= row
 #pragma unroll
@@ -404,6 +449,8 @@ __global__ void __launch_bounds__(608, 1)
       const bool raise = rmax2 > m_ref + 8.f;
       const float m_new = raise ? rmax2 : m_ref;
       const float alpha = raise ? ex2(m_ref - m_new) : 1.f;
+      // a row that has seen no visible key yet keeps m = -inf and P = 0
+      const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
       // P in bf16 (the P.V operand); the row sum adds the same rounded values
       uint32_t pk[32];
       float r8[8];
@@ -415,13 +462,13 @@ __global__ void __launch_bounds__(608, 1)
       if (C::kExpFmaEvery > 0 && j != L - 1) {
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
-          const float x0 = fmaf(s[e], scale2, -m_new), x1 = fmaf(s[e + 1], scale2, -m_new);
+          const float x0 = fmaf(s[e], scale2, -m_sub), x1 = fmaf(s[e + 1], scale2, -m_sub);
           const bool f1 = ((e + 1) % (C::kExpFmaEvery > 0 ? C::kExpFmaEvery : 1)) == 0;
           pk[e >> 1] = pack_bf16x2(ex2(x0), f1 ? ex2_fma(x1) : ex2(x1));
         }
       } else {
         // exponent arguments two at a time (packed fp32 FMA), then MUFU ex2
-        const uint64_t sc2 = f2_pack(scale2, scale2), nm2 = f2_pack(-m_new, -m_new);
+        const uint64_t sc2 = f2_pack(scale2, scale2), nm2 = f2_pack(-m_sub, -m_sub);
 #pragma unroll
         for (int e = 0; e < 64; e += 2) {
           float x0, x1;

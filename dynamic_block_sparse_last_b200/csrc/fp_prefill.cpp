@@ -69,7 +69,7 @@ void release(fp_prefill *p) {
 // Shapes fp_index_create accepts (checked here too so that nothing is
 // allocated for a shape it would reject).
 bool shape_ok(int S, int Hq, int Hkv, int d, int b) {
-  if (d != 128 || (b != 128 && b != 256)) return false;
+  if (d != 128 || (b != 64 && b != 128 && b != 256)) return false;
   if (S <= 0 || (S + b - 1) / b > 1024) return false;
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return false;
   if ((int64_t)Hq * S > (int64_t)INT32_MAX) return false;

@@ -25,6 +25,7 @@ static __device__ int g_fp_dev_error;
 
 struct fp_index {
   int S, Hq, Hkv, d, b, n, nch, g;
+  int npart;               // column parts of the statistics: nch, or 2 nch when b = 64 (one per block)
   int ld;                  // rows from one head to the next in q, k, v, out (S, or T when packed)
   int device;
   int built;
@@ -32,10 +33,10 @@ struct fp_index {
   int R2, chunks_per_part;
   void *slab;
   size_t slab_bytes;
-  float *pm, *plo, *phi;   // [Hq][nch][b]
+  float *pm, *plo, *phi;   // [Hq][npart][b]
   float *partM, *partL;    // [Hq][R2][b]
-  float *LOc, *HIc;        // [Hq][nch]
-  float *ksum;             // [Hkv][nch][128]
+  float *LOc, *HIc;        // [Hq][npart]
+  float *ksum;             // [Hkv][npart][128]
   float *kbar;             // [Hkv][n][128]
   float *qbar;             // [Hq][n][128]
   float *vhat, *shat, *pest;  // [Hq][n]
@@ -100,7 +101,7 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool shape_ok(int S, int Hq, int Hkv, int d, int b) {
   if (d != 128) return false;
-  if (b != 128 && b != 256) return false;
+  if (b != 64 && b != 128 && b != 256) return false;
   if (S <= 0 || (S + b - 1) / b > kSelMaxN) return false;
   if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return false;
   if ((int64_t)Hq * S > (int64_t)INT32_MAX || (int64_t)Hkv * S > (int64_t)INT32_MAX) return false;
@@ -142,7 +143,8 @@ int set_smem_attrs() {
 // Shape, inputs and scratch of the pattern-statistics launches (steps 1-3 of
 // fp_build_index), shared by the index build and the allocation-free call.
 struct StatsJob {
-  int S, Hq, Hkv, d, b, n, nch, g, R2, chunks_per_part;
+  int S, Hq, Hkv, d, b, n, nch, g, R2, chunks_per_part;  // R2, chunks_per_part over the npart parts
+  int npart;  // column parts: nch, or 2 nch when b = 64
   int ld;  // rows from one head to the next
   const void *q, *k;
   const float *q_scale, *k_scale;  // int8 only
@@ -171,6 +173,7 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   R = (J.nch + cpc - 1) / cpc;
   ScoreParams sp;
   sp.S = J.S; sp.Hq = J.Hq; sp.Hkv = J.Hkv; sp.b = J.b; sp.n = J.n; sp.nch = J.nch; sp.g = J.g;
+  sp.nsub = J.npart / J.nch;
   sp.ld = J.ld;
   sp.nlast = nlast;
   sp.tiles_per_head = tiles_per_head;
@@ -183,20 +186,20 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   sp.err = err;
   k_score_last<I8><<<dim3(R, tgroups, J.Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
   if ((rc = launch_status())) return rc;
-  k_row_stats<<<dim3(J.Hq, J.R2), J.b, 0, st>>>(J.pm, J.plo, J.phi, J.nch, J.b, nlast, J.chunks_per_part,
+  k_row_stats<<<dim3(J.Hq, J.R2), J.b, 0, st>>>(J.pm, J.plo, J.phi, J.npart, J.b, nlast, J.chunks_per_part,
                                                 J.partM, J.partL);
   if ((rc = launch_status())) return rc;
   const size_t red_bytes = (size_t)(J.b / 32) * J.chunks_per_part * 2 * sizeof(float);
-  k_block_mass<<<dim3(J.Hq, J.R2), J.b, red_bytes, st>>>(J.pm, J.plo, J.phi, J.partM, J.partL, J.nch, J.b,
+  k_block_mass<<<dim3(J.Hq, J.R2), J.b, red_bytes, st>>>(J.pm, J.plo, J.phi, J.partM, J.partL, J.npart, J.b,
                                                          nlast, J.chunks_per_part, J.LOc, J.HIc);
   if ((rc = launch_status())) return rc;
   const float *kbar = J.ext_kbar;
   if (!kbar) {
-    k_kbar<<<dim3(J.n, J.Hkv), 128, 0, st>>>(J.ksum, I8 ? J.k_scale : nullptr, J.S, J.nch, J.b, J.n, J.kbar);
+    k_kbar<<<dim3(J.n, J.Hkv), 128, 0, st>>>(J.ksum, I8 ? J.k_scale : nullptr, J.S, J.npart, J.b, J.n, J.kbar);
     if ((rc = launch_status())) return rc;
     kbar = J.kbar;
   }
-  k_pattern<I8><<<J.Hq, 1024, 0, st>>>(J.q, J.q_scale, J.LOc, J.HIc, kbar, J.S, J.ld, J.g, J.b, J.n, J.nch,
+  k_pattern<I8><<<J.Hq, 1024, 0, st>>>(J.q, J.q_scale, J.LOc, J.HIc, kbar, J.S, J.ld, J.g, J.b, J.n, J.npart,
                                        1.0f / sqrtf((float)J.d), J.tau, J.vhat, J.shat, J.pest, J.jsd,
                                        J.pattern);
   return launch_status();
@@ -222,6 +225,7 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   if (!err) return FP_ERR_CUDA;
   StatsJob J;
   J.S = I->S; J.Hq = I->Hq; J.Hkv = I->Hkv; J.d = I->d; J.b = I->b; J.n = I->n; J.nch = I->nch; J.g = I->g;
+  J.npart = I->npart;
   J.R2 = I->R2; J.chunks_per_part = I->chunks_per_part; J.ld = I->ld;
   J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
   J.pm = I->pm; J.plo = I->plo; J.phi = I->phi; J.partM = I->partM; J.partL = I->partL;
@@ -287,9 +291,10 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   if (!I) return FP_ERR_CUDA;
   I->S = S; I->Hq = Hq; I->Hkv = Hkv; I->d = d; I->b = b; I->ld = ld;
   I->n = (S + b - 1) / b; I->nch = (S + 127) / 128; I->g = Hq / Hkv;
-  row_parts(I->nch, I->R2, I->chunks_per_part);
+  I->npart = b < 128 ? I->nch * (128 / b) : I->nch;
+  row_parts(I->npart, I->R2, I->chunks_per_part);
   cudaGetDevice(&I->device);
-  const size_t n = I->n, nch = I->nch, bb = b;
+  const size_t n = I->n, nch = I->npart, bb = b;  // statistics arrays are per column part
   const size_t tri = n * (n + 1) / 2;
   size_t need = 0;
   auto add = [&](size_t bytes) { need += ((bytes + 255) / 256) * 256; };
@@ -521,11 +526,11 @@ template <bool I8>
 int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int d, int b, float tau,
                        const float *q_scale, const float *k_scale, float *vhat, float *shat, float *pest,
                        float *jsd, int32_t *pattern, cudaStream_t st) {
-  const int n = (S + b - 1) / b, nch = (S + 127) / 128;
+  const int n = (S + b - 1) / b, nch = (S + 127) / 128, npart = b < 128 ? nch * (128 / b) : nch;
   int R2, cpp;
-  row_parts(nch, R2, cpp);
-  const size_t e_part = (size_t)Hq * nch * b, e_rs = (size_t)Hq * R2 * b, e_blk = (size_t)Hq * nch;
-  const size_t e_ksum = (size_t)Hkv * nch * 128, e_kbar = (size_t)Hkv * n * 128;
+  row_parts(npart, R2, cpp);
+  const size_t e_part = (size_t)Hq * npart * b, e_rs = (size_t)Hq * R2 * b, e_blk = (size_t)Hq * npart;
+  const size_t e_ksum = (size_t)Hkv * npart * 128, e_kbar = (size_t)Hkv * n * 128;
   const size_t need = 3 * round256(e_part * 4) + 2 * round256(e_rs * 4) + 2 * round256(e_blk * 4) +
                       round256(e_ksum * 4) + round256(e_kbar * 4);
   if (need > kNoAllocScratchBytes) return FP_ERR_ARG;
@@ -543,6 +548,7 @@ int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int
 
   StatsJob J;
   J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.d = d; J.b = b; J.n = n; J.nch = nch; J.g = Hq / Hkv;
+  J.npart = npart;
   J.R2 = R2; J.chunks_per_part = cpp; J.ld = S; J.ext_kbar = nullptr;
   J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
   J.pm = pm; J.plo = plo; J.phi = phi; J.partM = partM; J.partL = partL;

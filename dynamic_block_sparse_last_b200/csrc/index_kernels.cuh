@@ -51,6 +51,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ---------------------------------------------------------------------------
 struct ScoreParams {
   int S, Hq, Hkv, b, n, nch, g;
+  int nsub;             // column parts per 128-key chunk: 2 when b = 64 (one per block), else 1
   int ld;               // rows from one head to the next (S, or more for packed sequences)
   int nlast;            // rows of the last block, S - (n-1)b
   int tiles_per_head;   // ceil(nlast / 128)
@@ -59,8 +60,8 @@ struct ScoreParams {
   float scale2;          // log2(e)/sqrt(d) (bf16); int8: multiplied by per-head scales
   const float *q_scale;  // int8 only
   const float *k_scale;
-  float *pm, *plo, *phi;  // [Hq][nch][b]
-  float *ksum;            // [Hkv][nch][128]
+  float *pm, *plo, *phi;  // [Hq][nch * nsub][b]: per (head, column part, last-block row)
+  float *ksum;            // [Hkv][nch * nsub][128]: K column sums per part
   int *err;
 };
 
@@ -210,14 +211,18 @@ __global__ void __launch_bounds__(736, 1)
           const int st = u % C::kStages;
           if (!mbar_wait(smem_u32(&bar_kfull[st]), (u / C::kStages) & 1, abort_flag, P.err)) break;
           const uint8_t *tile = k_gen + st * C::kTileBytes;
-          float *out = P.ksum + ((size_t)kvh * P.nch + (ch0 + u)) * 128 + kh * 64;
           const int nrows = min(128, P.S - (ch0 + u) * 128);
+          // one column sum per part: rows [sub*prow, (sub+1)*prow) of the chunk
+          const int prow = 128 / P.nsub;
+          for (int sub = 0; sub < P.nsub; ++sub) {
+          float *out = P.ksum + ((size_t)kvh * P.nch * P.nsub + (size_t)(ch0 + u) * P.nsub + sub) * 128 + kh * 64;
+          const int r_lo = sub * prow, r_hi = min(nrows, r_lo + prow);
           if (I8) {
             // one 128-byte row per key; lane owns bytes 64kh + 2lane, +1
             const int c16 = 4 * kh + (lane >> 3), within = (2 * lane) & 15;
             int acc0 = 0, acc1 = 0;
 #pragma unroll 4
-            for (int r = 0; r < nrows; ++r) {
+            for (int r = r_lo; r < r_hi; ++r) {
               const int phys = ((c16 ^ (r & 7)) << 4) | within;
               const uint32_t w = *reinterpret_cast<const uint16_t *>(tile + r * 128 + phys);
               acc0 += (int)(int8_t)(w & 0xff);
@@ -236,18 +241,19 @@ __global__ void __launch_bounds__(736, 1)
               const uint32_t w = *reinterpret_cast<const uint32_t *>(hsrc + r * 128 + (((c16 ^ (r & 7)) << 4) | within));
               return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
             };
-            int r = 0;
+            int r = r_lo;
 #pragma unroll 2
-            for (; r + 1 < nrows; r += 2) {
+            for (; r + 1 < r_hi; r += 2) {
               ae = f2_add(ae, row_pair(r));
               ao = f2_add(ao, row_pair(r + 1));
             }
-            if (r < nrows) ae = f2_add(ae, row_pair(r));
+            if (r < r_hi) ae = f2_add(ae, row_pair(r));
             float x0, x1, y0, y1;
             f2_unpack(ae, x0, x1);
             f2_unpack(ao, y0, y1);
             out[2 * lane] = x0 + y0;
             out[2 * lane + 1] = x1 + y1;
+          }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bar_kempty[st]));
@@ -265,17 +271,22 @@ __global__ void __launch_bounds__(736, 1)
         if (I8) scale2 *= P.q_scale[hh] * P.k_scale[kvh];
         const uint32_t taddr = tmem + t * 128 + (((warp & 3) * 32) << 16);
         bool ok = true;
+        float m = -INFINITY;
+        float lo4[4] = {0.f, 0.f, 0.f, 0.f}, hi4[4] = {0.f, 0.f, 0.f, 0.f};
         for (int u = 0; u < U && ok; ++u) {
           const int ch = ch0 + u;
-          const int tb = (ch * 128) % P.b;                 // chunk offset inside its block
-          const bool last_block = (ch * 128) / P.b == P.n - 1;
           // One pass over the chunk in 32-column pieces with an online max:
           // lo/hi are kept relative to the running max m and rescaled when a
           // piece raises it.  Columns t <= i (block-relative) go to lo, the
           // rest to hi; in the last block columns t > i are causally masked.
-          float m = -INFINITY;
-          float lo4[4] = {0.f, 0.f, 0.f, 0.f}, hi4[4] = {0.f, 0.f, 0.f, 0.f};
+          // With b = 64 each 64-column half is a block of its own and gets
+          // its own (max, lo, hi) part; otherwise the chunk is one part.
           for (int hf = 0; hf < 2; ++hf) {
+            if (hf == 0 || P.nsub == 2) {
+              m = -INFINITY;
+#pragma unroll
+              for (int w4 = 0; w4 < 4; ++w4) lo4[w4] = hi4[w4] = 0.f;
+            }
             if (!mbar_wait(smem_u32(&bar_sfull[t][hf]), u & 1, abort_flag, P.err)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
@@ -283,7 +294,11 @@ __global__ void __launch_bounds__(736, 1)
               uint32_t r[32];
               tmem_ld32(taddr + hf * 64 + qq * 32, r);
               tmem_ld_wait(r);
-              const int t0 = tb + hf * 64 + qq * 32;
+              const int key0 = ch * 128 + hf * 64 + qq * 32;  // first key of the piece
+              const int blk = key0 / P.b;
+              if (blk > P.n - 1) continue;                    // past the last block: masked
+              const bool last_block = blk == P.n - 1;
+              const int t0 = key0 - blk * P.b;                // block-relative column of the piece
               const int dlt = i - t0;  // columns e <= dlt are on the lo side
               float pm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -331,17 +346,18 @@ __global__ void __launch_bounds__(736, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bar_sfree[t][hf]));
+            if ((hf == 1 || P.nsub == 2) && i < P.nlast) {
+              const float m2 = m * scale2;
+              const float lo = (lo4[0] + lo4[1]) + (lo4[2] + lo4[3]);
+              const float hi = (hi4[0] + hi4[1]) + (hi4[2] + hi4[3]);
+              const int part = ch * P.nsub + (P.nsub == 2 ? hf : 0);
+              const size_t o = ((size_t)hh * P.nch * P.nsub + part) * P.b + i;
+              P.pm[o] = m2;
+              P.plo[o] = lo;
+              P.phi[o] = hi;
+            }
           }
           if (!ok) break;
-          const float m2 = m * scale2;
-          const float lo = (lo4[0] + lo4[1]) + (lo4[2] + lo4[3]);
-          const float hi = (hi4[0] + hi4[1]) + (hi4[2] + hi4[3]);
-          if (i < P.nlast) {
-            const size_t o = ((size_t)hh * P.nch + ch) * P.b + i;
-            P.pm[o] = m2;
-            P.plo[o] = lo;
-            P.phi[o] = hi;
-          }
         }
       }
     }
@@ -462,7 +478,7 @@ __global__ void k_block_mass(const float *__restrict__ pm, const float *__restri
 __global__ void k_kbar(const float *__restrict__ ksum, const float *__restrict__ k_scale, int S, int nch,
                        int b, int n, float *__restrict__ kbar) {
   const int c = blockIdx.x, kvh = blockIdx.y, t = threadIdx.x;
-  const int per = b / 128, rows = min(b, S - c * b);
+  const int per = b >= 128 ? b / 128 : 1, rows = min(b, S - c * b);  // column parts per block
   float s = 0.f;
   for (int k = 0; k < per && c * per + k < nch; ++k) s += ksum[((size_t)kvh * nch + c * per + k) * 128 + t];
   if (k_scale) s *= k_scale[kvh];
@@ -487,7 +503,7 @@ __global__ void __launch_bounds__(1024)
   __shared__ float part[1024 / 32];
   __shared__ float lo_s[1024], hi_s[1024];
   const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int kvh = h / g, per = b / 128, nlast = S - (n - 1) * b;
+  const int kvh = h / g, per = b >= 128 ? b / 128 : 1, nlast = S - (n - 1) * b;  // parts per block
   // block masses
   for (int c = tid; c < n; c += blockDim.x) {
     float a = 0.f, e = 0.f;

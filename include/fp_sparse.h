@@ -18,8 +18,8 @@
  *
  * Conventions (all arguments): batch 1, tensors head-major and contiguous,
  * q[Hq][S][d], k[Hkv][S][d], v[Hkv][S][d], out[Hq][S][d]; query head h reads
- * KV head h / (Hq/Hkv).  Supported: d = 128, b in {128, 256}, any S >= 1 with
- * n = ceil(S/b) <= 1024 blocks, Hq a multiple of Hkv.  When b does not divide
+ * KV head h / (Hq/Hkv).  Supported: d = 128, b in {64, 128, 256}, any S >= 1
+ * with n = ceil(S/b) <= 1024 blocks, Hq a multiple of Hkv.  When b does not divide
  * S the last block is partial: it holds the S - (n-1)b rows (n-1)b .. S-1,
  * the statistics of steps 1-2 below average over those rows and every block
  * mean is taken over the rows the block actually has (the articles only

@@ -43,7 +43,7 @@ def test_strerror(fp):
 
 
 @pytest.mark.parametrize("S,Hq,Hkv,d,b", [(131073, 4, 2, 128, 128), (1024, 4, 3, 128, 128), (1024, 4, 2, 64, 128),
-                                           (1024, 4, 2, 128, 64), (0, 4, 2, 128, 128), (262144, 4, 2, 128, 128),
+                                           (1024, 4, 2, 128, 32), (0, 4, 2, 128, 128), (262144, 4, 2, 128, 128),
                                            (1024, 0, 2, 128, 128)])
 def test_create_rejects_unsupported_shapes(fp, S, Hq, Hkv, d, b):
     h = ctypes.c_void_p()
@@ -89,7 +89,7 @@ def test_varlen_create_rejects_bad_offsets(fp):
     L = fp.lib()
     h = ctypes.c_void_p()
     for cu, nseq, b in [([1, 100], 1, 128), ([0, 100, 50], 2, 128), ([0, 100], 0, 128), ([0, 131073], 1, 128),
-                        ([0, 0], 1, 128), ([0, 100], 1, 64)]:
+                        ([0, 0], 1, 128), ([0, 100], 1, 32), ([0, 65600], 1, 64)]:
         arr = (ctypes.c_int32 * len(cu))(*cu)
         assert L.fp_varlen_create(arr, nseq, 4, 2, 128, b, ctypes.byref(h)) == fp.FP_ERR_ARG, cu
         assert h.value is None

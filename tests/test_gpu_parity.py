@@ -71,11 +71,15 @@ def check_tiles(P, exp, out, w, tiles):
     n = nblocks(w.S, w.b)
 
     def one(t):
+        # the tile's rows, query block by query block (two blocks per tile when b = 64)
         h, qc = t
-        r = qc * 128 // w.b
-        rows = parity.gpu_rows(exp, h, n)[r]
-        ref = P.attn_rows(h, qc * 128, min(qc * 128 + 128, w.S), rows)
-        return ref
+        lo, hi = qc * 128, min(qc * 128 + 128, w.S)
+        lists = parity.gpu_rows(exp, h, n)
+        parts = []
+        for r in range(lo // w.b, (hi - 1) // w.b + 1):
+            a, z = max(lo, r * w.b), min(hi, (r + 1) * w.b)
+            parts.append(P.attn_rows(h, a, z, lists[r]))
+        return np.concatenate(parts, 0)
 
     refs = parity.run_parallel(one, tiles)
     worst_max, sum_mean = 0.0, 0.0
@@ -108,6 +112,12 @@ SMALL = [
     synth.Workload("ragged_single_block", S=77, Hq=2, Hkv=2, b=256, seed=20),
     synth.Workload("ragged_int8", S=2000, Hq=4, Hkv=2, b=128, int8=True, seed=21),
     synth.Workload("ragged_int8_b256", S=1800, Hq=4, Hkv=2, b=256, gamma=0.95, int8=True, seed=22),
+    # block size 64: two query blocks per 128-row tile, two key blocks per chunk
+    synth.Workload("b64", S=1024, Hq=4, Hkv=2, b=64, seed=24),
+    synth.Workload("b64_ragged", S=1000, Hq=4, Hkv=2, b=64, gamma=0.95, seed=25),
+    synth.Workload("b64_odd_blocks", S=1088, Hq=2, Hkv=1, b=64, seed=26),
+    synth.Workload("b64_g1", S=1536, Hq=2, Hkv=2, b=64, gamma=0.8, seed=27),
+    synth.Workload("b64_int8", S=2048, Hq=4, Hkv=2, b=64, int8=True, seed=28),
 ]
 
 
@@ -127,7 +137,8 @@ DENSE = [synth.Workload("dense", S=2048, Hq=8, Hkv=2, b=128, gamma=1.0, seed=13)
          synth.Workload("sweep_gen_b256", S=4096, Hq=32, Hkv=8, b=256, gamma=1.0, n_vertical=64, n_topics=32,
                         seed=2),
          synth.Workload("dense_ragged_b128", S=1234, Hq=8, Hkv=2, b=128, gamma=1.0, seed=23),
-         synth.Workload("dense_ragged_b256", S=1234, Hq=8, Hkv=2, b=256, gamma=1.0, seed=23)]
+         synth.Workload("dense_ragged_b256", S=1234, Hq=8, Hkv=2, b=256, gamma=1.0, seed=23),
+         synth.Workload("dense_ragged_b64", S=1234, Hq=8, Hkv=2, b=64, gamma=1.0, seed=23)]
 
 
 @pytest.mark.parametrize("w", DENSE, ids=[w.name for w in DENSE])
