@@ -243,7 +243,7 @@ def run_ours(args, w):
     assert fp.fp_get_device_error(stream) == fp.FP_OK
     exp = fp.fp_index_export(idx, stream)
     nq = w.S // 128
-    n = w.S // w.b
+    n = (w.S + w.b - 1) // w.b
     rp = exp["row_ptr"]
     counts = np.diff(rp).reshape(w.Hq, n)
     per = w.b // 128
@@ -339,9 +339,17 @@ def run_ours(args, w):
     qa_heads = int((exp["pattern"] == 1).sum())
     idx_bytes = (w.Hkv * w.S * w.d + qa_heads * w.S * w.d + w.Hq * w.b * w.d) * elt
     idx_gbs = idx_bytes / (index_ms / 1e3) / 1e9
+    # the other floor of the pass: one exponential per (last-block row, causal key) of every head,
+    # at the 16 ex2 per clock per SM the MUFU delivers, at the SM clock sampled during the run
+    nlast = w.S - (n - 1) * w.b
+    n_exp = w.Hq * sum(w.S - nlast + i + 1 for i in range(nlast))
+    sm_hz = (clocks.get("sm_mhz") or 1965.0) * 1e6
+    mufu_floor_ms = n_exp / (16.0 * torch.cuda.get_device_properties(dev).multi_processor_count * sm_hz) * 1e3
     extra = {"roofline": roof,
              "index_pass": {"ms": index_ms, "algorithmic_bytes": idx_bytes, "achieved_gbs": idx_gbs,
-                            "frac_of_hbm": idx_gbs / peaks["hbm_gbs"], "qa_heads": qa_heads},
+                            "frac_of_hbm": idx_gbs / peaks["hbm_gbs"], "qa_heads": qa_heads,
+                            "hbm_floor_ms": idx_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
+                            "exponentials": n_exp, "mufu_floor_ms": mufu_floor_ms},
              "attn_ms": attn_ms, "density": density, "chunks": chunks,
              "e2e": e2e, "clocks": clocks, "gpu_launches": KERNELS_PER_STEP * args.steps,
              "gpu": torch.cuda.get_device_name(dev)}
@@ -385,7 +393,7 @@ def run_sweep(args):
             e[2].record()
         torch.cuda.synchronize()
         assert fp.fp_get_device_error() == fp.FP_OK
-        n = w.S // w.b
+        n = (w.S + w.b - 1) // w.b
         nnz = fp.fp_index_nnz(idx)
         idx_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
         attn_ms = float(np.median([e[1].elapsed_time(e[2]) for e in ev]))
