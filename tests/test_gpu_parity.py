@@ -206,6 +206,22 @@ def test_full_size_layers(fp, name, ntiles):
             assert np.array_equal(t.cpu().numpy(), P.qk_int_tile(h, p0, j0, 128, 128))
 
 
+LARGE_N = [synth.Workload("b64_n1024", S=65536, Hq=8, Hkv=2, b=64, n_vertical=64, n_topics=32, seed=31),
+           synth.Workload("b256_S131072", S=131072, Hq=8, Hkv=2, b=256, n_vertical=64, n_topics=32, seed=32)]
+
+
+@pytest.mark.parametrize("w", LARGE_N, ids=[w.name for w in LARGE_N])
+def test_largest_block_counts(fp, w):
+    """The largest index a block size allows or the longest layer at b = 256:
+    n = 1024 blocks of 64 (every key-block bit of the attention bitmaps in
+    use) and S = 131072 at b = 256; full index, 32 sampled tiles."""
+    x = synth.make_inputs(w)
+    exp, out, idx = run_gpu(fp, x, w)
+    P = oracle_problem(x, w)
+    check_index(P, exp, w)
+    check_tiles(P, exp, out, w, sampled_tiles(w, 32, seed=w.seed))
+
+
 def test_batched_sequences_equal_separate_calls(fp):
     """B sequences of equal length run as one call with B*Hq / B*Hkv heads
     (stacked sequence-major) and give bit-identical index and output."""
