@@ -160,7 +160,7 @@ def make_inputs(w: Workload):
         mu = q[h].to(torch.float64).mean(dim=0)
         nrm = float(mu.norm())
         mu = (mu / nrm if nrm > 0 else mu).to(torch.float32)
-        extra = torch.randperm(S - 4, generator=gen)[: min(w.n_vertical, max(S - 4, 0))] + 4
+        extra = torch.randperm(max(S - 4, 0), generator=gen)[: min(w.n_vertical, max(S - 4, 0))] + 4
         pos = torch.cat([torch.arange(min(4, S)), extra])
         k[h // g, pos] += 3.0 * mu
     out = {

@@ -118,6 +118,10 @@ SMALL = [
     synth.Workload("b64_odd_blocks", S=1088, Hq=2, Hkv=1, b=64, seed=26),
     synth.Workload("b64_g1", S=1536, Hq=2, Hkv=2, b=64, gamma=0.8, seed=27),
     synth.Workload("b64_int8", S=2048, Hq=4, Hkv=2, b=64, int8=True, seed=28),
+    # degenerate lengths: one token, three tokens, exactly one block of 64
+    synth.Workload("S1", S=1, Hq=2, Hkv=1, b=128, seed=33),
+    synth.Workload("S3_b64", S=3, Hq=2, Hkv=2, b=64, seed=34),
+    synth.Workload("S64_b64", S=64, Hq=4, Hkv=2, b=64, seed=35),
 ]
 
 
