@@ -3,7 +3,10 @@
 TEST INFRASTRUCTURE ONLY: imported by the tests, by the package smoke check
 and by the benchmark's CPU-baseline leg.  The product path never imports it.
 The oracle is compiled with the host C compiler into ``oracle/_build`` on
-first use (or by ``build()``), single-threaded, no fast-math.
+first use (or by ``build()``), single-threaded, no fast-math.  The
+environment variable ORACLE_LIB, when set, names another build of oracle.c
+to load instead; only the mutation test of the pins sets it (to builds with
+one planted mistake each).
 """
 from __future__ import annotations
 
@@ -47,7 +50,7 @@ class Problem(ctypes.Structure):
 def lib():
     global _lib
     if _lib is None:
-        L = ctypes.CDLL(build())
+        L = ctypes.CDLL(os.environ.get("ORACLE_LIB") or build())
         dp = ctypes.POINTER(ctypes.c_double)
         ip = ctypes.POINTER(ctypes.c_int32)
         pp = ctypes.POINTER(Problem)

@@ -164,6 +164,21 @@ def test_qa_scores_match_scipy_softmax():
     assert np.allclose(pe, sp_softmax(kbar @ qbar / 4.0), rtol=1e-13)
 
 
+def test_qa_scores_finite_for_large_logits():
+    """Block logits near 800 (exp overflows float64 past ~709) that differ by
+    a few units: the scores are the softmax of the differences, finite."""
+    x = np.array([0.0, 1.0, -2.0, 0.5, 3.0, -1.0])
+    kbar = np.zeros((6, 4))
+    kbar[:, 0] = 40.0
+    kbar[:, 1] = x
+    qbar = np.array([40.0, 1.0, 0.0, 0.0])  # logits (1600 + x_c) / 2
+    w = orc.row_scores(orc.QA, 5, np.zeros(6), np.zeros(6), qbar, kbar)
+    assert np.all(np.isfinite(w))
+    assert np.allclose(w, sp_softmax(x / 2.0), rtol=1e-12, atol=0)
+    pe = orc.pest(qbar, kbar)
+    assert np.all(np.isfinite(pe)) and np.allclose(pe, sp_softmax(x / 2.0), rtol=1e-12, atol=0)
+
+
 # ---------------------------------------------------------------- last-block statistics
 
 @pytest.mark.parametrize("S,b,d,int8", [(16, 4, 8, False), (24, 8, 16, False), (32, 8, 8, True),
