@@ -129,6 +129,7 @@ int set_smem_attrs() {
   static bool done[128] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(g_mu);  // first calls from several host threads
   if (dev >= 0 && dev < 128 && done[dev]) return FP_OK;
   if (cudaFuncSetAttribute(k_score_last<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            ScoreCfg<I8>::kSmem) != cudaSuccess)

@@ -71,8 +71,9 @@ void fp_prefill_free(fp_prefill *p);
  * it queues work and then restores the caller's device; `stream` must belong
  * to the pipeline's device.  Returns FP_ERR_ARG for NULL buffers or
  * out-of-range gamma/tau (nothing is queued), FP_ERR_CUDA if queueing a copy,
- * launch or event fails; device-side wait timeouts are reported by
- * fp_get_device_error as for the other calls. */
+ * launch or event fails (part of the run may then be queued: synchronise the
+ * device before reusing the buffers); device-side wait timeouts are reported
+ * by fp_get_device_error as for the other calls. */
 int fp_prefill_enqueue(fp_prefill *p, const void *h_q, const void *h_k, const void *h_v,
                        const float *h_q_scale, const float *h_k_scale, float gamma, float tau, void *h_out,
                        void *stream);
