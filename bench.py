@@ -118,6 +118,24 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def attention_peak(bf16_peak: float, int8: bool) -> float:
+    """Tensor peak for the attention's contractions: bf16 for both, or for W8A8
+    Q.K^T (half the FLOPs) as int8 at the nominal 2x of bf16 and P.V as bf16,
+    whose roofline time F/2/(2P) + F/2/P makes an effective peak of 4/3 P."""
+    return bf16_peak * 4.0 / 3.0 if int8 else bf16_peak
+
+
+def index_pass_floors(S: int, Hq: int, b: int, idx_bytes: int, hbm_gbs: float, sm_count: int, sm_mhz: float):
+    """The index pass's two floors: its algorithmic bytes at the HBM copy
+    bandwidth, and one exponential per (last-block row, causal key) of every
+    head at 16 ex2 per clock per SM.  Returns (hbm_floor_ms, n_exp, mufu_floor_ms)."""
+    n = (S + b - 1) // b
+    nlast = S - (n - 1) * b
+    n_exp = Hq * sum(S - nlast + i + 1 for i in range(nlast))
+    mufu_ms = n_exp / (16.0 * sm_count * sm_mhz * 1e6) * 1e3
+    return idx_bytes / (hbm_gbs * 1e9) * 1e3, n_exp, mufu_ms
+
+
 def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -327,13 +345,9 @@ def run_ours(args, w):
     bf16_peak = peaks["bf16_tflops_sustained"]
     src = (f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
            else "fallback 1.4 PFLOP/s sustained")
+    peak = attention_peak(bf16_peak, w.int8)
     if w.int8:
-        # Q.K^T (half the FLOPs) runs as int8 at the nominal 2x of bf16, P.V as bf16: the roofline
-        # time is F/2/(2P) + F/2/P, i.e. an effective peak of 4/3 P
-        peak = bf16_peak * 4.0 / 3.0
         src += "; int8 Q.K^T at the nominal 2x (4.5 vs 2.25 PFLOP/s dense), bf16 P.V: 4/3 of it"
-    else:
-        peak = bf16_peak
     achieved = attn_flops / (attn_ms / 1e3) / 1e12
     trec = attn_traffic_record() if not w.int8 else None  # the record is of the bf16 kernel
     roof = {"kernel": "k_sparse_attn<int8>" if w.int8 else "k_sparse_attn", "bound": "tensor",
@@ -347,16 +361,15 @@ def run_ours(args, w):
     qa_heads = int((exp["pattern"] == 1).sum())
     idx_bytes = (w.Hkv * w.S * w.d + qa_heads * w.S * w.d + w.Hq * w.b * w.d) * elt
     idx_gbs = idx_bytes / (index_ms / 1e3) / 1e9
-    # the other floor of the pass: one exponential per (last-block row, causal key) of every head,
-    # at the 16 ex2 per clock per SM the MUFU delivers, at the SM clock sampled during the run
-    nlast = w.S - (n - 1) * w.b
-    n_exp = w.Hq * sum(w.S - nlast + i + 1 for i in range(nlast))
-    sm_hz = (clocks.get("sm_mhz") or 1965.0) * 1e6
-    mufu_floor_ms = n_exp / (16.0 * torch.cuda.get_device_properties(dev).multi_processor_count * sm_hz) * 1e3
+    # the pass's floors: its bytes at the HBM copy bandwidth, and its exponentials at the MUFU
+    # rate and the SM clock sampled during the run
+    hbm_floor_ms, n_exp, mufu_floor_ms = index_pass_floors(
+        w.S, w.Hq, w.b, idx_bytes, peaks["hbm_gbs"], torch.cuda.get_device_properties(dev).multi_processor_count,
+        clocks.get("sm_mhz") or 1965.0)
     extra = {"roofline": roof,
              "index_pass": {"ms": index_ms, "algorithmic_bytes": idx_bytes, "achieved_gbs": idx_gbs,
                             "frac_of_hbm": idx_gbs / peaks["hbm_gbs"], "qa_heads": qa_heads,
-                            "hbm_floor_ms": idx_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3,
+                            "hbm_floor_ms": hbm_floor_ms,
                             "exponentials": n_exp, "mufu_floor_ms": mufu_floor_ms},
              "attn_ms": attn_ms, "density": density, "chunks": chunks,
              "e2e": e2e, "clocks": clocks, "gpu_launches": KERNELS_PER_STEP * args.steps,

@@ -77,3 +77,24 @@ def test_traffic_record_is_dropped_when_the_kernel_source_changes(tmp_path, monk
     fake.write_text("// another kernel\n")
     monkeypatch.setattr(bench, "ATTN_SRC", str(fake))
     assert bench.attn_traffic_record() is None
+
+
+def test_attention_peak_for_mixed_int8():
+    import bench
+    assert bench.attention_peak(1400.0, False) == 1400.0
+    # W8A8: half the FLOPs at 2P and half at P take 0.75 F / P
+    F, P = 1.0e15, 1400.0e12
+    t = (F / 2) / (2 * P) + (F / 2) / P
+    assert abs(bench.attention_peak(1400.0, True) * 1e12 - F / t) < 1e-3 * P
+
+
+def test_index_pass_floors():
+    import bench
+    # S = 2b: the last block's rows see b+1 .. 2b causal keys, sum = b(3b+1)/2 per head
+    hbm, n_exp, mufu = bench.index_pass_floors(256, 2, 128, 6_550_000_000, 6550.0, 148, 1000.0)
+    assert n_exp == 2 * (128 * (3 * 128 + 1) // 2)
+    assert abs(hbm - 1.0) < 1e-12
+    assert abs(mufu - n_exp / (16 * 148 * 1e9) * 1e3) < 1e-15
+    # a partial last block of 3 rows: keys S-2, S-1, S
+    _, n_exp, _ = bench.index_pass_floors(259, 1, 128, 1, 1.0, 1, 1.0)
+    assert n_exp == 257 + 258 + 259
