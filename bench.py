@@ -118,6 +118,27 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def computed_chunk_tiles(row_ptr, col, Hq: int, S: int, b: int) -> int:
+    """128 x 128 query-tile x key-chunk tiles the attention kernel computes for
+    an index in CSR form (rows h*n + r): a tile attends to every chunk of its
+    listed blocks up to its own position; with b = 64 a tile holds two query
+    blocks and a chunk two key blocks, so it computes the chunks of the union
+    of both lists."""
+    n = (S + b - 1) // b
+    nq = (S + 127) // 128
+    total = 0
+    for h in range(Hq):
+        lists = [col[row_ptr[h * n + r]: row_ptr[h * n + r + 1]] for r in range(n)]
+        for qc in range(nq):
+            if b >= 128:
+                per, r = b // 128, qc * 128 // b
+                total += (len(lists[r]) - 1) * per + qc % per + 1
+            else:
+                blocks = np.concatenate([lists[r] for r in (2 * qc, 2 * qc + 1) if r < n])
+                total += len({int(c) // 2 for c in blocks if int(c) // 2 <= qc})
+    return total
+
+
 def attention_peak(bf16_peak: float, int8: bool) -> float:
     """Tensor peak for the attention's contractions: bf16 for both, or for W8A8
     Q.K^T (half the FLOPs) as int8 at the nominal 2x of bf16 and P.V as bf16,
@@ -172,7 +193,7 @@ def oracle_sample(w, x, P, step, tiles_per_step=1):
     `tiles_per_step` 128-row tiles of that head; returns (seconds, extrapolated
     seconds per layer, description)."""
     h = step % w.Hq
-    nq = w.S // 128
+    nq = (w.S + 127) // 128
     t0 = time.perf_counter()
     o = P.build_index_head(h, w.gamma, w.tau, want_scores=False)
     t1 = time.perf_counter()
@@ -180,9 +201,10 @@ def oracle_sample(w, x, P, step, tiles_per_step=1):
     tile_t = []
     for _ in range(tiles_per_step):
         qc = int(rng.integers(0, nq))
-        r = qc * 128 // w.b
+        lo, hi = qc * 128, min(qc * 128 + 128, w.S)
         s = time.perf_counter()
-        P.attn_rows(h, qc * 128, qc * 128 + 128, o["rows"][r])
+        for r in range(lo // w.b, (hi - 1) // w.b + 1):  # the tile's query blocks
+            P.attn_rows(h, max(lo, r * w.b), min(hi, (r + 1) * w.b), o["rows"][r])
         tile_t.append(time.perf_counter() - s)
     t2 = time.perf_counter()
     per_layer = (t1 - t0) * w.Hq + float(np.mean(tile_t)) * w.Hq * nq
@@ -260,15 +282,8 @@ def run_ours(args, w):
     stream.synchronize()
     assert fp.fp_get_device_error(stream) == fp.FP_OK
     exp = fp.fp_index_export(idx, stream)
-    nq = w.S // 128
     n = (w.S + w.b - 1) // w.b
-    rp = exp["row_ptr"]
-    counts = np.diff(rp).reshape(w.Hq, n)
-    per = w.b // 128
-    chunks = 0
-    for qc in range(nq):
-        r = qc * 128 // w.b
-        chunks += int(((counts[:, r] - 1) * per + (qc % per) + 1).sum())
+    chunks = computed_chunk_tiles(exp["row_ptr"], exp["col"], w.Hq, w.S, w.b)
     attn_flops = chunks * 4.0 * 128 * 128 * 128
     density = exp["nnz"] / (w.Hq * n * (n + 1) / 2)
 

@@ -98,3 +98,29 @@ def test_index_pass_floors():
     # a partial last block of 3 rows: keys S-2, S-1, S
     _, n_exp, _ = bench.index_pass_floors(259, 1, 128, 1, 1.0, 1, 1.0)
     assert n_exp == 257 + 258 + 259
+
+
+def csr(rows_per_head):
+    rp, col = [0], []
+    for rows in rows_per_head:
+        for r in rows:
+            col += r
+            rp.append(len(col))
+    return np.array(rp), np.array(col)
+
+
+def test_computed_chunk_tiles():
+    import bench
+    # b = 128, S = 384, one head: rows [0], [0,1], [1,2] -> tiles compute 1 + 2 + 2 chunks
+    rp, col = csr([[[0], [0, 1], [1, 2]]])
+    assert bench.computed_chunk_tiles(rp, col, 1, 384, 128) == 5
+    # b = 256, S = 512: block 0 = tiles 0,1, block 1 = tiles 2,3; lists [0], [0, 1]
+    rp, col = csr([[[0], [0, 1]]])
+    assert bench.computed_chunk_tiles(rp, col, 1, 512, 256) == 1 + 2 + 3 + 4
+    # b = 64, S = 256: blocks 0..3, tile 0 = blocks 0,1, tile 1 = blocks 2,3
+    # lists: [0], [1], [0, 2], [3]: tile 0 -> chunks {0}; tile 1 -> chunks {0, 1}
+    rp, col = csr([[[0], [1], [0, 2], [3]]])
+    assert bench.computed_chunk_tiles(rp, col, 1, 256, 64) == 1 + 2
+    # b = 64 with a last tile holding one query block (S = 192: blocks 0..2)
+    rp, col = csr([[[0], [0, 1], [2]]])
+    assert bench.computed_chunk_tiles(rp, col, 1, 192, 64) == 1 + 1
