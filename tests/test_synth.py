@@ -2,6 +2,8 @@
 property, planted structure bookkeeping and the int8 quantisation bounds."""
 import math
 
+import numpy as np
+
 import torch
 
 from dynamic_block_sparse_last_b200 import synth
@@ -58,3 +60,25 @@ def test_int8_quantisation_bounds():
 def test_dense_equivalent_flops():
     assert synth.dense_equiv_flops(131072, 32, 128) == 2.0 * 32 * 128 * 131072 ** 2
     assert math.isclose(synth.dense_equiv_flops(131072, 32, 128), 1.407e14, rel_tol=1e-3)
+
+
+def test_rope_tables_angles_and_rounding():
+    """cos/sin tables: fp64 angles p * theta^(-2i/d) rounded to float32."""
+    cos, sin = synth.rope_tables(300, 128)
+    assert cos.shape == (300, 64) and cos.dtype == torch.float32 and sin.dtype == torch.float32
+    p = np.arange(300)[:, None].astype(np.float64)
+    inv = synth.ROPE_THETA ** (-np.arange(64) * 2.0 / 128)
+    assert np.array_equal(cos.numpy(), np.cos(p * inv).astype(np.float32))
+    assert np.array_equal(sin.numpy(), np.sin(p * inv).astype(np.float32))
+    assert np.all(cos[0].numpy() == 1.0) and np.all(sin[0].numpy() == 0.0)
+
+
+def test_prerope_inputs_are_seeded_and_shaped():
+    w = synth.Workload("pr", S=200, Hq=4, Hkv=2, b=64, seed=7)
+    a, b = synth.make_prerope_inputs(w), synth.make_prerope_inputs(w)
+    assert a["q_in"].shape == (4, 200, 128) and a["k_in"].shape == (2, 200, 128) and a["v"].shape == (2, 200, 128)
+    assert a["q_in"].dtype == torch.bfloat16 and a["cos"].shape == (200, 64)
+    for key in ("q_in", "k_in", "v", "cos", "sin"):
+        assert torch.equal(a[key], b[key]), key
+    c = synth.make_prerope_inputs(synth.Workload("pr", S=200, Hq=4, Hkv=2, b=64, seed=8))
+    assert not torch.equal(a["q_in"], c["q_in"])
