@@ -275,14 +275,6 @@ int attn_impl(const void *q, const void *k, const void *v, const float *q_scale,
   return launch_status();
 }
 
-}  // namespace
-
-extern "C" {
-
-}  // extern "C"
-
-namespace {
-
 // Index for one sequence of S rows per head, heads ld rows apart.
 int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   if (!out) return FP_ERR_ARG;
