@@ -38,6 +38,15 @@ MUTANTS = [
     ("qa_softmax_without_max_shift", "for (int c = 0; c < m; ++c) { out[c] = exp(out[c] - mx); z += out[c]; }",
      "for (int c = 0; c < m; ++c) { out[c] = exp(out[c]); z += out[c]; }"),
     ("qa_logit_transposed", "acc += qbar[t] * kbar[(size_t)c * d + t];", "acc += qbar[c] * kbar[(size_t)t * d + c];"),
+    # wiring of the whole-head index (which operand feeds which step)
+    ("pest_from_first_block_qbar", "orc_pest(qbar + (size_t)(n - 1) * d, kbar, n, d, pest);",
+     "orc_pest(qbar, kbar, n, d, pest);"),
+    ("qa_rows_use_last_block_qbar", "orc_row_scores(*pattern, r, vhat, shat, qbar + (size_t)r * d, kbar, d, w);",
+     "orc_row_scores(*pattern, r, vhat, shat, qbar + (size_t)(n - 1) * d, kbar, d, w);"),
+    ("jsd_on_slash_not_vertical", "*jsd = orc_jsd(vhat, pest, n);", "*jsd = orc_jsd(shat, pest, n);"),
+    ("kbar_of_wrong_kv_head", "int b = P->b, d = P->d, n = nblocks(P), kvh = h / (P->Hq / P->Hkv);",
+     "int b = P->b, d = P->d, n = nblocks(P), kvh = h % P->Hkv;"),
+    ("qbar_of_kv_head_index", "orc_block_means(P, 0, h, qbar);", "orc_block_means(P, 0, kvh, qbar);"),
 ]
 
 

@@ -417,3 +417,103 @@ def test_rope_pair_norms_and_block_means():
     assert means.shape == (3, 3, 128)
     for c, (lo, hi) in enumerate(((0, 128), (128, 256), (256, 300))):
         assert np.allclose(means[:, c], out[:, lo:hi].mean(1), rtol=0, atol=1e-13)
+
+
+# ---------------------------------------------------------------- index wiring
+
+def _wiring_problem(seed):
+    """S = 48, b = 8, d = 16, Hq = 4, Hkv = 2: Q and K carry a per-block offset
+    so the block means q-bar_r, k-bar_c differ from block to block (a q-bar of
+    the wrong block, or of the wrong head, changes the result)."""
+    S, b, d, Hq, Hkv = 48, 8, 16, 4, 2
+    n = S // b
+    g = torch.Generator().manual_seed(seed)
+    qoff = torch.randn(Hq, n, 1, d, generator=g) * 1.5
+    koff = torch.randn(Hkv, n, 1, d, generator=g) * 1.5
+    q = (torch.randn(Hq, n, b, d, generator=g) + qoff).reshape(Hq, S, d).to(torch.bfloat16)
+    k = (torch.randn(Hkv, n, b, d, generator=g) + koff).reshape(Hkv, S, d).to(torch.bfloat16)
+    v = torch.randn(Hkv, S, d, generator=g).to(torch.bfloat16)
+    return orc.OracleProblem(q, k, v, b), q, k, S, b, d, Hq, Hkv
+
+
+def _index_by_hand(q, k, h, S, b, d, g):
+    """Every quantity of one head's index, computed here in torch fp64 from the
+    definitions (FAST-Prefill article 1.2 and 2.1; maplevalley article 1.1
+    steps 1-3) without the oracle."""
+    n = S // b
+    kv = h // g
+    qh, kh = q[h].double(), k[kv].double()
+    logits = (qh @ kh.T) / math.sqrt(d)
+    mask = torch.ones(S, S, dtype=torch.bool).tril()
+    A = torch.softmax(logits.masked_fill(~mask, float("-inf")), dim=-1)
+    last = A[(n - 1) * b:]
+    vhat = last.reshape(b, n, b).sum(dim=(0, 2)) / b            # column blocks of the last block's rows
+    pos = torch.arange(S)
+    p = pos[(n - 1) * b:, None]
+    off = (p - pos[None, :]).clamp(min=0) // b                  # offset block of (p, j), causal part only
+    shat = torch.zeros(n, dtype=torch.float64).index_add_(0, off.flatten(), last.flatten()) / b
+    qbar = qh.reshape(n, b, d).mean(1)
+    kbar = kh.reshape(n, b, d).mean(1)
+    pest = torch.softmax(kbar @ qbar[n - 1] / math.sqrt(d), 0)
+    jsd = float(jensenshannon(vhat.numpy(), pest.numpy())) ** 2
+    qa = [torch.softmax(kbar[: r + 1] @ qbar[r] / math.sqrt(d), 0).numpy() for r in range(n)]
+    vs = []
+    for r in range(n):
+        wr = torch.stack([vhat[c] + shat[r - c] for c in range(r + 1)])
+        vs.append((wr / wr.sum()).numpy())
+    return vhat.numpy(), shat.numpy(), pest.numpy(), jsd, qa, vs
+
+
+@pytest.mark.parametrize("seed", [31, 32])
+def test_index_head_wiring_matches_hand_computation(seed):
+    """orc_build_index_head feeds the right operands to each step: P_est from
+    the LAST block's q-bar, the JSD between v-hat and P_est, query-aware row r
+    scored with q-bar_r against k-bar of the head's own KV head, vertical-slash
+    row r from v-hat[c] + s-hat[r-c]; then the pattern rule and the selection
+    (diagonal forced, score descending, minimal count reaching gamma)."""
+    P, q, k, S, b, d, Hq, Hkv = _wiring_problem(seed)
+    n, g = S // b, Hq // Hkv
+    gamma = 0.8
+    for h in range(Hq):
+        vhat, shat, pest, jsd, qa, vs = _index_by_hand(q, k, h, S, b, d, g)
+        assert not np.allclose(vhat, shat, atol=1e-3)           # the two statistics really differ
+        for tau, pat in ((jsd * 1.01, orc.QA), (jsd * 0.99, orc.VS)):
+            out = P.build_index_head(h, gamma, tau)
+            assert np.allclose(out["vhat"], vhat, atol=1e-14)
+            assert np.allclose(out["shat"], shat, atol=1e-14)
+            assert np.allclose(out["pest"], pest, rtol=1e-12, atol=1e-15)
+            assert abs(out["jsd"] - jsd) < 1e-12
+            assert out["pattern"] == pat
+            ref = qa if pat == orc.QA else vs
+            for r in range(n):
+                assert np.allclose(out["scores"][r], ref[r], rtol=1e-12, atol=1e-15), (h, pat, r)
+                row = list(out["rows"][r])
+                assert r in row
+                assert len(row) == brute_min_cover(ref[r], r, gamma)
+                rest = [c for c in range(r) if c not in row]
+                kept = [c for c in row if c != r]
+                if kept and rest:
+                    assert min(ref[r][kept]) >= max(ref[r][rest])
+        # Forcing a pattern switches only the row scores, not the statistics.
+        for force, ref in ((orc.QA, qa), (orc.VS, vs)):
+            out = P.build_index_head(h, gamma, 0.1, force_pattern=force)
+            assert out["pattern"] == force and abs(out["jsd"] - jsd) < 1e-12
+            for r in range(n):
+                assert np.allclose(out["scores"][r], ref[r], rtol=1e-12, atol=1e-15)
+
+
+def test_index_wiring_inputs_distinguish_the_operands():
+    """The wiring pin is only meaningful if its inputs separate the operands a
+    mistake could swap in: P_est from the first block's q-bar, or JSD against
+    s-hat, or a QA row from the last block's q-bar, differ measurably."""
+    P, q, k, S, b, d, Hq, Hkv = _wiring_problem(31)
+    n, g = S // b, Hq // Hkv
+    for h in range(Hq):
+        vhat, shat, pest, jsd, qa, vs = _index_by_hand(q, k, h, S, b, d, g)
+        qh, kh = q[h].double(), k[h // g].double()
+        qbar, kbar = qh.reshape(n, b, d).mean(1), kh.reshape(n, b, d).mean(1)
+        first = torch.softmax(kbar @ qbar[0] / math.sqrt(d), 0).numpy()
+        assert np.abs(first - pest).max() > 1e-3
+        assert abs(float(jensenshannon(shat, pest)) ** 2 - jsd) > 1e-4
+        wrong = torch.softmax(kbar[:3] @ qbar[n - 1] / math.sqrt(d), 0).numpy()
+        assert np.abs(wrong - qa[2]).max() > 1e-3
