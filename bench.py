@@ -139,11 +139,50 @@ def computed_chunk_tiles(row_ptr, col, Hq: int, S: int, b: int) -> int:
     return total
 
 
-def attention_peak(bf16_peak: float, int8: bool) -> float:
-    """Tensor peak for the attention's contractions: bf16 for both, or for W8A8
-    Q.K^T (half the FLOPs) as int8 at the nominal 2x of bf16 and P.V as bf16,
-    whose roofline time F/2/(2P) + F/2/P makes an effective peak of 4/3 P."""
-    return bf16_peak * 4.0 / 3.0 if int8 else bf16_peak
+def attention_peak(bf16_peak: float, int8_peak=None) -> float:
+    """Tensor peak for the attention's contractions.  bf16: the bf16 peak.
+    W8A8 (int8_peak given): Q.K^T (half the FLOPs) runs at the int8 peak and
+    P.V at the bf16 peak, so the roofline time of F FLOPs is
+    F/2/P_i8 + F/2/P_bf16 and the effective peak 2 / (1/P_i8 + 1/P_bf16)."""
+    if int8_peak is None:
+        return bf16_peak
+    return 2.0 / (1.0 / int8_peak + 1.0 / bf16_peak)
+
+
+def int8_gemm_peak(dev, n: int = 8192, sustain_s: float = 1.5):
+    """Measured int8 tensor throughput on this GPU: torch._int_mm (int8 x int8
+    -> int32, a library GEMM) at n^3.  burst = best of 10 single launches;
+    sustained = mean over a loop of about sustain_s seconds (the power-capped
+    figure, for kernels timed inside a long step).  TOPS = 2 n^3 / t.
+    Returns a dict, or None when the library call is unavailable."""
+    try:
+        a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+        for _ in range(3):
+            torch._int_mm(a, b)
+        torch.cuda.synchronize(dev)
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._int_mm(a, b)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            best = min(best, e0.elapsed_time(e1))
+        reps = max(10, int(sustain_s * 1e3 / best))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        mean = e0.elapsed_time(e1) / reps
+        flops = 2.0 * n ** 3
+        del a, b
+        return {"burst_tops": flops / (best / 1e3) / 1e12, "sustained_tops": flops / (mean / 1e3) / 1e12,
+                "n": n, "reps": reps, "how": "torch._int_mm int8 x int8 -> int32, CUDA events"}
+    except (RuntimeError, AttributeError) as e:  # library call missing for this shape or build
+        return {"unavailable": str(e).splitlines()[0][:200]}
 
 
 def index_pass_floors(S: int, Hq: int, b: int, idx_bytes: int, hbm_gbs: float, sm_count: int, sm_mhz: float):
@@ -188,29 +227,58 @@ def make_line(args, w, value, ms_per_step, extra):
 
 # ----------------------------------------------------------------------------- oracle (CPU)
 
-def oracle_sample(w, x, P, step, tiles_per_step=1):
-    """One bounded oracle sample: the full index of one head plus attention of
-    `tiles_per_step` 128-row tiles of that head; returns (seconds, extrapolated
-    seconds per layer, description)."""
-    h = step % w.Hq
+def oracle_sample(w, P, seed, heads, tiles, threads):
+    """A bounded oracle sample of the workload: the full index of `heads`
+    query heads (both patterns' kinds) and the attention of `tiles` seeded
+    128-row query tiles, spread over `threads` host threads; every item is
+    timed by its own thread's CPU clock.  The layer estimate scales the mean
+    item times to all Hq heads and Hq*ceil(S/128) tiles (extrapolated).
+    Returns a dict with the per-layer CPU seconds, the estimate on `threads`
+    cores, and the spread of the item times."""
+    import concurrent.futures as cf
+    rng = np.random.default_rng(seed)
     nq = (w.S + 127) // 128
-    t0 = time.perf_counter()
-    o = P.build_index_head(h, w.gamma, w.tau, want_scores=False)
-    t1 = time.perf_counter()
-    rng = np.random.default_rng(1000 + step)
-    tile_t = []
-    for _ in range(tiles_per_step):
-        qc = int(rng.integers(0, nq))
+    kinds = w.head_kinds()
+    vs = [h for h in range(w.Hq) if kinds[h] == "vs"]
+    qa = [h for h in range(w.Hq) if kinds[h] != "vs"]
+    pick = []
+    for i in range(heads):
+        pool = (vs if i % 2 == 0 else qa) or list(range(w.Hq))
+        pick.append(int(pool[int(rng.integers(0, len(pool)))]))
+    tile_list = [(int(rng.integers(0, w.Hq)), int(rng.integers(0, nq))) for _ in range(tiles)]
+
+    def index_item(h):
+        t0 = time.thread_time()
+        o = P.build_index_head(h, w.gamma, w.tau, want_scores=False)
+        return time.thread_time() - t0, o["rows"]
+
+    def tile_item(t, rows_of):
+        h, qc = t
         lo, hi = qc * 128, min(qc * 128 + 128, w.S)
-        s = time.perf_counter()
+        t0 = time.thread_time()
         for r in range(lo // w.b, (hi - 1) // w.b + 1):  # the tile's query blocks
-            P.attn_rows(h, max(lo, r * w.b), min(hi, (r + 1) * w.b), o["rows"][r])
-        tile_t.append(time.perf_counter() - s)
-    t2 = time.perf_counter()
-    per_layer = (t1 - t0) * w.Hq + float(np.mean(tile_t)) * w.Hq * nq
-    desc = (f"oracle index of head {h} ({t1 - t0:.2f} s) x {w.Hq} heads + {tiles_per_step} attention "
-            f"tile(s) of 128 rows ({np.mean(tile_t):.2f} s mean) x {w.Hq * nq} tiles; 1 thread; extrapolated")
-    return t2 - t0, per_layer, desc
+            P.attn_rows(h, max(lo, r * w.b), min(hi, (r + 1) * w.b), rows_of[r])
+        return time.thread_time() - t0
+
+    wall0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        idx_res = list(ex.map(index_item, pick))
+        # attention tiles use the rows of a head whose index was just built (same kind of
+        # structure), so no extra index is built inside the timed items
+        rows_by_head = {h: rows for h, (_, rows) in zip(pick, idx_res)}
+        tile_list = [(pick[i % len(pick)], qc) for i, (_, qc) in enumerate(tile_list)]
+        tile_t = list(ex.map(lambda t: tile_item(t, rows_by_head[t[0]]), tile_list))
+    wall = time.perf_counter() - wall0
+    head_t = [t for t, _ in idx_res]
+    layer_cpu_s = float(np.mean(head_t)) * w.Hq + float(np.mean(tile_t)) * w.Hq * nq
+    spread = {"index_head_s": [float(min(head_t)), float(np.median(head_t)), float(max(head_t))],
+              "tile_s": [float(min(tile_t)), float(np.median(tile_t)), float(max(tile_t))]}
+    desc = (f"oracle (fp64, one head or tile per thread) on {threads} host threads: full index of {heads} heads "
+            f"(vertical-slash and query-aware kinds, {np.mean(head_t):.2f} s CPU each) and {tiles} seeded 128-row "
+            f"attention tiles ({np.mean(tile_t):.3f} s CPU each), each timed by its thread's CPU clock; "
+            f"extrapolated to {w.Hq} heads and {w.Hq * nq} tiles; per-layer = CPU seconds / {threads} cores")
+    return {"layer_cpu_s": layer_cpu_s, "layer_s": layer_cpu_s / threads, "threads": threads, "wall_s": wall,
+            "spread_min_median_max": spread, "desc": desc}
 
 
 def oracle_problem(w, x):
@@ -228,20 +296,27 @@ def run_reference(args, w):
     x = synth.make_inputs(w)
     P = oracle_problem(w, x)
     dense = synth.dense_equiv_flops(w.S, w.Hq, w.d)
+    threads = max(1, min(8, os.cpu_count() or 1))
     for s in range(args.warmup):
-        oracle_sample(w, x, P, s)
-    per_layer, wall, desc = [], 0.0, ""
+        oracle_sample(w, P, 500 + s, heads=1, tiles=2, threads=threads)
+    per_layer, cpu_s, wall = [], [], 0.0
+    res = None
     for s in range(args.steps):
-        t, pl, desc = oracle_sample(w, x, P, args.warmup + s)
-        wall += t
-        per_layer.append(pl)
+        res = oracle_sample(w, P, 1000 + s, heads=2, tiles=threads, threads=threads)
+        wall += res["wall_s"]
+        per_layer.append(res["layer_s"])
+        cpu_s.append(res["layer_cpu_s"])
     layer_s = float(np.mean(per_layer))
     value = dense / layer_s / 1e12
-    cpu = {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc}
+    cpu = {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+           "sample": f"{args.steps} steps, each: " + res["desc"],
+           "layer_cpu_s_one_thread": float(np.mean(cpu_s)),
+           "layer_s_spread_over_steps": [float(min(per_layer)), float(np.median(per_layer)), float(max(per_layer))],
+           "host_cpus": os.cpu_count()}
     line = make_line(args, w, value, layer_s * 1e3,
                      {"impl": "reference", "cpu_baseline": cpu,
                       "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-                      "reference_note": f"fp64 oracle on host cores, {args.steps} bounded samples "
+                      "reference_note": f"fp64 oracle on {threads} host threads, {args.steps} bounded samples "
                                         f"({wall:.1f} s), ms_per_step = extrapolated ms per layer"})
     print(json.dumps(line), flush=True)
     return 0
@@ -249,28 +324,12 @@ def run_reference(args, w):
 
 # ----------------------------------------------------------------------------- CUDA path
 
-def run_ours(args, w):
-    world, rank, local = dist_env()
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
-    dev = torch.device("cuda", local if world > 1 else 0)
-    torch.cuda.set_device(dev)
-    from dynamic_block_sparse_last_b200 import fp
-
-    x = synth.make_inputs(w)
-    q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
-    if w.int8:
-        qq, kk = x["q8"].to(dev), x["k8"].to(dev)
-        qs, ks = x["q_scale"].to(dev), x["k_scale"].to(dev)
-        dt = fp.FP_QK_INT8
-    else:
-        qq, kk, qs, ks, dt = q, k, None, None, fp.FP_QK_BF16
-    out = torch.empty_like(q)
+def time_layer(fp, w, qq, kk, v, qs, ks, dt, args, dev, stream, world):
+    """Warm-up, then args.steps timed steps of fp_build_index + fp_sparse_attn
+    on `stream` (CUDA events around each stage and around the whole region,
+    barrier + synchronize on both sides, clocks sampled meanwhile)."""
+    out = torch.empty(w.Hq, w.S, w.d, dtype=torch.bfloat16, device=dev)
     idx = fp.fp_index_create(w.S, w.Hq, w.Hkv, w.d, w.b)
-    stream = torch.cuda.Stream(device=dev)
 
     def step():
         fp.fp_build_index(qq, kk, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, dt, qs, ks, idx, stream)
@@ -284,10 +343,6 @@ def run_ours(args, w):
     exp = fp.fp_index_export(idx, stream)
     n = (w.S + w.b - 1) // w.b
     chunks = computed_chunk_tiles(exp["row_ptr"], exp["col"], w.Hq, w.S, w.b)
-    attn_flops = chunks * 4.0 * 128 * 128 * 128
-    density = exp["nnz"] / (w.Hq * n * (n + 1) / 2)
-
-    # timed region: K steps, events around each stage on the launching stream
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     if world > 1:
@@ -310,11 +365,40 @@ def run_ours(args, w):
     clocks = sampler.stop()
     if world > 1:
         torch.distributed.barrier()
-    total_ms = t_start.elapsed_time(t_end)
-    index_ms = float(np.mean([e[0].elapsed_time(e[1]) for e in ev]))
-    attn_ms = float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))
     assert fp.fp_get_device_error(stream) == fp.FP_OK
-    total_ms = max_over_ranks(total_ms, dev)
+    return {"idx": idx, "out": out, "exp": exp, "clocks": clocks, "chunks": chunks,
+            "attn_flops": chunks * 4.0 * 128 * 128 * 128,
+            "density": exp["nnz"] / (w.Hq * n * (n + 1) / 2),
+            "total_ms": t_start.elapsed_time(t_end),
+            "index_ms": float(np.mean([e[0].elapsed_time(e[1]) for e in ev])),
+            "attn_ms": float(np.mean([e[1].elapsed_time(e[2]) for e in ev]))}
+
+
+def run_ours(args, w):
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    from dynamic_block_sparse_last_b200 import fp
+
+    x = synth.make_inputs(w)
+    q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+    if w.int8:
+        qq, kk = x["q8"].to(dev), x["k8"].to(dev)
+        qs, ks = x["q_scale"].to(dev), x["k_scale"].to(dev)
+        dt = fp.FP_QK_INT8
+    else:
+        qq, kk, qs, ks, dt = q, k, None, None, fp.FP_QK_BF16
+    stream = torch.cuda.Stream(device=dev)
+    L = time_layer(fp, w, qq, kk, v, qs, ks, dt, args, dev, stream, world)
+    idx, out, exp, clocks = L["idx"], L["out"], L["exp"], L["clocks"]
+    chunks, attn_flops, density = L["chunks"], L["attn_flops"], L["density"]
+    index_ms, attn_ms = L["index_ms"], L["attn_ms"]
+    total_ms = max_over_ranks(L["total_ms"], dev)
     ms_per_step = total_ms / args.steps
     dense = synth.dense_equiv_flops(w.S, w.Hq, w.d)
     value = world * dense * args.steps / (total_ms / 1e3) / 1e12
@@ -360,9 +444,16 @@ def run_ours(args, w):
     bf16_peak = peaks["bf16_tflops_sustained"]
     src = (f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
            else "fallback 1.4 PFLOP/s sustained")
-    peak = attention_peak(bf16_peak, w.int8)
-    if w.int8:
-        src += "; int8 Q.K^T at the nominal 2x (4.5 vs 2.25 PFLOP/s dense), bf16 P.V: 4/3 of it"
+    i8 = int8_gemm_peak(dev) if (w.int8 or not args.no_w8a8) else None
+    i8_sus = i8.get("sustained_tops") if i8 else None
+    if w.int8 and i8_sus:
+        peak = attention_peak(bf16_peak, i8_sus)
+        src += f"; int8 Q.K^T at the measured int8 sustained {i8_sus:.0f} TOPS, bf16 P.V: 2/(1/P_i8 + 1/P_bf16)"
+    elif w.int8:
+        peak = attention_peak(bf16_peak, 2.0 * bf16_peak)
+        src += "; int8 measurement unavailable: int8 at the nominal 2x of bf16"
+    else:
+        peak = attention_peak(bf16_peak)
     achieved = attn_flops / (attn_ms / 1e3) / 1e12
     trec = attn_traffic_record() if not w.int8 else None  # the record is of the bf16 kernel
     roof = {"kernel": "k_sparse_attn<int8>" if w.int8 else "k_sparse_attn", "bound": "tensor",
@@ -389,15 +480,47 @@ def run_ours(args, w):
              "attn_ms": attn_ms, "density": density, "chunks": chunks,
              "e2e": e2e, "clocks": clocks, "gpu_launches": KERNELS_PER_STEP * args.steps,
              "gpu": torch.cuda.get_device_name(dev)}
+    extra["int8_peak"] = i8
+    if not w.int8 and not args.no_w8a8:
+        # the W8A8 variant of the same layer: Q and K quantised per head from these bf16 tensors
+        del q, k, qq, kk
+        wq = synth.Workload(w.name + "_w8a8", S=w.S, Hq=w.Hq, Hkv=w.Hkv, d=w.d, b=w.b, gamma=w.gamma, tau=w.tau,
+                            n_vertical=w.n_vertical, n_topics=w.n_topics, seed=w.seed, int8=True)
+        q8, q_sc = synth.quantize_per_head(x["q"])
+        k8, k_sc = synth.quantize_per_head(x["k"])
+        q8, k8, q_sc, k_sc = q8.to(dev), k8.to(dev), q_sc.to(dev), k_sc.to(dev)
+        idx.free()
+        L8 = time_layer(fp, wq, q8, k8, v, q_sc, k_sc, fp.FP_QK_INT8, args, dev, stream, world)
+        ms8 = max_over_ranks(L8["total_ms"], dev) / args.steps
+        pk8 = attention_peak(bf16_peak, i8_sus if i8_sus else 2.0 * bf16_peak)
+        ach8 = L8["attn_flops"] / (L8["attn_ms"] / 1e3) / 1e12
+        extra["w8a8"] = {"workload": wq.name, "ms_per_layer": ms8, "index_ms": L8["index_ms"],
+                         "attn_ms": L8["attn_ms"], "value": world * dense / (ms8 / 1e3) / 1e12, "unit": UNIT,
+                         "density": L8["density"], "chunks": L8["chunks"],
+                         "roofline": {"kernel": "k_sparse_attn<int8>", "bound": "tensor", "achieved": ach8,
+                                      "peak": pk8, "unit": "TFLOP/s", "frac": ach8 / pk8,
+                                      "peak_source": ("int8 Q.K^T at the measured int8 sustained TOPS and bf16 P.V "
+                                                      "at the bf16 sustained peak: 2/(1/P_i8 + 1/P_bf16)"
+                                                      if i8_sus else "int8 at the nominal 2x of bf16")},
+                         "clocks": L8["clocks"]}
+        extra["w8a8"]["gpu_launches"] = KERNELS_PER_STEP * args.steps
+        L8["idx"].free()
+        del q8, k8
+        idx = None
     if world == 1 and not args.no_cpu_baseline and rank == 0:
         P = oracle_problem(w, x)
-        t, per_layer, desc = oracle_sample(w, x, P, 0)
-        extra["cpu_baseline"] = {"value": synth.dense_equiv_flops(w.S, w.Hq, w.d) / per_layer / 1e12,
-                                 "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc,
-                                 "host_cpus": os.cpu_count()}
+        threads = max(1, min(16, os.cpu_count() or 1))
+        res = oracle_sample(w, P, 7, heads=4, tiles=64, threads=threads)
+        dense = synth.dense_equiv_flops(w.S, w.Hq, w.d)
+        extra["cpu_baseline"] = {"value": dense / res["layer_s"] / 1e12, "unit": UNIT, "cores": threads,
+                                 "kind": "oracle", "sample": res["desc"],
+                                 "value_one_thread": dense / res["layer_cpu_s"] / 1e12,
+                                 "spread_min_median_max": res["spread_min_median_max"],
+                                 "sample_wall_s": res["wall_s"], "host_cpus": os.cpu_count()}
     if rank == 0:
         print(json.dumps(make_line(args, w, value, ms_per_step, extra)), flush=True)
-    idx.free()
+    if idx is not None:
+        idx.free()
     if world > 1:
         torch.distributed.destroy_process_group()
     return 0
@@ -496,6 +619,35 @@ def run_rope_pool(args):
     return 0
 
 
+def run_profile_case(args):
+    """One layer of a given shape, for profiler captures of a small case:
+    --profile-case S:Hq:Hkv:b[:int8] on the 128K layer's generator (64
+    vertical positions, 32 topics, seed 2, gamma 0.9, tau 0.1); warm-up, then
+    --steps builds + attentions on one stream.  Prints one JSON line with the
+    mean times per stage (not a bench line)."""
+    from dynamic_block_sparse_last_b200 import fp
+    parts = args.profile_case.split(":")
+    S, Hq, Hkv, b = (int(v) for v in parts[:4])
+    int8 = len(parts) > 4 and parts[4] == "int8"
+    w = synth.Workload(f"profile_S{S}_Hq{Hq}_Hkv{Hkv}_b{b}" + ("_int8" if int8 else ""), S=S, Hq=Hq, Hkv=Hkv, b=b,
+                       n_vertical=64, n_topics=32, seed=2, int8=int8)
+    dev = torch.device("cuda", 0)
+    x = synth.make_inputs(w)
+    v = x["v"].to(dev)
+    if int8:
+        qq, kk = x["q8"].to(dev), x["k8"].to(dev)
+        qs, ks, dt = x["q_scale"].to(dev), x["k_scale"].to(dev), fp.FP_QK_INT8
+    else:
+        qq, kk, qs, ks, dt = x["q"].to(dev), x["k"].to(dev), None, None, fp.FP_QK_BF16
+    stream = torch.cuda.Stream(device=dev)
+    L = time_layer(fp, w, qq, kk, v, qs, ks, dt, args, dev, stream, 1)
+    print(json.dumps({"profile_case": w.name, "index_ms": L["index_ms"], "attn_ms": L["attn_ms"],
+                      "density": L["density"], "chunks": L["chunks"], "steps": args.steps,
+                      "warmup": args.warmup}), flush=True)
+    L["idx"].free()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -504,12 +656,17 @@ def main():
     ap.add_argument("--workload", default="llama8b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-w8a8", action="store_true", help="skip the W8A8 sub-record of the default line")
     ap.add_argument("--e2e-groups", type=int, default=0,
                     help="KV-head groups of the host-to-host pipeline (0 = one KV head per group)")
     ap.add_argument("--sweep", action="store_true", help="S x b x gamma sweep (one line per point)")
     ap.add_argument("--rope-pool", action="store_true",
                     help="time the rotary epilogue with block pooling and the index build on its means")
+    ap.add_argument("--profile-case", default="",
+                    help="S:Hq:Hkv:b[:int8] -- one small layer for profiler captures (not a bench line)")
     args = ap.parse_args()
+    if args.profile_case:
+        return run_profile_case(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.sweep:

@@ -59,6 +59,11 @@ struct AttnParams {
   float scale2;                    // log2(e)/sqrt(d)
   __nv_bfloat16 *out;              // [Hq][S][128]
   int *err;
+  // int8 test capture (null in normal use): the raw int32 score tile of
+  // query head cap_h, query tile cap_qc and key chunk cap_kc, copied from
+  // tensor memory before masking, row-major [128][128]
+  int32_t *cap;
+  int cap_h, cap_qc, cap_kc;
 };
 
 template <bool I8>
@@ -411,6 +416,14 @@ __global__ void __launch_bounds__(608, 1)
       uint32_t rr[64];
       tmem_ld64(s_tm, rr);
       tmem_ld_wait64(rr);
+      if constexpr (I8) {
+        if (P.cap != nullptr && me.h == P.cap_h && me.qc == P.cap_qc && kc == P.cap_kc) {
+          int4 *dst = reinterpret_cast<int4 *>(P.cap + (size_t)row * 128 + ch * 64);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            dst[e] = make_int4((int)rr[4 * e], (int)rr[4 * e + 1], (int)rr[4 * e + 2], (int)rr[4 * e + 3]);
+        }
+      }
       float s[64];
 #pragma unroll
       for (int e = 0; e < 64; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);

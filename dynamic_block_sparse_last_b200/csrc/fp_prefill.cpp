@@ -42,7 +42,10 @@ namespace {
 
 void release(fp_prefill *p) {
   if (!p) return;
-  cudaDeviceSynchronize();
+  // all of the pipeline's work runs on its own three streams
+  if (p->s_in) cudaStreamSynchronize(p->s_in);
+  if (p->s_comp) cudaStreamSynchronize(p->s_comp);
+  if (p->s_out) cudaStreamSynchronize(p->s_out);
   for (fp_index *i : p->idx) fp_index_free(i);
   for (cudaEvent_t e : p->ev_qk) if (e) cudaEventDestroy(e);
   for (cudaEvent_t e : p->ev_in) if (e) cudaEventDestroy(e);

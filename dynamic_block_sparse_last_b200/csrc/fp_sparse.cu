@@ -33,6 +33,9 @@ struct fp_index {
   int R2, chunks_per_part;
   void *slab;
   size_t slab_bytes;
+  bool slab_pooled;        // slab from the stream-ordered allocator (else cudaMalloc)
+  cudaStream_t own;        // the index's own stream: allocation and release of the slab
+  cudaEvent_t last_use;    // recorded on the caller's stream at the end of every build / attention call
   float *pm, *plo, *phi;   // [Hq][npart][b]
   float *partM, *partL;    // [Hq][R2][b]
   float *LOc, *HIc;        // [Hq][npart]
@@ -50,18 +53,78 @@ struct fp_index {
 namespace {
 
 std::mutex g_mu;
-int *g_err_ptr[128] = {nullptr};
 
-int *device_error_word() {
+// Per-device set-up (device addresses of the library's __device__ arrays,
+// raised shared-memory limits of the big kernels), valid for one context of
+// that device: a device reset destroys the primary context and everything
+// set up in it, so the entry is redone when the current context changes.
+struct DevState {
+  void *ctx;
+  int *err;                 // g_fp_dev_error
+  unsigned char *scratch;   // g_fp_stats_scratch (allocation-free call)
+  bool attrs[2];            // set_smem_attrs<false>, <true>
+};
+DevState g_dev[128] = {};
+
+// The calling thread's current context (the device's primary context once
+// the runtime has made it current), through the driver entry point.
+void *current_context() {
+  using Fn = CUresult (*)(CUcontext *);
+  static Fn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(p);
+  });
+  CUcontext c = nullptr;
+  if (!fn || fn(&c) != CUDA_SUCCESS) return nullptr;
+  if (!c) {
+    cudaFree(nullptr);  // no-op that makes the runtime's primary context current
+    if (fn(&c) != CUDA_SUCCESS) return nullptr;
+  }
+  return c;
+}
+
+// The current device's entry, refreshed when its context changed; call with
+// g_mu held.  Returns null for an unusable device.
+DevState *dev_state() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  void *ctx = current_context();
+  if (!ctx) return nullptr;
+  DevState &d = g_dev[dev];
+  if (d.ctx != ctx) d = DevState{ctx, nullptr, nullptr, {false, false}};
+  return &d;
+}
+
+// Armed int8 tile captures (fp_debug_capture_i8); read when an int8 launch
+// is prepared, so the captured tile comes from the normal launch path.
+struct CaptureI8 {
+  int32_t *score;
+  int s_h, s_slice, s_ch;
+  int32_t *attn;
+  int a_h, a_qc, a_kc;
+};
+CaptureI8 g_cap = {nullptr, 0, 0, 0, nullptr, 0, 0, 0};
+
+CaptureI8 capture_settings() {
   std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_err_ptr[dev]) {
+  return g_cap;
+}
+
+int *device_error_word() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevState *d = dev_state();
+  if (!d) return nullptr;
+  if (!d->err) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_fp_dev_error) != cudaSuccess) return nullptr;
-    g_err_ptr[dev] = static_cast<int *>(p);
+    d->err = static_cast<int *>(p);
   }
-  return g_err_ptr[dev];
+  return d->err;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -126,18 +189,17 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? FP_OK : FP_ERR_
 
 template <bool I8>
 int set_smem_attrs() {
-  static bool done[128] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lk(g_mu);  // first calls from several host threads
-  if (dev >= 0 && dev < 128 && done[dev]) return FP_OK;
+  DevState *d = dev_state();
+  if (!d) return FP_ERR_CUDA;
+  if (d->attrs[I8]) return FP_OK;
   if (cudaFuncSetAttribute(k_score_last<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            ScoreCfg<I8>::kSmem) != cudaSuccess)
     return FP_ERR_CUDA;
   if (cudaFuncSetAttribute(k_sparse_attn<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            AttnCfg<I8>::kSmem) != cudaSuccess)
     return FP_ERR_CUDA;
-  if (dev >= 0 && dev < 128) done[dev] = true;
+  d->attrs[I8] = true;
   return FP_OK;
 }
 
@@ -185,6 +247,13 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   sp.k_scale = J.k_scale;
   sp.pm = J.pm; sp.plo = J.plo; sp.phi = J.phi; sp.ksum = J.ext_kbar ? nullptr : J.ksum;
   sp.err = err;
+  sp.cap = nullptr;
+  sp.cap_h = sp.cap_slice = sp.cap_ch = 0;
+  if (I8) {
+    const CaptureI8 c = capture_settings();
+    sp.cap = c.score;
+    sp.cap_h = c.s_h; sp.cap_slice = c.s_slice; sp.cap_ch = c.s_ch;
+  }
   k_score_last<I8><<<dim3(R, tgroups, J.Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
   if ((rc = launch_status())) return rc;
   k_row_stats<<<dim3(J.Hq, J.R2), J.b, 0, st>>>(J.pm, J.plo, J.phi, J.npart, J.b, nlast, J.chunks_per_part,
@@ -247,7 +316,8 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   if ((rc = launch_status())) return rc;
   k_cut<<<(I->Hq * I->n + 7) / 8, 256, 0, st>>>(I->pattern, I->vhat, I->shat, I->zlog, I->Hq, I->n, gamma,
                                                I->counts, I->cols);
-  return launch_status();
+  if ((rc = launch_status())) return rc;
+  return cudaEventRecord(I->last_use, st) == cudaSuccess ? FP_OK : FP_ERR_CUDA;
 }
 
 template <bool I8>
@@ -270,9 +340,17 @@ int attn_impl(const void *q, const void *k, const void *v, const float *q_scale,
   ap.scale2 = kLog2e / sqrtf((float)I->d);
   ap.out = static_cast<__nv_bfloat16 *>(out);
   ap.err = err;
+  ap.cap = nullptr;
+  ap.cap_h = ap.cap_qc = ap.cap_kc = 0;
+  if (I8) {
+    const CaptureI8 c = capture_settings();
+    ap.cap = c.attn;
+    ap.cap_h = c.a_h; ap.cap_qc = c.a_qc; ap.cap_kc = c.a_kc;
+  }
   const unsigned grid = (unsigned)attn_pairs(I->Hq, I->Hkv, I->S, I->b);
   k_sparse_attn<I8><<<grid, AttnCfg<I8>::kThreads, AttnCfg<I8>::kSmem, st>>>(tq, tk, tv, ap);
-  return launch_status();
+  if ((rc = launch_status())) return rc;
+  return cudaEventRecord(I->last_use, st) == cudaSuccess ? FP_OK : FP_ERR_CUDA;
 }
 
 // Index for one sequence of S rows per head, heads ld rows apart.
@@ -303,9 +381,28 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   add((size_t)Hq * n * 4);
   add((size_t)Hq * tri * 4);
   add((size_t)Hq * tri * 4);
-  if (cudaMalloc(&I->slab, need) != cudaSuccess) {
+  if (cudaStreamCreateWithFlags(&I->own, cudaStreamNonBlocking) != cudaSuccess) {
     free(I);
     return FP_ERR_CUDA;
+  }
+  if (cudaEventCreateWithFlags(&I->last_use, cudaEventDisableTiming) != cudaSuccess) {
+    cudaStreamDestroy(I->own);
+    free(I);
+    return FP_ERR_CUDA;
+  }
+  // stream-ordered allocation, so that freeing waits for this index's work
+  // only; plain cudaMalloc where the device has no memory pools
+  I->slab_pooled = cudaMallocAsync(&I->slab, need, I->own) == cudaSuccess &&
+                   cudaStreamSynchronize(I->own) == cudaSuccess;
+  if (!I->slab_pooled) {
+    cudaGetLastError();
+    I->slab = nullptr;
+    if (cudaMalloc(&I->slab, need) != cudaSuccess) {
+      cudaEventDestroy(I->last_use);
+      cudaStreamDestroy(I->own);
+      free(I);
+      return FP_ERR_CUDA;
+    }
   }
   I->slab_bytes = need;
   char *cur = static_cast<char *>(I->slab);
@@ -341,8 +438,20 @@ int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out) {
 
 void fp_index_free(fp_index *I) {
   if (!I) return;
-  cudaDeviceSynchronize();
-  if (I->slab) cudaFree(I->slab);
+  int prev = -1;
+  if (cudaGetDevice(&prev) == cudaSuccess && prev != I->device) cudaSetDevice(I->device);
+  else prev = -1;
+  if (I->slab_pooled) {
+    // released in stream order after the index's last call; nothing else waits
+    cudaStreamWaitEvent(I->own, I->last_use, 0);
+    cudaFreeAsync(I->slab, I->own);
+  } else if (I->slab) {
+    cudaEventSynchronize(I->last_use);
+    cudaFree(I->slab);
+  }
+  cudaEventDestroy(I->last_use);
+  cudaStreamDestroy(I->own);  // returns at once; the stream's pending free still completes
+  if (prev >= 0) cudaSetDevice(prev);
   free(I);
 }
 
@@ -484,6 +593,20 @@ int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int H
   return launch_status();
 }
 
+int fp_debug_capture_i8(int which, int h, int tile, int chunk, int32_t *out) {
+  if (which != 0 && which != 1) return FP_ERR_ARG;
+  if (out && (!aligned16(out) || h < 0 || tile < 0 || chunk < 0)) return FP_ERR_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (which == 0) {
+    g_cap.score = out;
+    g_cap.s_h = h; g_cap.s_slice = tile; g_cap.s_ch = chunk;
+  } else {
+    g_cap.attn = out;
+    g_cap.a_h = h; g_cap.a_qc = tile; g_cap.a_kc = chunk;
+  }
+  return FP_OK;
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
@@ -495,22 +618,20 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;
 static __device__ __align__(256) unsigned char g_fp_stats_scratch[kNoAllocScratchBytes];
 
-std::mutex g_scratch_mu;
-unsigned char *g_scratch_ptr[128] = {nullptr};
-
 // Device address of g_fp_stats_scratch on the current device.  In host code
 // the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// once per device (with that device current) and cached; the lookup is
+// redone in a new context of the device (after a device reset).
 unsigned char *stats_scratch() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  DevState *d = dev_state();
+  if (!d) return nullptr;
+  if (!d->scratch) {
     void *p = nullptr;
     if (cudaGetSymbolAddress(&p, g_fp_stats_scratch) != cudaSuccess || p == nullptr) return nullptr;
-    g_scratch_ptr[dev] = static_cast<unsigned char *>(p);
+    d->scratch = static_cast<unsigned char *>(p);
   }
-  return g_scratch_ptr[dev];
+  return d->scratch;
 }
 
 size_t round256(size_t x) { return ((x + 255) / 256) * 256; }

@@ -63,6 +63,11 @@ struct ScoreParams {
   float *pm, *plo, *phi;  // [Hq][nch * nsub][b]: per (head, column part, last-block row)
   float *ksum;            // [Hkv][nch * nsub][128]: K column sums per part
   int *err;
+  // int8 test capture (null in normal use): the raw int32 score tile of
+  // query head cap_h, last-block row slice cap_slice and key chunk cap_ch,
+  // copied from tensor memory as the MMAs left it, row-major [128][128]
+  int32_t *cap;
+  int cap_h, cap_slice, cap_ch;
 };
 
 template <bool I8>
@@ -270,6 +275,7 @@ __global__ void __launch_bounds__(736, 1)
         float scale2 = P.scale2;
         if (I8) scale2 *= P.q_scale[hh] * P.k_scale[kvh];
         const uint32_t taddr = tmem + t * 128 + (((warp & 3) * 32) << 16);
+        const bool cap_on = I8 && P.cap != nullptr && hh == P.cap_h && (tile % tiles_per_head) == P.cap_slice;
         bool ok = true;
         float m = -INFINITY;
         float lo4[4] = {0.f, 0.f, 0.f, 0.f}, hi4[4] = {0.f, 0.f, 0.f, 0.f};
@@ -294,6 +300,14 @@ __global__ void __launch_bounds__(736, 1)
               uint32_t r[32];
               tmem_ld32(taddr + hf * 64 + qq * 32, r);
               tmem_ld_wait(r);
+              if constexpr (I8) {
+                if (cap_on && ch == P.cap_ch) {
+                  int4 *dst = reinterpret_cast<int4 *>(P.cap + (size_t)rloc * 128 + hf * 64 + qq * 32);
+#pragma unroll
+                  for (int e = 0; e < 8; ++e)
+                    dst[e] = make_int4((int)r[4 * e], (int)r[4 * e + 1], (int)r[4 * e + 2], (int)r[4 * e + 3]);
+                }
+              }
               const int key0 = ch * 128 + hf * 64 + qq * 32;  // first key of the piece
               const int blk = key0 / P.b;
               if (blk > P.n - 1) continue;                    // past the last block: masked

@@ -20,7 +20,7 @@ FP_PATTERN_VS, FP_PATTERN_QA = 0, 1
 
 SYMBOLS = ("fp_index_create", "fp_index_free", "fp_build_index", "fp_sparse_attn", "fp_index_info",
            "fp_index_nnz", "fp_index_export", "fp_get_device_error", "fp_debug_wait_timeout",
-           "fp_debug_qk_tile_i8", "fp_pattern_stats_noalloc", "fp_strerror",
+           "fp_debug_qk_tile_i8", "fp_debug_capture_i8", "fp_pattern_stats_noalloc", "fp_strerror",
            "fp_prefill_create", "fp_prefill_free", "fp_prefill_enqueue", "fp_prefill_wait", "fp_prefill_run",
            "fp_prefill_group_index", "fp_varlen_create", "fp_varlen_free", "fp_varlen_build_index",
            "fp_varlen_sparse_attn", "fp_varlen_index", "fp_rope_pool", "fp_build_index_pooled")
@@ -49,6 +49,7 @@ def _load():
     L.fp_get_device_error.argtypes = [vp]
     L.fp_debug_wait_timeout.argtypes = [i, vp]
     L.fp_debug_qk_tile_i8.argtypes = [vp, vp, i, i, i, i, i, i, i, vp, vp]
+    L.fp_debug_capture_i8.argtypes = [i, i, i, i, vp]
     L.fp_pattern_stats_noalloc.argtypes = [vp, vp, i, i, i, i, i, f, i, vp, vp, vp, vp, vp, vp, vp, vp]
     L.fp_strerror.argtypes = [i]
     L.fp_strerror.restype = ctypes.c_char_p
@@ -203,6 +204,12 @@ def fp_debug_wait_timeout(timeout_us: int, stream=None):
 def fp_debug_qk_tile_i8(q8, k8, S, Hq, Hkv, d, h, p0, j0, out, stream=None):
     _check(_lib.fp_debug_qk_tile_i8(_ptr(q8), _ptr(k8), S, Hq, Hkv, d, h, p0, j0, _ptr(out), _stream(stream)),
            "fp_debug_qk_tile_i8")
+
+
+def fp_debug_capture_i8(which, h, tile, chunk, out):
+    """Arms (out a device int32 [128][128] tensor) or disarms (out None) the
+    capture of one raw int8 score tile: which 0 = index pass, 1 = attention."""
+    _check(_lib.fp_debug_capture_i8(int(which), int(h), int(tile), int(chunk), _ptr(out)), "fp_debug_capture_i8")
 
 
 def fp_pattern_stats_noalloc(q, k, S, Hq, Hkv, d, b, tau, qk_dtype, q_scale, k_scale, vhat, shat, pest, jsd,

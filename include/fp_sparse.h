@@ -72,8 +72,12 @@ typedef struct fp_index fp_index;
  * Returns FP_ERR_ARG for unsupported shapes, FP_ERR_CUDA if allocation fails. */
 int fp_index_create(int S, int Hq, int Hkv, int d, int b, fp_index **out);
 
-/* Frees an index and its workspace (NULL is ignored).  Synchronises the
- * device before freeing. */
+/* Frees an index and its workspace (NULL is ignored).  The workspace is
+ * released in stream order once the index's most recent fp_build_index or
+ * fp_sparse_attn call has finished on its stream; the call does not wait for
+ * the device or for other streams (work of earlier calls still running on
+ * other streams must be ordered before that last call by the caller, as for
+ * any buffer it frees). */
 void fp_index_free(fp_index *idx);
 
 /* Sparse-index generation (articles above: section 2.1 and 3.1 of the
@@ -137,6 +141,24 @@ int fp_debug_wait_timeout(int timeout_us, void *stream);
  * S a multiple of 128; p0, j0 multiples of 128 inside [0, S). */
 int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int Hkv, int d, int h,
                         int p0, int j0, int32_t *out, void *stream);
+
+/* Test hook for the int8 score tiles of the production kernels (first
+ * article, section 3.3: INT8 multiply, exact INT32 accumulation).  Arms
+ * (out != NULL) or disarms (out = NULL) a capture: while armed, every int8
+ * fp_build_index (which = 0) or int8 fp_sparse_attn (which = 1) on any
+ * device copies one raw 128 x 128 int32 score tile, exactly as the
+ * tensor-core MMAs accumulated it and before any masking or scaling, to the
+ * device buffer out[128][128] (row-major, 16-byte aligned, caller-owned):
+ *   which = 0: the index pass's last-block scores of query head h, 128-row
+ *              slice `tile` of the last block (rows (n-1)b + 128*tile ..),
+ *              key chunk `chunk` (keys 128*chunk .. 128*chunk + 127);
+ *   which = 1: the attention's scores of query head h, query tile `tile`
+ *              (rows 128*tile ..), key chunk `chunk`; written only if that
+ *              tile attends to that chunk (the chunk of a listed block).
+ * Row i, column t of out is then q8[h][row0 + i] . k8[h/g][128*chunk + t].
+ * The setting is process-wide; bf16 calls ignore it.  Returns FP_ERR_ARG for
+ * which outside {0, 1}, a misaligned out or a negative coordinate. */
+int fp_debug_capture_i8(int which, int h, int tile, int chunk, int32_t *out);
 
 /* Per-head pattern statistics with no device allocation at all.  The papers
  * have no counterpart of this call; it exists for callers that must not
@@ -213,7 +235,7 @@ typedef struct fp_varlen fp_varlen;
  * fails. */
 int fp_varlen_create(const int32_t *cu_seqlens, int nseq, int Hq, int Hkv, int d, int b, fp_varlen **out);
 
-/* Frees the set and its indexes (NULL is ignored); synchronises the device. */
+/* Frees the set and its indexes (NULL is ignored), each as fp_index_free does. */
 void fp_varlen_free(fp_varlen *set);
 
 /* fp_build_index for every sequence, queued in order on `stream`.  q, k:

@@ -174,6 +174,82 @@ def test_int8_score_tiles_bit_exact(fp):
         assert np.array_equal(out.cpu().numpy(), ref), (h, p0, j0)
 
 
+def attended_chunks(exp, h, qc, w):
+    """128-key chunks the attention kernel computes for query tile qc of head
+    h: the chunks of the tile's listed blocks up to the tile itself (with
+    b = 64 the tile holds two query blocks and a chunk two key blocks)."""
+    n = nblocks(w.S, w.b)
+    lists = parity.gpu_rows(exp, h, n)
+    if w.b >= 128:
+        per, r = w.b // 128, qc * 128 // w.b
+        return sorted({int(c) * per + k for c in lists[r] for k in range(per) if int(c) * per + k <= qc})
+    return sorted({int(c) // 2 for r in (2 * qc, 2 * qc + 1) if r < n for c in lists[r] if int(c) // 2 <= qc})
+
+
+def check_production_int8_tiles(fp, w, x, P, idx, score_cases, attn_tiles, dev):
+    """Captures raw int32 score tiles from the production int8 kernels (the
+    index pass's last-block scores and the attention's score tiles) on their
+    normal launch paths and compares each bit for bit with the oracle's exact
+    integer products (first article, section 3.3).  Rows past S (a short last
+    block) are not compared."""
+    q8, k8 = x["q8"].to(dev), x["k8"].to(dev)
+    qs, ks, v = x["q_scale"].to(dev), x["k_scale"].to(dev), x["v"].to(dev)
+    cap = torch.empty(128, 128, dtype=torch.int32, device=dev)
+    n = nblocks(w.S, w.b)
+    p_last = (n - 1) * w.b
+    checked = 0
+    try:
+        for h, sl, ch in score_cases:
+            cap.fill_(-(2 ** 31))
+            fp.fp_debug_capture_i8(0, h, sl, ch, cap)
+            fp.fp_build_index(q8, k8, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, fp.FP_QK_INT8, qs, ks, idx)
+            torch.cuda.synchronize()
+            fp.fp_debug_capture_i8(0, 0, 0, 0, None)
+            p0 = p_last + 128 * sl
+            rows, cols = min(128, w.S - p0), min(128, w.S - 128 * ch)
+            ref = P.qk_int_tile(h, p0, 128 * ch, rows, cols)
+            assert np.array_equal(cap[:rows, :cols].cpu().numpy(), ref), ("score", h, sl, ch)
+            checked += 1
+        fp.fp_build_index(q8, k8, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, fp.FP_QK_INT8, qs, ks, idx)
+        exp = fp.fp_index_export(idx)
+        out = torch.empty(w.Hq, w.S, w.d, dtype=torch.bfloat16, device=dev)
+        for h, qc in attn_tiles:
+            chunks = attended_chunks(exp, h, qc, w)
+            for kc in sorted({chunks[0], chunks[len(chunks) // 2], chunks[-1]}):
+                cap.fill_(-(2 ** 31))
+                fp.fp_debug_capture_i8(1, h, qc, kc, cap)
+                fp.fp_sparse_attn(q8, k8, v, qs, ks, idx, out)
+                torch.cuda.synchronize()
+                fp.fp_debug_capture_i8(1, 0, 0, 0, None)
+                rows, cols = min(128, w.S - 128 * qc), min(128, w.S - 128 * kc)
+                ref = P.qk_int_tile(h, 128 * qc, 128 * kc, rows, cols)
+                assert np.array_equal(cap[:rows, :cols].cpu().numpy(), ref), ("attn", h, qc, kc)
+                checked += 1
+    finally:
+        fp.fp_debug_capture_i8(0, 0, 0, 0, None)
+        fp.fp_debug_capture_i8(1, 0, 0, 0, None)
+    assert fp.fp_get_device_error() == fp.FP_OK
+    print(f"[{w.name}] {checked} production int8 score tiles bit-exact")
+
+
+INT8_CAPTURE = [synth.Workload("i8cap_b128", S=4096, Hq=8, Hkv=2, b=128, int8=True, seed=41),
+                synth.Workload("i8cap_b256", S=4096, Hq=4, Hkv=1, b=256, int8=True, seed=42),
+                synth.Workload("i8cap_b64_ragged", S=2000, Hq=4, Hkv=2, b=64, int8=True, seed=43)]
+
+
+@pytest.mark.parametrize("w", INT8_CAPTURE, ids=[w.name for w in INT8_CAPTURE])
+def test_int8_production_score_tiles_bit_exact(fp, w):
+    x = synth.make_inputs(w)
+    P = oracle_problem(x, w)
+    idx = fp.fp_index_create(w.S, w.Hq, w.Hkv, w.d, w.b)
+    n, nch = nblocks(w.S, w.b), nblocks(w.S, 128)
+    slices = nblocks(w.S - (n - 1) * w.b, 128)
+    score_cases = [(0, 0, 0), (w.Hq - 1, slices - 1, nch - 1), (w.Hq // 2, slices - 1, nch // 2), (1, 0, 1)]
+    attn_tiles = [(1, nch - 1), (w.Hq - 1, nch // 2), (0, 3)]
+    check_production_int8_tiles(fp, w, x, P, idx, score_cases, attn_tiles, torch.device("cuda:0"))
+    idx.free()
+
+
 def test_bounded_wait_reports_timeout_and_context_survives(fp):
     fp.fp_debug_wait_timeout(200000)
     assert fp.fp_get_device_error() == fp.FP_ERR_TIMEOUT
@@ -202,12 +278,9 @@ def test_full_size_layers(fp, name, ntiles):
     check_index(P, exp, w)
     check_tiles(P, exp, out, w, sampled_tiles(w, ntiles, seed=w.seed))
     if w.int8:
-        q8, k8 = x["q8"].cuda(), x["k8"].cuda()
-        t = torch.empty(128, 128, dtype=torch.int32, device="cuda")
-        for h, p0, j0 in [(0, w.S - 128, 0), (31, w.S - 128, w.S - 128), (17, 65536, 4096)]:
-            fp.fp_debug_qk_tile_i8(q8, k8, w.S, w.Hq, w.Hkv, w.d, h, p0, j0, t)
-            torch.cuda.synchronize()
-            assert np.array_equal(t.cpu().numpy(), P.qk_int_tile(h, p0, j0, 128, 128))
+        nch = nblocks(w.S, 128)
+        check_production_int8_tiles(fp, w, x, P, idx, [(0, 0, 0), (31, 0, nch - 1), (17, 0, 512)],
+                                    [(31, nch - 1), (17, 512), (2, 40)], torch.device("cuda:0"))
 
 
 LARGE_N = [synth.Workload("b64_n1024", S=65536, Hq=8, Hkv=2, b=64, n_vertical=64, n_topics=32, seed=31),
@@ -243,3 +316,47 @@ def test_batched_sequences_equal_separate_calls(fp):
             rows_b = parity.gpu_rows(exp_b, 4 * i + h, n)
             rows_s = parity.gpu_rows(exp, h, n)
             assert all(np.array_equal(a, c) for a, c in zip(rows_b, rows_s))
+
+
+# The S x b x gamma sweep on the 128K generator (Hq=32, Hkv=8): the points the
+# other tests do not already cover at this head count.
+SWEEP_BY_NAME = {w.name: w for w in synth.sweep_workloads()}
+SWEEP_GAMMA1 = ["sweep_S16384_b128_g1.0", "sweep_S65536_b128_g1.0", "sweep_S131072_b128_g1.0",
+                "sweep_S131072_b256_g1.0"]
+SWEEP_B256 = ["sweep_S16384_b256_g0.8", "sweep_S16384_b256_g0.95", "sweep_S131072_b256_g0.8",
+              "sweep_S131072_b256_g0.95"]
+
+
+@pytest.mark.parametrize("name", SWEEP_GAMMA1)
+def test_sweep_gamma_one_is_dense_causal(fp, name):
+    """gamma = 1 keeps every causal block, so the layer is dense causal
+    attention: the index holds Hq n(n+1)/2 blocks, and 64 seeded query tiles
+    (the longest rows of several heads among them) equal the oracle's dense
+    causal attention."""
+    w = SWEEP_BY_NAME[name]
+    x = synth.make_inputs(w)
+    exp, out, idx = run_gpu(fp, x, w)
+    n = nblocks(w.S, w.b)
+    assert exp["nnz"] == w.Hq * n * (n + 1) // 2
+    for h in range(w.Hq):
+        rows = parity.gpu_rows(exp, h, n)
+        assert all(len(r) == i + 1 for i, r in enumerate(rows)), h
+    P = oracle_problem(x, w)
+    check_index(P, exp, w)
+    check_tiles(P, exp, out, w, sampled_tiles(w, 64, seed=w.seed + w.S))
+
+
+@pytest.mark.parametrize("name", SWEEP_B256)
+def test_sweep_b256_gammas(fp, name):
+    """b = 256 at gamma 0.8 and 0.95 on the 128K generator: the full index
+    against the oracle, and query tiles against the oracle on the GPU's index
+    (every tile at S = 16K, 64 seeded tiles at S = 128K)."""
+    w = SWEEP_BY_NAME[name]
+    x = synth.make_inputs(w)
+    exp, out, idx = run_gpu(fp, x, w)
+    P = oracle_problem(x, w)
+    check_index(P, exp, w)
+    nq = nblocks(w.S, 128)
+    tiles = [(h, qc) for h in range(w.Hq) for qc in range(nq)] if w.S <= 16384 else \
+        sampled_tiles(w, 64, seed=w.seed + w.S)
+    check_tiles(P, exp, out, w, tiles)

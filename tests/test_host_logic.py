@@ -81,11 +81,30 @@ def test_traffic_record_is_dropped_when_the_kernel_source_changes(tmp_path, monk
 
 def test_attention_peak_for_mixed_int8():
     import bench
-    assert bench.attention_peak(1400.0, False) == 1400.0
-    # W8A8: half the FLOPs at 2P and half at P take 0.75 F / P
-    F, P = 1.0e15, 1400.0e12
-    t = (F / 2) / (2 * P) + (F / 2) / P
-    assert abs(bench.attention_peak(1400.0, True) * 1e12 - F / t) < 1e-3 * P
+    assert bench.attention_peak(1400.0) == 1400.0
+    # W8A8: half the FLOPs at the int8 peak and half at the bf16 peak
+    F, P, P8 = 1.0e15, 1400.0e12, 2600.0e12
+    t = (F / 2) / P8 + (F / 2) / P
+    assert abs(bench.attention_peak(1400.0, 2600.0) * 1e12 - F / t) < 1e-6 * P
+    # int8 at exactly 2x bf16: 0.75 F / P, an effective peak of 4/3 P
+    assert abs(bench.attention_peak(1400.0, 2800.0) - 1400.0 * 4.0 / 3.0) < 1e-9
+
+
+def test_oracle_sample_extrapolates_items_to_the_layer():
+    """The CPU baseline's sample: per-item thread CPU times scaled to every
+    head and tile of the layer, divided over the threads used."""
+    import bench
+    from dynamic_block_sparse_last_b200 import synth
+    from oracle import oracle as orc
+    w = synth.Workload("t", S=512, Hq=4, Hkv=2, b=128, seed=0)
+    x = synth.make_inputs(w)
+    P = orc.OracleProblem(x["q"], x["k"], x["v"], w.b)
+    res = bench.oracle_sample(w, P, 3, heads=2, tiles=6, threads=3)
+    assert res["threads"] == 3 and res["layer_s"] > 0
+    assert abs(res["layer_s"] * 3 - res["layer_cpu_s"]) < 1e-9
+    lo, med, hi = res["spread_min_median_max"]["tile_s"]
+    assert 0 <= lo <= med <= hi
+    assert "extrapolated" in res["desc"]
 
 
 def test_index_pass_floors():
