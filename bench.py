@@ -35,8 +35,8 @@ from dynamic_block_sparse_last_b200 import synth  # noqa: E402
 
 METRIC = "sparse-prefill ms/layer & dense-equiv TFLOPS at S=128K; % of HBM/TC roofline"
 UNIT = "dense-equiv TFLOP/s"
-# k_score_last, k_row_stats, k_block_mass, k_kbar, k_pattern, k_qbar, k_qa_logits, k_cut, k_sparse_attn
-KERNELS_PER_STEP = 9
+# k_score_last, k_head_stats, k_qbar, k_qa_logits, k_cut, k_sparse_attn
+KERNELS_PER_STEP = 6
 ATTN_SRC = os.path.join(ROOT, "dynamic_block_sparse_last_b200", "csrc", "attn_kernel.cuh")
 
 

@@ -206,8 +206,9 @@ struct UnionWalk {
   }
 };
 
+// One CTA per SM (608 threads): 104 registers per thread fit (608 x 104 <= 65536).
 template <bool I8>
-__global__ void __launch_bounds__(608, 1)
+__global__ void __maxnreg__(104)
     k_sparse_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, AttnParams P) {
   using C = AttnCfg<I8>;
@@ -426,7 +427,7 @@ __global__ void __launch_bounds__(608, 1)
       }
       float s[64];
 #pragma unroll
-      for (int e = 0; e < 64; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
+      for (int e = 0; e < 64; ++e) s[e] = I8 ? i32_to_f32_small(rr[e]) : __uint_as_float(rr[e]);
       if (P.b < 128) {
         // the warp's quadrant is one (query block, key block 2kc + ch) pair
         const int kb = 2 * kc + ch;

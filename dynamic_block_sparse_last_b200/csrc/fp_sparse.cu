@@ -30,15 +30,12 @@ struct fp_index {
   int device;
   int built;
   int qk_dtype;
-  int R2, chunks_per_part;
   void *slab;
   size_t slab_bytes;
   bool slab_pooled;        // slab from the stream-ordered allocator (else cudaMalloc)
   cudaStream_t own;        // the index's own stream: allocation and release of the slab
   cudaEvent_t last_use;    // recorded on the caller's stream at the end of every build / attention call
   float *pm, *plo, *phi;   // [Hq][npart][b]
-  float *partM, *partL;    // [Hq][R2][b]
-  float *LOc, *HIc;        // [Hq][npart]
   float *ksum;             // [Hkv][npart][128]
   float *kbar;             // [Hkv][n][128]
   float *qbar;             // [Hq][n][128]
@@ -206,19 +203,19 @@ int set_smem_attrs() {
 // Shape, inputs and scratch of the pattern-statistics launches (steps 1-3 of
 // fp_build_index), shared by the index build and the allocation-free call.
 struct StatsJob {
-  int S, Hq, Hkv, d, b, n, nch, g, R2, chunks_per_part;  // R2, chunks_per_part over the npart parts
+  int S, Hq, Hkv, d, b, n, nch, g;
   int npart;  // column parts: nch, or 2 nch when b = 64
   int ld;  // rows from one head to the next
   const void *q, *k;
   const float *q_scale, *k_scale;  // int8 only
   float tau;
-  float *pm, *plo, *phi, *partM, *partL, *LOc, *HIc, *ksum, *kbar;
+  float *pm, *plo, *phi, *ksum, *kbar;
   float *vhat, *shat, *pest, *jsd;
   int *pattern;
   const float *ext_kbar;  // K block means given by the caller (then ksum/kbar are not computed), or null
 };
 
-// k_score_last, k_row_stats, k_block_mass, k_kbar and k_pattern on `st`.
+// k_score_last and k_head_stats on `st`.
 template <bool I8>
 int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   int rc;
@@ -256,30 +253,17 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
   }
   k_score_last<I8><<<dim3(R, tgroups, J.Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
   if ((rc = launch_status())) return rc;
-  k_row_stats<<<dim3(J.Hq, J.R2), J.b, 0, st>>>(J.pm, J.plo, J.phi, J.npart, J.b, nlast, J.chunks_per_part,
-                                                J.partM, J.partL);
-  if ((rc = launch_status())) return rc;
-  const size_t red_bytes = (size_t)(J.b / 32) * J.chunks_per_part * 2 * sizeof(float);
-  k_block_mass<<<dim3(J.Hq, J.R2), J.b, red_bytes, st>>>(J.pm, J.plo, J.phi, J.partM, J.partL, J.npart, J.b,
-                                                         nlast, J.chunks_per_part, J.LOc, J.HIc);
-  if ((rc = launch_status())) return rc;
-  const float *kbar = J.ext_kbar;
-  if (!kbar) {
-    k_kbar<<<dim3(J.n, J.Hkv), 128, 0, st>>>(J.ksum, I8 ? J.k_scale : nullptr, J.S, J.npart, J.b, J.n, J.kbar);
-    if ((rc = launch_status())) return rc;
-    kbar = J.kbar;
-  }
-  k_pattern<I8><<<J.Hq, 1024, 0, st>>>(J.q, J.q_scale, J.LOc, J.HIc, kbar, J.S, J.ld, J.g, J.b, J.n, J.npart,
-                                       1.0f / sqrtf((float)J.d), J.tau, J.vhat, J.shat, J.pest, J.jsd,
-                                       J.pattern);
+  HeadStatsParams hp;
+  hp.S = J.S; hp.b = J.b; hp.n = J.n; hp.npart = J.npart; hp.g = J.g; hp.ld = J.ld; hp.nlast = nlast;
+  hp.pm = J.pm; hp.plo = J.plo; hp.phi = J.phi;
+  hp.ksum = J.ksum; hp.ext_kbar = J.ext_kbar; hp.k_scale = J.k_scale;
+  hp.q = J.q; hp.q_scale = J.q_scale;
+  hp.inv_sqrt_d = 1.0f / sqrtf((float)J.d);
+  hp.tau = J.tau;
+  hp.vhat = J.vhat; hp.shat = J.shat; hp.pest = J.pest; hp.jsd = J.jsd; hp.pattern = J.pattern;
+  hp.kbar = J.kbar;
+  k_head_stats<I8><<<dim3(kStatCta, J.Hq), kStatThreads, 0, st>>>(hp);
   return launch_status();
-}
-
-// Row-part split of the per-row reductions: at most 16 parts over the chunks.
-void row_parts(int nch, int &R2, int &chunks_per_part) {
-  R2 = nch < 16 ? nch : 16;
-  chunks_per_part = (nch + R2 - 1) / R2;
-  R2 = (nch + chunks_per_part - 1) / chunks_per_part;
 }
 
 // ext_qbar / ext_kbar: block means of Q [Hq][n][128] and K [Hkv][n][128]
@@ -296,10 +280,10 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   StatsJob J;
   J.S = I->S; J.Hq = I->Hq; J.Hkv = I->Hkv; J.d = I->d; J.b = I->b; J.n = I->n; J.nch = I->nch; J.g = I->g;
   J.npart = I->npart;
-  J.R2 = I->R2; J.chunks_per_part = I->chunks_per_part; J.ld = I->ld;
+  J.ld = I->ld;
   J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
-  J.pm = I->pm; J.plo = I->plo; J.phi = I->phi; J.partM = I->partM; J.partL = I->partL;
-  J.LOc = I->LOc; J.HIc = I->HIc; J.ksum = I->ksum; J.kbar = I->kbar;
+  J.pm = I->pm; J.plo = I->plo; J.phi = I->phi;
+  J.ksum = I->ksum; J.kbar = I->kbar;
   J.vhat = I->vhat; J.shat = I->shat; J.pest = I->pest; J.jsd = I->jsd; J.pattern = I->pattern;
   J.ext_kbar = ext_kbar;
   if ((rc = launch_pattern_stats<I8>(J, err, st))) return rc;
@@ -363,15 +347,12 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   I->S = S; I->Hq = Hq; I->Hkv = Hkv; I->d = d; I->b = b; I->ld = ld;
   I->n = (S + b - 1) / b; I->nch = (S + 127) / 128; I->g = Hq / Hkv;
   I->npart = b < 128 ? I->nch * (128 / b) : I->nch;
-  row_parts(I->npart, I->R2, I->chunks_per_part);
   cudaGetDevice(&I->device);
   const size_t n = I->n, nch = I->npart, bb = b;  // statistics arrays are per column part
   const size_t tri = n * (n + 1) / 2;
   size_t need = 0;
   auto add = [&](size_t bytes) { need += ((bytes + 255) / 256) * 256; };
   for (int i = 0; i < 3; ++i) add((size_t)Hq * nch * bb * 4);
-  for (int i = 0; i < 2; ++i) add((size_t)Hq * I->R2 * bb * 4);
-  for (int i = 0; i < 2; ++i) add((size_t)Hq * nch * 4);
   add((size_t)Hkv * nch * 128 * 4);
   add((size_t)Hkv * n * 128 * 4);
   add((size_t)Hq * n * 128 * 4);
@@ -409,10 +390,6 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   I->pm = carve<float>(cur, (size_t)Hq * nch * bb);
   I->plo = carve<float>(cur, (size_t)Hq * nch * bb);
   I->phi = carve<float>(cur, (size_t)Hq * nch * bb);
-  I->partM = carve<float>(cur, (size_t)Hq * I->R2 * bb);
-  I->partL = carve<float>(cur, (size_t)Hq * I->R2 * bb);
-  I->LOc = carve<float>(cur, (size_t)Hq * nch);
-  I->HIc = carve<float>(cur, (size_t)Hq * nch);
   I->ksum = carve<float>(cur, (size_t)Hkv * nch * 128);
   I->kbar = carve<float>(cur, (size_t)Hkv * n * 128);
   I->qbar = carve<float>(cur, (size_t)Hq * n * 128);
@@ -641,12 +618,9 @@ int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int
                        const float *q_scale, const float *k_scale, float *vhat, float *shat, float *pest,
                        float *jsd, int32_t *pattern, cudaStream_t st) {
   const int n = (S + b - 1) / b, nch = (S + 127) / 128, npart = b < 128 ? nch * (128 / b) : nch;
-  int R2, cpp;
-  row_parts(npart, R2, cpp);
-  const size_t e_part = (size_t)Hq * npart * b, e_rs = (size_t)Hq * R2 * b, e_blk = (size_t)Hq * npart;
+  const size_t e_part = (size_t)Hq * npart * b;
   const size_t e_ksum = (size_t)Hkv * npart * 128, e_kbar = (size_t)Hkv * n * 128;
-  const size_t need = 3 * round256(e_part * 4) + 2 * round256(e_rs * 4) + 2 * round256(e_blk * 4) +
-                      round256(e_ksum * 4) + round256(e_kbar * 4);
+  const size_t need = 3 * round256(e_part * 4) + round256(e_ksum * 4) + round256(e_kbar * 4);
   if (need > kNoAllocScratchBytes) return FP_ERR_ARG;
   unsigned char *base = stats_scratch();
   if (!base) return FP_ERR_CUDA;
@@ -656,17 +630,15 @@ int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int
   if (!err) return FP_ERR_CUDA;
   char *cur = reinterpret_cast<char *>(base);
   float *pm = carve<float>(cur, e_part), *plo = carve<float>(cur, e_part), *phi = carve<float>(cur, e_part);
-  float *partM = carve<float>(cur, e_rs), *partL = carve<float>(cur, e_rs);
-  float *LOc = carve<float>(cur, e_blk), *HIc = carve<float>(cur, e_blk);
   float *ksum = carve<float>(cur, e_ksum), *kbar = carve<float>(cur, e_kbar);
 
   StatsJob J;
   J.S = S; J.Hq = Hq; J.Hkv = Hkv; J.d = d; J.b = b; J.n = n; J.nch = nch; J.g = Hq / Hkv;
   J.npart = npart;
-  J.R2 = R2; J.chunks_per_part = cpp; J.ld = S; J.ext_kbar = nullptr;
+  J.ld = S; J.ext_kbar = nullptr;
   J.q = q; J.k = k; J.q_scale = q_scale; J.k_scale = k_scale; J.tau = tau;
-  J.pm = pm; J.plo = plo; J.phi = phi; J.partM = partM; J.partL = partL;
-  J.LOc = LOc; J.HIc = HIc; J.ksum = ksum; J.kbar = kbar;
+  J.pm = pm; J.plo = plo; J.phi = phi;
+  J.ksum = ksum; J.kbar = kbar;
   J.vhat = vhat; J.shat = shat; J.pest = pest; J.jsd = jsd; J.pattern = pattern;
   return launch_pattern_stats<I8>(J, err, st);
 }

@@ -13,14 +13,15 @@
 //                  KV group through a TMA ring; per (row, chunk) max and the
 //                  two offset-half sums; per-chunk K column sums.  Nothing of
 //                  size S x b reaches global memory.
-//   k_row_stats    per (head, row, chunk range): running max / sum.
-//   k_block_mass   per (head, chunk): row-normalised lo/hi masses.
-//   k_kbar         block means of K.
-//   k_pattern      per head: vhat, shat, P_est, JSD, pattern.
+//   k_head_stats   one cluster per head: row max / sum, row-normalised
+//                  block masses, vhat, shat, block means of K, P_est, JSD,
+//                  pattern.
 //   k_qbar         block means of Q for query-aware heads only.
 //   k_qa_logits    q-bar . k-bar logits of query-aware heads (tiled fp32).
 //   k_cut          per (head, query block): scores, gamma cut, sorted list.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "ptx.cuh"
 
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(736, 1)
               float pm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
               for (int e = 0; e < 32; ++e) {
-                const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+                const float s = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
                 const bool valid = !last_block || (e <= dlt);
                 pm4[e & 3] = valid ? fmaxf(pm4[e & 3], s) : pm4[e & 3];
               }
@@ -336,21 +337,21 @@ __global__ void __launch_bounds__(736, 1)
               if (dlt >= 31) {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                  const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+                  const float s = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
                   lo4[e & 3] += ex2(fmaf(s, scale2, -m2p));
                 }
               } else if (dlt < 0) {
                 if (!last_block) {
 #pragma unroll
                   for (int e = 0; e < 32; ++e) {
-                    const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+                    const float s = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
                     hi4[e & 3] += ex2(fmaf(s, scale2, -m2p));
                   }
                 }
               } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
-                  const float s = I8 ? (float)(int)r[e] : __uint_as_float(r[e]);
+                  const float s = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
                   const float p = ex2(fmaf(s, scale2, -m2p));
                   if (e <= dlt) lo4[e & 3] += p;
                   else if (!last_block) hi4[e & 3] += p;
@@ -385,224 +386,285 @@ __global__ void __launch_bounds__(736, 1)
 }
 
 // ---------------------------------------------------------------------------
-// k_row_stats: grid (Hq, R2), block b threads.  Row i's running max M and
-// sum L = sum_chunks (lo + hi) 2^(m - M) over the CTA's chunk range; rows at
-// or past nlast (absent from a partial last block) get M = -inf, L = 0.
+// k_head_stats: statistics finalise and pattern choice, one cluster of
+// kStatCta CTAs per query head h (grid (kStatCta, Hq), 256 threads).  Rank
+// k of the cluster owns the key blocks [k n / C, (k+1) n / C) and their
+// column parts.  With nlast = S - (n-1)b rows in the last block and the
+// score kernel's per-(row, part) partials (m in log2 units, lo, hi):
+//   1. row statistics over the owned parts, combined over the cluster
+//      through distributed shared memory (in rank order):
+//        M_i = max_p m_ip,  L_i = sum_p (lo_ip + hi_ip) 2^(m_ip - M_i);
+//      and a rank's slice of the last block's query rows summed per column
+//      (qbar_last = mean of the nlast rows);
+//   2. per owned part: LO_p = sum_i lo_ip 2^(m_ip - M_i) / L_i, HI_p alike;
+//      per owned block: vhat[c] = (LO[c] + HI[c]) / nlast, the block mean
+//      kbar_c of K, and the logit z_c = qbar_last . kbar_c / sqrt(d);
+//   3. shat[o] = (LO[n-1-o] + HI[n-2-o]) / nlast (the mirrored blocks are
+//      read from their owners), P_est = softmax_c(z_c) with the cluster's
+//      max and sum, and JSD(vhat, P_est) (natural log) summed over ranks;
+//      pattern = QA iff JSD < tau.
+// Every reduction runs in a fixed order.  kbar is written for the KV head by
+// the cluster of its first query head (h % g == 0); when the caller supplies
+// the K block means (ext_kbar) they are read instead of the column sums.
 // ---------------------------------------------------------------------------
-__global__ void k_row_stats(const float *__restrict__ pm, const float *__restrict__ plo,
-                            const float *__restrict__ phi, int nch, int b, int nlast, int chunks_per_part,
-                            float *__restrict__ partM, float *__restrict__ partL) {
-  const int h = blockIdx.x, part = blockIdx.y, R2 = gridDim.y, i = threadIdx.x;
-  const int c0 = part * chunks_per_part, c1 = i < nlast ? min(nch, c0 + chunks_per_part) : c0;
-  float M = -INFINITY, L = 0.f;
-  for (int ch = c0; ch < c1; ch += 4) {
-    // four chunks' loads in flight, then the running combine in order
-    float mv[4], sv[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const size_t o = ((size_t)h * nch + ch + u) * b + i;
-      const bool in = ch + u < c1;
-      mv[u] = in ? pm[o] : -INFINITY;
-      sv[u] = in ? plo[o] + phi[o] : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float m = mv[u];
-      if (m == -INFINITY) continue;
-      if (m > M) {
-        L = L * ex2(M - m) + sv[u];
-        M = m;
-      } else {
-        L += sv[u] * ex2(m - M);
-      }
-    }
-  }
-  partM[((size_t)h * R2 + part) * b + i] = M;
-  partL[((size_t)h * R2 + part) * b + i] = L;
-}
+constexpr int kStatCta = 8;
+constexpr int kStatThreads = 256;
+constexpr int kStatMaxOwnParts = 256;   // npart <= 2048
+constexpr int kStatMaxOwnBlocks = 128;  // n <= 1024
 
-// ---------------------------------------------------------------------------
-// k_block_mass: grid (Hq, R2), block b threads.  Combines the R2 partial row
-// statistics, then for every chunk of the CTA's range sums over rows
-//   LOc[ch] = sum_i lo_i 2^(m_i - M_i) / L_i,  HIc[ch] likewise,
-// in a fixed order (per-warp shuffle tree, then warps in index order).
-// ---------------------------------------------------------------------------
-__global__ void k_block_mass(const float *__restrict__ pm, const float *__restrict__ plo,
-                             const float *__restrict__ phi, const float *__restrict__ partM,
-                             const float *__restrict__ partL, int nch, int b, int nlast,
-                             int chunks_per_part, float *__restrict__ LOc, float *__restrict__ HIc) {
-  extern __shared__ float red[];  // [nwarps][chunks_per_part][2]
-  const int h = blockIdx.x, part = blockIdx.y, R2 = gridDim.y, i = threadIdx.x;
-  const int warp = i >> 5, lane = i & 31, nw = blockDim.x >> 5;
-  float M = -INFINITY;
-  for (int r = 0; r < R2; ++r) M = fmaxf(M, partM[((size_t)h * R2 + r) * b + i]);
-  float L = 0.f;
-  for (int r = 0; r < R2; ++r) {
-    const float m = partM[((size_t)h * R2 + r) * b + i];
-    if (m != -INFINITY) L += partL[((size_t)h * R2 + r) * b + i] * ex2(m - M);
-  }
-  const float invL = 1.f / L;
-  const int c0 = part * chunks_per_part, c1 = min(nch, c0 + chunks_per_part);
-  for (int ch = c0; ch < c1; ch += 4) {
-    float a[4], c[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const size_t o = ((size_t)h * nch + ch + u) * b + i;
-      const bool in = i < nlast && ch + u < c1;  // rows past nlast hold no partials
-      const float m = in ? pm[o] : -INFINITY;
-      const float w = (m == -INFINITY) ? 0.f : ex2(m - M) * invL;
-      a[u] = in ? plo[o] * w : 0.f;
-      c[u] = in ? phi[o] * w : 0.f;
-    }
-#pragma unroll
-    for (int s = 16; s > 0; s >>= 1) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        a[u] += __shfl_xor_sync(0xffffffffu, a[u], s);
-        c[u] += __shfl_xor_sync(0xffffffffu, c[u], s);
-      }
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (ch + u < c1) {
-          red[(warp * chunks_per_part + (ch + u - c0)) * 2 + 0] = a[u];
-          red[(warp * chunks_per_part + (ch + u - c0)) * 2 + 1] = c[u];
+struct HeadStatsParams {
+  int S, b, n, npart, g, ld, nlast;
+  const float *pm, *plo, *phi;   // [Hq][npart][b]
+  const float *ksum;             // [Hkv][npart][128] K column sums per part
+  const float *ext_kbar;         // [Hkv][n][128] block means given by the caller, or null
+  const float *k_scale;          // int8 only
+  const void *q;                 // last block rows for qbar_last
+  const float *q_scale;          // int8 only
+  float inv_sqrt_d, tau;
+  float *vhat, *shat, *pest, *jsd;
+  int *pattern;
+  float *kbar;                   // [Hkv][n][128] out (when computed here)
+};
+
+__device__ __forceinline__ int stat_block0(int k, int n) { return (k * n) / kStatCta; }
+
+template <bool I8>
+__global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads)
+    k_head_stats(HeadStatsParams P) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cl = cg::this_cluster();
+  __shared__ float grpM[kStatThreads], grpL[kStatThreads];   // per thread group, phase 1
+  __shared__ float rowM[256], rowL[256];                     // this rank's row partials (shared)
+  __shared__ float gM[256], gInvL[256];                      // cluster row statistics
+  __shared__ float qpart[128], qb[128];                      // last-block query column sums / mean
+  __shared__ float LOp[kStatMaxOwnParts], HIp[kStatMaxOwnParts];
+  __shared__ float LOb[kStatMaxOwnBlocks], HIb[kStatMaxOwnBlocks];  // owned blocks (shared)
+  __shared__ float vh[kStatMaxOwnBlocks], zc[kStatMaxOwnBlocks];
+  __shared__ float red[kStatThreads / 32];
+  __shared__ float xch[4];                                    // [0] local max, [1] local sum, [2] local JSD
+
+  const int k = (int)cl.block_rank(), h = blockIdx.y, tid = threadIdx.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarp = kStatThreads / 32;
+  const int b = P.b, n = P.n, npart = P.npart, nlast = P.nlast;
+  const int kvh = h / P.g;
+  const int per = b >= 128 ? b / 128 : 1;  // parts per block
+  const int c0 = stat_block0(k, n), c1 = stat_block0(k + 1, n);
+  const int p0 = min(npart, c0 * per), p1 = min(npart, c1 * per);
+  const size_t hoff = (size_t)h * npart * b;
+
+  // ---- 1. row statistics over the owned parts; query column sums of a row slice
+  {
+    const int G = kStatThreads / b, i = tid % b, j = tid / b;
+    float M = -INFINITY, L = 0.f;
+    if (i < nlast) {
+      for (int p = p0 + j; p < p1; p += G) {
+        const size_t o = hoff + (size_t)p * b + i;
+        const float m = P.pm[o];
+        if (m == -INFINITY) continue;
+        const float sv = P.plo[o] + P.phi[o];
+        if (m > M) {
+          L = L * ex2(M - m) + sv;
+          M = m;
+        } else {
+          L += sv * ex2(m - M);
         }
       }
     }
-  }
-  __syncthreads();
-  for (int ch = c0 + i; ch < c1; ch += blockDim.x) {
-    float a = 0.f, c = 0.f;
-    for (int w = 0; w < nw; ++w) {
-      a += red[(w * chunks_per_part + (ch - c0)) * 2 + 0];
-      c += red[(w * chunks_per_part + (ch - c0)) * 2 + 1];
-    }
-    LOc[(size_t)h * nch + ch] = a;
-    HIc[(size_t)h * nch + ch] = c;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// k_kbar: grid (n, Hkv), block 128: kbar[kvh][c][t] = mean of the K rows of
-// block c (b rows, or S - (n-1)b for a partial last block); for int8 keys the
-// exact integer sum times k_scale[kvh].
-// ---------------------------------------------------------------------------
-__global__ void k_kbar(const float *__restrict__ ksum, const float *__restrict__ k_scale, int S, int nch,
-                       int b, int n, float *__restrict__ kbar) {
-  const int c = blockIdx.x, kvh = blockIdx.y, t = threadIdx.x;
-  const int per = b >= 128 ? b / 128 : 1, rows = min(b, S - c * b);  // column parts per block
-  float s = 0.f;
-  for (int k = 0; k < per && c * per + k < nch; ++k) s += ksum[((size_t)kvh * nch + c * per + k) * 128 + t];
-  if (k_scale) s *= k_scale[kvh];
-  kbar[((size_t)kvh * n + c) * 128 + t] = s / (float)rows;
-}
-
-// ---------------------------------------------------------------------------
-// k_pattern: grid (Hq), block 1024.  With nlast = S - (n-1)b rows in the
-// last block: vhat[c] = (LO[c] + HI[c]) / nlast, shat[o] = (LO[n-1-o] +
-// HI[n-2-o]) / nlast, P_est = softmax_c(qbar_last . kbar_c / sqrt(d)) with
-// qbar_last the mean of those nlast rows, JSD(vhat, P_est) (natural log),
-// pattern = QA iff JSD < tau.
-// ---------------------------------------------------------------------------
-template <bool I8>
-__global__ void __launch_bounds__(1024)
-    k_pattern(const void *__restrict__ q, const float *__restrict__ q_scale,
-              const float *__restrict__ LOc, const float *__restrict__ HIc,
-              const float *__restrict__ kbar, int S, int ld, int g, int b, int n, int nch, float inv_sqrt_d,
-              float tau, float *__restrict__ vhat, float *__restrict__ shat,
-              float *__restrict__ pest, float *__restrict__ jsd, int *__restrict__ pattern) {
-  __shared__ float qb[128];
-  __shared__ float part[1024 / 32];
-  __shared__ float lo_s[1024], hi_s[1024];
-  const int h = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int kvh = h / g, per = b >= 128 ? b / 128 : 1, nlast = S - (n - 1) * b;  // parts per block
-  // block masses
-  for (int c = tid; c < n; c += blockDim.x) {
-    float a = 0.f, e = 0.f;
-    for (int k = 0; k < per && c * per + k < nch; ++k) {
-      a += LOc[(size_t)h * nch + c * per + k];
-      e += HIc[(size_t)h * nch + c * per + k];
-    }
-    lo_s[c] = a / (float)nlast;
-    hi_s[c] = e / (float)nlast;
-  }
-  // mean of the last block's query rows
-  if (tid < 128) {
-    const size_t base = ((size_t)h * ld + (size_t)(n - 1) * b) * 128 + tid;
-    if (I8) {
-      const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
-      int acc = 0;
-      for (int r = 0; r < nlast; ++r) acc += q8[base + (size_t)r * 128];
-      qb[tid] = (float)acc * q_scale[h] / (float)nlast;
-    } else {
-      const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(q);
+    grpM[tid] = M;
+    grpL[tid] = L;
+    if (tid < 128) {
+      const int r0 = (k * nlast) / kStatCta, r1 = ((k + 1) * nlast) / kStatCta;
+      const size_t base = ((size_t)h * P.ld + (size_t)(n - 1) * b) * 128 + tid;
       float acc = 0.f;
-      for (int r = 0; r < nlast; ++r) acc += __bfloat162float(qh[base + (size_t)r * 128]);
-      qb[tid] = acc / (float)nlast;
+      if (I8) {
+        const int8_t *q8 = reinterpret_cast<const int8_t *>(P.q);
+        int ia = 0;
+        for (int r = r0; r < r1; ++r) ia += q8[base + (size_t)r * 128];
+        acc = (float)ia;
+      } else {
+        const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(P.q);
+        for (int r = r0; r < r1; ++r) acc += __bfloat162float(qh[base + (size_t)r * 128]);
+      }
+      qpart[tid] = acc;
+    }
+    __syncthreads();
+    if (tid < b) {
+      float Mi = -INFINITY, Li = 0.f;
+      for (int jj = 0; jj < G; ++jj) {
+        const float m = grpM[jj * b + tid];
+        if (m == -INFINITY) continue;
+        const float l = grpL[jj * b + tid];
+        if (m > Mi) {
+          Li = Li * ex2(Mi - m) + l;
+          Mi = m;
+        } else {
+          Li += l * ex2(m - Mi);
+        }
+      }
+      rowM[tid] = Mi;
+      rowL[tid] = Li;
+    }
+  }
+  cl.sync();  // (1) row partials and query column sums of every rank visible
+  if (tid < b) {
+    float Mi = -INFINITY;
+    for (int r = 0; r < kStatCta; ++r) Mi = fmaxf(Mi, cl.map_shared_rank(rowM, r)[tid]);
+    float Li = 0.f;
+    for (int r = 0; r < kStatCta; ++r) {
+      const float m = cl.map_shared_rank(rowM, r)[tid];
+      if (m != -INFINITY) Li += cl.map_shared_rank(rowL, r)[tid] * ex2(m - Mi);
+    }
+    gM[tid] = Mi;
+    gInvL[tid] = (tid < nlast && Li > 0.f) ? 1.f / Li : 0.f;
+  }
+  if (tid < 128) {
+    float a = 0.f;
+    for (int r = 0; r < kStatCta; ++r) a += cl.map_shared_rank(qpart, r)[tid];
+    qb[tid] = (I8 ? a * P.q_scale[h] : a) / (float)nlast;
+  }
+  __syncthreads();
+
+  // ---- 2. part masses (warp per part, lanes over rows), block masses, kbar and logits
+  for (int p = p0 + warp; p < p1; p += nwarp) {
+    float a = 0.f, c = 0.f;
+    for (int i = lane; i < b; i += 32) {
+      if (i >= nlast) break;
+      const size_t o = hoff + (size_t)p * b + i;
+      const float m = P.pm[o];
+      const float w = (m == -INFINITY) ? 0.f : ex2(m - gM[i]) * gInvL[i];
+      a += P.plo[o] * w;
+      c += P.phi[o] * w;
+    }
+#pragma unroll
+    for (int sft = 16; sft > 0; sft >>= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, sft);
+      c += __shfl_xor_sync(0xffffffffu, c, sft);
+    }
+    if (lane == 0) {
+      LOp[p - p0] = a;
+      HIp[p - p0] = c;
     }
   }
   __syncthreads();
-  for (int c = tid; c < n; c += blockDim.x) {
-    vhat[(size_t)h * n + c] = lo_s[c] + hi_s[c];
-    const int o = c;
-    shat[(size_t)h * n + o] = lo_s[n - 1 - o] + (o <= n - 2 ? hi_s[n - 2 - o] : 0.f);
+  const float inv_nl = 1.f / (float)nlast;
+  for (int c = c0 + tid; c < c1; c += kStatThreads) {
+    float a = 0.f, e = 0.f;
+    for (int q = 0; q < per && c * per + q < npart; ++q) {
+      a += LOp[c * per + q - p0];
+      e += HIp[c * per + q - p0];
+    }
+    LOb[c - c0] = a;
+    HIb[c - c0] = e;
+    vh[c - c0] = (a + e) * inv_nl;
+    P.vhat[(size_t)h * n + c] = (a + e) * inv_nl;
   }
-  // logits of P_est, one warp per block c
-  float *z = lo_s;  // reuse after vhat/shat are written
-  __syncthreads();
-  for (int c = warp; c < n; c += blockDim.x / 32) {
-    const float *kr = kbar + ((size_t)kvh * n + c) * 128;
-    float a = 0.f;
+  // block means of K (warp per block) and the logits of P_est
+  const bool write_kbar = (h % P.g) == 0 && P.ext_kbar == nullptr;
+  for (int c = c0 + warp; c < c1; c += nwarp) {
+    float kv[4];
+    if (P.ext_kbar) {
 #pragma unroll
-    for (int t = 0; t < 4; ++t) a = fmaf(qb[lane + 32 * t], kr[lane + 32 * t], a);
+      for (int t = 0; t < 4; ++t) kv[t] = P.ext_kbar[((size_t)kvh * n + c) * 128 + lane + 32 * t];
+    } else {
+      const int rows = min(b, P.S - c * b);
+      float sc = 1.f / (float)rows;
+      if (I8) sc *= P.k_scale[kvh];
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1) a += __shfl_xor_sync(0xffffffffu, a, s);
-    if (lane == 0) z[c] = a * inv_sqrt_d;
+      for (int t = 0; t < 4; ++t) {
+        float s2 = 0.f;
+        for (int q = 0; q < per && c * per + q < npart; ++q)
+          s2 += P.ksum[((size_t)kvh * npart + c * per + q) * 128 + lane + 32 * t];
+        kv[t] = s2 * sc;
+        if (write_kbar) P.kbar[((size_t)kvh * n + c) * 128 + lane + 32 * t] = kv[t];
+      }
+    }
+    float z = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) z = fmaf(qb[lane + 32 * t], kv[t], z);
+#pragma unroll
+    for (int sft = 16; sft > 0; sft >>= 1) z += __shfl_xor_sync(0xffffffffu, z, sft);
+    if (lane == 0) zc[c - c0] = z * P.inv_sqrt_d;
   }
   __syncthreads();
-  float mx = -INFINITY;
-  for (int c = tid; c < n; c += blockDim.x) mx = fmaxf(mx, z[c]);
+  {
+    float mx = -INFINITY;
+    for (int c = c0 + tid; c < c1; c += kStatThreads) mx = fmaxf(mx, zc[c - c0]);
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
-  if (lane == 0) part[warp] = mx;
-  __syncthreads();
-  mx = part[0];
-  for (int w = 1; w < (int)(blockDim.x / 32); ++w) mx = fmaxf(mx, part[w]);
-  __syncthreads();
-  float sum = 0.f;
-  for (int c = tid; c < n; c += blockDim.x) {
-    const float e = expf(z[c] - mx);
-    hi_s[c] = e;
-    sum += e;
+    for (int sft = 16; sft > 0; sft >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sft));
+    if (lane == 0) red[warp] = mx;
+    __syncthreads();
+    if (tid == 0) {
+      float m = red[0];
+      for (int w = 1; w < nwarp; ++w) m = fmaxf(m, red[w]);
+      xch[0] = m;
+    }
   }
-#pragma unroll
-  for (int s = 16; s > 0; s >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, s);
-  if (lane == 0) part[warp] = sum;
-  __syncthreads();
-  sum = 0.f;
-  for (int w = 0; w < (int)(blockDim.x / 32); ++w) sum += part[w];
-  __syncthreads();
-  float js = 0.f;
-  for (int c = tid; c < n; c += blockDim.x) {
-    const float pe = hi_s[c] / sum;
-    pest[(size_t)h * n + c] = pe;
-    const float pv = vhat[(size_t)h * n + c];
-    const float m = 0.5f * (pv + pe);
-    if (pv > 0.f) js += 0.5f * pv * logf(pv / m);
-    if (pe > 0.f) js += 0.5f * pe * logf(pe / m);
+  cl.sync();  // (2) block masses and logit maxima of every rank visible
+  // slash statistics of the owned offsets from the mirrored blocks' owners
+  for (int o = c0 + tid; o < c1; o += kStatThreads) {
+    const int cl_ = n - 1 - o;
+    int kr = kStatCta - 1;
+    while (stat_block0(kr, n) > cl_) --kr;
+    float sv = cl.map_shared_rank(LOb, kr)[cl_ - stat_block0(kr, n)];
+    if (o <= n - 2) {
+      const int ch = n - 2 - o;
+      int kh = kStatCta - 1;
+      while (stat_block0(kh, n) > ch) --kh;
+      sv += cl.map_shared_rank(HIb, kh)[ch - stat_block0(kh, n)];
+    }
+    P.shat[(size_t)h * n + o] = sv * inv_nl;
   }
+  float gmax = -INFINITY;
+  for (int r = 0; r < kStatCta; ++r) gmax = fmaxf(gmax, cl.map_shared_rank(xch, r)[0]);
+  {
+    float sum = 0.f;
+    for (int c = c0 + tid; c < c1; c += kStatThreads) {
+      const float e = expf(zc[c - c0] - gmax);
+      zc[c - c0] = e;
+      sum += e;
+    }
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) js += __shfl_xor_sync(0xffffffffu, js, s);
-  if (lane == 0) part[warp] = js;
-  __syncthreads();
-  if (tid == 0) {
+    for (int sft = 16; sft > 0; sft >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, sft);
+    if (lane == 0) red[warp] = sum;
+    __syncthreads();
+    if (tid == 0) {
+      float s2 = 0.f;
+      for (int w = 0; w < nwarp; ++w) s2 += red[w];
+      xch[1] = s2;
+    }
+  }
+  cl.sync();  // (3) local exponential sums visible
+  float gsum = 0.f;
+  for (int r = 0; r < kStatCta; ++r) gsum += cl.map_shared_rank(xch, r)[1];
+  {
+    float js = 0.f;
+    for (int c = c0 + tid; c < c1; c += kStatThreads) {
+      const float pe = zc[c - c0] / gsum;
+      P.pest[(size_t)h * n + c] = pe;
+      const float pv = vh[c - c0];
+      const float m = 0.5f * (pv + pe);
+      if (pv > 0.f) js += 0.5f * pv * logf(pv / m);
+      if (pe > 0.f) js += 0.5f * pe * logf(pe / m);
+    }
+#pragma unroll
+    for (int sft = 16; sft > 0; sft >>= 1) js += __shfl_xor_sync(0xffffffffu, js, sft);
+    __syncthreads();  // red[] reuse
+    if (lane == 0) red[warp] = js;
+    __syncthreads();
+    if (tid == 0) {
+      float s2 = 0.f;
+      for (int w = 0; w < nwarp; ++w) s2 += red[w];
+      xch[2] = s2;
+    }
+  }
+  cl.sync();  // (4) local divergences visible
+  if (k == 0 && tid == 0) {
     float tot = 0.f;
-    for (int w = 0; w < (int)(blockDim.x / 32); ++w) tot += part[w];
-    jsd[h] = tot;
-    pattern[h] = (tot < tau) ? 1 : 0;
+    for (int r = 0; r < kStatCta; ++r) tot += cl.map_shared_rank(xch, r)[2];
+    P.jsd[h] = tot;
+    P.pattern[h] = (tot < P.tau) ? 1 : 0;
   }
+  cl.sync();  // (5) no rank leaves while another may still read its shared memory
 }
 
 // ---------------------------------------------------------------------------
@@ -763,14 +825,21 @@ __global__ void __launch_bounds__(256)
 // max); normalised to sum 1.  The diagonal is kept; the others are kept in
 // order of descending score (ties: lower index) while the kept sum is below
 // gamma.  The cut is found by bisection on the fp32 bit pattern of the
-// scores (monotone for positive floats): T = largest t with
-// sum_{c < r, bits(w_c) >= t} w_c >= gamma - w_r, stopping as soon as one
-// candidate is left between the bounds; everything above T is kept, then
-// ties at T by ascending index until the target is reached.  The row lives
-// in registers (element c in lane c % 32, slot c / 32).
+// scores (monotone for positive floats), between the smallest and the
+// largest candidate: T = largest t with sum_{c < r, bits(w_c) >= t} w_c >=
+// gamma - w_r, stopping as soon as one candidate is left between the
+// bounds; everything above T is kept, then ties at T by ascending index
+// until the target is reached.  The row lives in registers (element c in
+// lane c % 32, slot c / 32; the diagonal's slot is zeroed once w_r is read,
+// so a slot's bit pattern is its key and non-candidates never qualify).
+// Sums: each lane adds its slots in fp32 in a fixed order; the lane sums
+// are converted to fixed point (2^-30 units, exact integer addition) and
+// reduced across the warp in one instruction, so every sum is deterministic
+// and monotone in the threshold.
 // Output: counts[h*n + r], ascending list at cols[h*n(n+1)/2 + r(r+1)/2].
 // ---------------------------------------------------------------------------
 constexpr int kSelMaxN = 1024;
+constexpr float kCutFx = 1073741824.f;  // 2^30
 
 template <int NL>
 __device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const float *__restrict__ vhat,
@@ -788,8 +857,7 @@ __device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const floa
       v[i] = val;
       mx = fmaxf(mx, val);
     }
-#pragma unroll
-    for (int s = 16; s > 0; s >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, s));
+    mx = redux_max_f32(mx);
 #pragma unroll
     for (int i = 0; i < NL; ++i) v[i] = (lane + 32 * i <= r) ? expf(v[i] - mx) : 0.f;
   } else {
@@ -809,83 +877,87 @@ __device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const floa
   for (int s = 16; s > 0; s >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, s);
 #pragma unroll
   for (int i = 0; i < NL; ++i) v[i] = v[i] / zs;
-  // diagonal score w_r from lane r % 32, slot r / 32
+  // diagonal score w_r from lane r % 32, slot r / 32; then that slot is zeroed
   float wr_l = 0.f;
 #pragma unroll
   for (int i = 0; i < NL; ++i)
     if (i == (r >> 5)) wr_l = v[i];
   const float wr = __shfl_sync(0xffffffffu, wr_l, r & 31);
+#pragma unroll
+  for (int i = 0; i < NL; ++i)
+    if (lane + 32 * i == r) v[i] = 0.f;
   const float need = gamma - wr;
-  // candidates: c < r (slot value 0 and bits 0 elsewhere never qualify)
+  // lane sum of the slots with key >= t (four chains, fixed order), in fixed point
+  auto lane_sum_fx = [&](uint32_t t, uint32_t &cnt) -> uint32_t {
+    float f4[4] = {0.f, 0.f, 0.f, 0.f};
+    uint32_t c4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int i = 0; i < NL; ++i) {
+      const bool ge = __float_as_uint(v[i]) >= t;
+      f4[i & 3] += ge ? v[i] : 0.f;
+      c4[i & 3] += ge ? 1u : 0u;
+    }
+    cnt = (c4[0] + c4[1]) + (c4[2] + c4[3]);
+    return __float2uint_rn(((f4[0] + f4[1]) + (f4[2] + f4[3])) * kCutFx);
+  };
   int mode;  // 0 = all, 1 = diagonal only, 2 = cut at T
-  uint32_t T = 0;
-  float s_gt = 0.f;
+  uint32_t T = 0, need_fx = 0, s_gt = 0;
   if (gamma >= 1.f) {
     mode = 0;
   } else if (need <= 0.f) {
     mode = 1;
   } else {
-    float tot = 0.f;
-#pragma unroll
-    for (int i = 0; i < NL; ++i) tot += (lane + 32 * i < r) ? v[i] : 0.f;
-#pragma unroll
-    for (int s = 16; s > 0; s >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, s);
-    if (tot < need) {
+    need_fx = __float2uint_ru(need * kCutFx);
+    uint32_t cnt;
+    const uint32_t tot = redux_add_u32(lane_sum_fx(1u, cnt));  // every candidate with w > 0
+    if (tot < need_fx) {
       mode = 0;
     } else {
       mode = 2;
-      // invariant: f(lo) >= need > f(hi); c_lo / c_hi count candidates with
-      // bits >= lo / >= hi; f_hi = f(hi)
-      uint32_t lo = 0u, hi = 0x7F800000u;
-      int c_lo = r, c_hi = 0;
-      float f_hi = 0.f;
-      while (hi - lo > 1u && c_lo - c_hi > 1) {
+      // bracket: f(lo) >= need > f(hi); c_lo / c_hi count candidates with key >= lo / >= hi
+      uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+#pragma unroll
+      for (int i = 0; i < NL; ++i) {
+        const uint32_t key = __float_as_uint(v[i]);
+        if (key != 0u) {
+          kmin = min(kmin, key);
+          kmax = max(kmax, key);
+        }
+      }
+      uint32_t lo = redux_min_u32(kmin), hi = redux_max_u32(kmax) + 1u;
+      uint32_t c_lo = redux_add_u32(cnt), c_hi = 0u, f_hi = 0u;
+      while (hi - lo > 1u && c_lo - c_hi > 1u) {
         const uint32_t mid = lo + ((hi - lo) >> 1);
-        // four independent accumulation chains
-        float f4[4] = {0.f, 0.f, 0.f, 0.f};
-        int c4[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int i = 0; i < NL; ++i) {
-          const bool ge = (lane + 32 * i < r) && __float_as_uint(v[i]) >= mid;
-          f4[i & 3] += ge ? v[i] : 0.f;
-          c4[i & 3] += ge ? 1 : 0;
-        }
-        float f = (f4[0] + f4[1]) + (f4[2] + f4[3]);
-        int cnt = (c4[0] + c4[1]) + (c4[2] + c4[3]);
-#pragma unroll
-        for (int s = 16; s > 0; s >>= 1) {
-          f += __shfl_xor_sync(0xffffffffu, f, s);
-          cnt += __shfl_xor_sync(0xffffffffu, cnt, s);
-        }
-        if (f >= need) {
+        uint32_t cm;
+        const uint32_t fl = lane_sum_fx(mid, cm);
+        const uint32_t f = redux_add_u32(fl), cs = redux_add_u32(cm);
+        if (f >= need_fx) {
           lo = mid;
-          c_lo = cnt;
+          c_lo = cs;
         } else {
           hi = mid;
-          c_hi = cnt;
+          c_hi = cs;
           f_hi = f;
         }
       }
-      if (c_lo - c_hi == 1) {
+      if (c_lo - c_hi == 1u) {
         uint32_t tb = 0u;
 #pragma unroll
         for (int i = 0; i < NL; ++i) {
-          const uint32_t bits = __float_as_uint(v[i]);
-          if (lane + 32 * i < r && bits >= lo && bits < hi) tb = bits;
+          const uint32_t key = __float_as_uint(v[i]);
+          if (key >= lo && key < hi) tb = key;
         }
-#pragma unroll
-        for (int s = 16; s > 0; s >>= 1) tb = max(tb, __shfl_xor_sync(0xffffffffu, tb, s));
-        T = tb;
+        T = redux_max_u32(tb);
       } else {
         T = lo;
       }
-      s_gt = f_hi;  // every candidate above T has bits >= hi
+      s_gt = f_hi;  // every candidate above T has key >= hi
     }
   }
   // emit ascending; ties at T in index order until the target is reached
   int written = 0;
-  float tie_acc = s_gt;
-  const float tval = __uint_as_float(T);
+  uint32_t tie_acc = s_gt;
+  const uint32_t t_fx = __float2uint_rn(__uint_as_float(T) * kCutFx);
   bool ties_done = false;
 #pragma unroll
   for (int i = 0; i < NL; ++i) {
@@ -894,21 +966,21 @@ __device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const floa
     if (c <= r) {
       if (mode == 0 || c == r) keep = true;
       else if (mode == 2) {
-        const uint32_t bits = __float_as_uint(v[i]);
-        keep = bits > T;
-        is_tie = (bits == T);
+        const uint32_t key = __float_as_uint(v[i]);
+        keep = key > T;
+        is_tie = (key == T);
       }
     }
     if (mode == 2) {
       uint32_t tmask = __ballot_sync(0xffffffffu, is_tie);
       uint32_t take = 0u;
       while (tmask && !ties_done) {
-        if (tie_acc >= need) {
+        if (tie_acc >= need_fx) {
           ties_done = true;
           break;
         }
         take |= 1u << (__ffs(tmask) - 1);
-        tie_acc += tval;
+        tie_acc += t_fx;
         tmask &= tmask - 1u;
       }
       if (take & (1u << lane)) keep = true;

@@ -291,6 +291,28 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// Warp-wide reductions in one instruction (all 32 lanes take part).
+__device__ __forceinline__ uint32_t redux_add_u32(uint32_t v) {
+  uint32_t r;
+  asm volatile("redux.sync.add.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t redux_min_u32(uint32_t v) {
+  uint32_t r;
+  asm volatile("redux.sync.min.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ uint32_t redux_max_u32(uint32_t v) {
+  uint32_t r;
+  asm volatile("redux.sync.max.u32 %0, %1, 0xffffffff;" : "=r"(r) : "r"(v));
+  return r;
+}
+__device__ __forceinline__ float redux_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -313,6 +335,14 @@ __device__ __forceinline__ float ex2_fma(float x) {
   p = fmaf(p, f, kEx2C1);
   p = fmaf(p, f, kEx2C0);
   return __int_as_float(__float_as_int(p) + ((__float_as_int(j) - 0x4B400000) << 23));
+}
+
+// Exact int32 -> fp32 for |x| < 2^22 on the integer and FMA pipes (no
+// conversion unit): adding x to the bit pattern of 1.5 * 2^23 gives the float
+// 1.5 * 2^23 + x, from which 1.5 * 2^23 is subtracted exactly.  Used for
+// int8 x int8 dot products over d = 128 (|x| <= 127^2 * 128 < 2^21).
+__device__ __forceinline__ float i32_to_f32_small(uint32_t x) {
+  return __uint_as_float(x + 0x4B400000u) - 12582912.f;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -173,14 +173,14 @@ int fp_debug_capture_i8(int which, int h, int tile, int chunk, int32_t *out);
  *
  * Scratch: a fixed 32 MiB array inside the library (a file-scope device
  * array; every GPU that loads the library keeps it until process exit).  A
- * problem needs at most 12*Hq*C*b + 128*Hq*b + 8*Hq*C + 512*Hkv*C +
- * 512*Hkv*n bytes of it, with C = ceil(S/128) column parts (2*ceil(S/128)
- * when b = 64) and n = ceil(S/b), plus 2 KiB of alignment; e.g. S=32768 with
- * Hq=32, Hkv=8, b=128 fits, and so does S=131072 with Hq=16, Hkv=4, b=128.
+ * problem needs at most 12*Hq*C*b + 512*Hkv*C + 512*Hkv*n bytes of it, with
+ * C = ceil(S/128) column parts (2*ceil(S/128) when b = 64) and n = ceil(S/b),
+ * plus 1.25 KiB of alignment; e.g. S=32768 with Hq=32, Hkv=8, b=128 fits, and
+ * so does S=131072 with Hq=16, Hkv=4, b=128.
  * Larger problems are rejected with FP_ERR_ARG before anything is launched.
  * The first call on a device looks up the array's device address (set-up,
- * once per device, with that device current); make that first call before
- * any stream capture.  All calls share the one array and it keeps the last
+ * once per device, with that device current; after a device reset the next
+ * call looks it up again); make that first call before any stream capture.  All calls share the one array and it keeps the last
  * call's contents; every scratch word a call reads is written earlier in
  * the same call, so nothing needs clearing.  Calls whose executions overlap
  * on the GPU (different streams, or different host threads) race on the
