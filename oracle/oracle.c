@@ -381,3 +381,77 @@ void orc_rope_pool(const double *x, const double *cosT, const double *sinT, int 
         }
     }
 }
+
+/* ------------------------------------------------------------------------
+ * Head-pattern sharing (maplevalley article, section 5, future directions:
+ * similar heads share one sparse pattern).  The pages give no rule for
+ * "similar"; the written convention: within one GQA group (the g query heads
+ * of a KV head, in head order), head a joins the class of the earliest
+ * earlier class representative b with JSD(vhat_a, vhat_b) < eps (natural
+ * log, no square root, as for the pattern decision); a head that joins no
+ * class represents its own.  Every head of a class then attends to the union
+ * of the class members' block lists, so each head keeps at least its own
+ * gamma-coverage.
+ * vhat: [g][n] of the group's heads; cls[a] receives the representative's
+ * position in the group (cls[a] = a for a representative). */
+void orc_share_classes(const double *vhat, int g, int n, double eps, int32_t *cls)
+{
+    for (int a = 0; a < g; ++a) {
+        cls[a] = a;
+        for (int b = 0; b < a; ++b) {
+            if (cls[b] != b) continue;
+            if (orc_jsd(vhat + (size_t)a * n, vhat + (size_t)b * n, n) < eps) {
+                cls[a] = b;
+                break;
+            }
+        }
+    }
+}
+
+/* Ascending union of the lists of the heads in one class for query block r:
+ * lists[m] (counts[m] entries each, ascending) for the class's members m.
+ * Writes the union to out and returns its size. */
+int orc_union_lists(const int32_t *const *lists, const int32_t *counts, int members, int r, int32_t *out)
+{
+    char *seen = (char *)calloc((size_t)(r + 1), 1);
+    int cnt = 0;
+    for (int m = 0; m < members; ++m)
+        for (int e = 0; e < counts[m]; ++e) seen[lists[m][e]] = 1;
+    for (int c = 0; c <= r; ++c) if (seen[c]) out[cnt++] = c;
+    free(seen);
+    return cnt;
+}
+
+/* ------------------------------------------------------------------------
+ * Adaptive block size (maplevalley article, section 5: block size adjusted
+ * to the complexity of the content; section 4.3 lists 64, 128 and 256).  The
+ * written convention: at b = 128, the concentration of head h is
+ * k_h / n, where k_h is the smallest number of key blocks whose vhat
+ * (the exact pooled last-block attention of that head) sums to at least
+ * gamma (blocks taken by descending vhat); rho is the mean over heads.
+ * Concentrated attention (rho < 0.1) gets the finer b = 64 when S/64 <= 1024
+ * blocks, diffuse attention (rho >= 0.5) the coarser b = 256, anything else
+ * b = 128.  vhat: [Hq][n] at b = 128. */
+int orc_cover_count(const double *v, int n, double gamma)
+{
+    int *order = (int *)malloc(sizeof(int) * (size_t)n);
+    for (int c = 0; c < n; ++c) order[c] = c;
+    g_sort_w = v;
+    qsort(order, (size_t)n, sizeof(int), by_score_desc);
+    double cum = 0.0;
+    int k = 0;
+    while (k < n && cum < gamma) cum += v[order[k++]];
+    free(order);
+    return k;
+}
+
+int orc_choose_block_size(const double *vhat, int Hq, int n, int S, double gamma, double *rho_out)
+{
+    double rho = 0.0;
+    for (int h = 0; h < Hq; ++h) rho += (double)orc_cover_count(vhat + (size_t)h * n, n, gamma) / n;
+    rho /= Hq;
+    if (rho_out) *rho_out = rho;
+    if (rho < 0.1 && (S + 63) / 64 <= 1024) return 64;
+    if (rho >= 0.5) return 256;
+    return 128;
+}

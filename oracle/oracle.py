@@ -80,6 +80,14 @@ def lib():
         L.orc_qk_int_tile.argtypes = [pp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                       ctypes.c_int, ip]
         L.orc_qk_int_tile.restype = None
+        L.orc_share_classes.argtypes = [dp, ctypes.c_int, ctypes.c_int, ctypes.c_double, ip]
+        L.orc_share_classes.restype = None
+        L.orc_union_lists.argtypes = [ctypes.POINTER(ip), ip, ctypes.c_int, ctypes.c_int, ip]
+        L.orc_union_lists.restype = ctypes.c_int
+        L.orc_cover_count.argtypes = [dp, ctypes.c_int, ctypes.c_double]
+        L.orc_cover_count.restype = ctypes.c_int
+        L.orc_choose_block_size.argtypes = [dp, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double, dp]
+        L.orc_choose_block_size.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -223,3 +231,57 @@ def rope_pool(x, cos, sin, b):
     means = np.zeros((H, n, d))
     lib().orc_rope_pool(_dp(x), _dp(cos), _dp(sin), H, S, d, b, _dp(out), _dp(means))
     return out, means
+
+
+def share_classes(vhat_group, eps):
+    """Classes of the heads of one GQA group (vhat_group [g][n]): position of
+    each head's class representative within the group."""
+    v = np.ascontiguousarray(vhat_group, dtype=np.float64)
+    g, n = v.shape
+    cls = np.zeros(g, dtype=np.int32)
+    lib().orc_share_classes(_dp(v), g, n, float(eps), _ip(cls))
+    return cls
+
+
+def union_lists(lists, r):
+    """Ascending union of the given ascending block lists of query block r."""
+    arrs = [np.ascontiguousarray(np.asarray(x, dtype=np.int32)) for x in lists]
+    ptrs = (ctypes.POINTER(ctypes.c_int32) * len(arrs))(*[_ip(a) for a in arrs])
+    counts = np.array([len(a) for a in arrs], dtype=np.int32)
+    out = np.zeros(r + 1, dtype=np.int32)
+    cnt = lib().orc_union_lists(ptrs, _ip(counts), len(arrs), int(r), _ip(out))
+    return out[:cnt].copy()
+
+
+def share_index(heads, g, eps):
+    """Head-pattern sharing applied to per-head oracle results (the dicts of
+    OracleProblem.build_index_head, in head order): returns (classes per head
+    as absolute head indices, rows per head after the class union)."""
+    Hq = len(heads)
+    n = len(heads[0]["rows"])
+    cls_abs = np.zeros(Hq, dtype=np.int64)
+    rows = [None] * Hq
+    for j in range(Hq // g):
+        grp = list(range(j * g, (j + 1) * g))
+        cls = share_classes(np.stack([heads[h]["vhat"] for h in grp]), eps)
+        for a, h in enumerate(grp):
+            cls_abs[h] = grp[int(cls[a])]
+        for a, h in enumerate(grp):
+            members = [grp[m] for m in range(g) if int(cls[m]) == int(cls[a])]
+            rows[h] = [union_lists([heads[m]["rows"][r] for m in members], r) for r in range(n)]
+    return cls_abs, rows
+
+
+def cover_count(v, gamma):
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    return int(lib().orc_cover_count(_dp(v), len(v), float(gamma)))
+
+
+def choose_block_size(vhat128, S, gamma):
+    """The block-size rule on the b = 128 vertical statistics of every head
+    (vhat128 [Hq][n]): returns (b, rho)."""
+    v = np.ascontiguousarray(vhat128, dtype=np.float64)
+    Hq, n = v.shape
+    rho = np.zeros(1)
+    b = lib().orc_choose_block_size(_dp(v), Hq, n, int(S), float(gamma), _dp(rho))
+    return int(b), float(rho[0])

@@ -47,6 +47,12 @@ MUTANTS = [
     ("kbar_of_wrong_kv_head", "int b = P->b, d = P->d, n = nblocks(P), kvh = h / (P->Hq / P->Hkv);",
      "int b = P->b, d = P->d, n = nblocks(P), kvh = h % P->Hkv;"),
     ("qbar_of_kv_head_index", "orc_block_means(P, 0, h, qbar);", "orc_block_means(P, 0, kvh, qbar);"),
+    # head-pattern sharing and the block-size rule
+    ("share_joins_any_earlier_head", "            if (cls[b] != b) continue;\n", ""),
+    ("union_skips_last_member", "for (int m = 0; m < members; ++m)", "for (int m = 0; m + 1 < members; ++m)"),
+    ("cover_count_one_short", "while (k < n && cum < gamma) cum += v[order[k++]];",
+     "while (k + 1 < n && cum + v[order[k]] < gamma) cum += v[order[k++]];"),
+    ("block_size_regimes_swapped", "if (rho >= 0.5) return 256;", "if (rho >= 0.5) return 64;"),
 ]
 
 

@@ -517,3 +517,68 @@ def test_index_wiring_inputs_distinguish_the_operands():
         assert abs(float(jensenshannon(shat, pest)) ** 2 - jsd) > 1e-4
         wrong = torch.softmax(kbar[:3] @ qbar[n - 1] / math.sqrt(d), 0).numpy()
         assert np.abs(wrong - qa[2]).max() > 1e-3
+
+
+
+# ---------------------------------------------------------------- head-pattern sharing, adaptive block size
+
+def test_share_classes_follow_jsd_between_representatives():
+    """Greedy classes in head order: a head joins the earliest earlier
+    representative whose vhat is within JSD < eps (scipy's Jensen-Shannon
+    distance squared), else it represents its own class."""
+    base = np.array([0.4, 0.3, 0.2, 0.1])
+    near = np.array([0.38, 0.32, 0.2, 0.1])                  # close to base
+    mid = np.array([0.25, 0.25, 0.25, 0.25])
+    far = np.array([0.01, 0.01, 0.08, 0.9])
+    d_bn = jensenshannon(base, near) ** 2
+    d_bm = jensenshannon(base, mid) ** 2
+    d_nm = jensenshannon(near, mid) ** 2
+    assert d_bn < 1e-3 < d_nm < d_bm
+    eps = 0.5 * (d_nm + d_bm) if d_nm < d_bm else None
+    # mid is within eps of near (a member, not a representative) but not of base: own class
+    cls = orc.share_classes(np.stack([base, near, mid, far]), eps)
+    assert list(cls) == [0, 0, 2, 3]
+    # a larger eps lets mid join base's class; far still stands alone
+    cls = orc.share_classes(np.stack([base, near, mid, far]), d_bm * 1.01)
+    assert list(cls) == [0, 0, 0, 3]
+    # eps = 0 keeps every head alone (JSD >= 0 is never < 0)
+    assert list(orc.share_classes(np.stack([base, base, base]), 0.0)) == [0, 1, 2]
+    # identical heads always share for eps > 0 (JSD(P, P) = 0)
+    assert list(orc.share_classes(np.stack([far, base, far]), 1e-12)) == [0, 1, 0]
+
+
+def test_union_lists_is_the_set_union():
+    rng = np.random.default_rng(3)
+    for r in (0, 5, 40):
+        lists = [sorted(set(rng.choice(r + 1, size=int(rng.integers(1, r + 2)), replace=False).tolist()) | {r})
+                 for _ in range(3)]
+        got = orc.union_lists(lists, r)
+        assert list(got) == sorted(set().union(*map(set, lists)))
+
+
+def test_cover_count_by_sorting():
+    rng = np.random.default_rng(4)
+    for n in (1, 7, 100, 1024):
+        v = rng.random(n) ** 3
+        v /= v.sum()
+        for gamma in (0.3, 0.8, 0.9, 0.99):
+            csum = np.cumsum(np.sort(v)[::-1])
+            want = int(np.searchsorted(csum, gamma) + 1)   # first prefix with sum >= gamma
+            want = min(want, n)
+            assert orc.cover_count(v, gamma) == want, (n, gamma)
+    assert orc.cover_count(np.full(4, 0.25), 1.0) == 4
+
+
+def test_block_size_rule_regimes():
+    """rho = mean over heads of (blocks covering gamma of vhat) / n: concentrated
+    attention -> 64 (if S/64 <= 1024 blocks), diffuse -> 256, otherwise 128."""
+    n = 100
+    conc = np.zeros(n); conc[-1] = 0.95; conc[:-1] = 0.05 / (n - 1)        # 1 block covers 0.9
+    flat = np.full(n, 1.0 / n)                                            # 90 blocks for 0.9
+    assert orc.choose_block_size(np.stack([conc, conc]), 12800, 0.9) == (64, 0.01)
+    b, rho = orc.choose_block_size(np.stack([flat, flat]), 12800, 0.9)
+    assert b == 256 and abs(rho - 0.90) < 1e-12
+    b, rho = orc.choose_block_size(np.stack([conc, flat]), 12800, 0.9)
+    assert b == 128 and abs(rho - 0.455) < 1e-12
+    # concentrated, but S = 131072 would need 2048 blocks of 64: stays at 128
+    assert orc.choose_block_size(np.stack([conc, conc]), 131072, 0.9)[0] == 128
