@@ -481,6 +481,32 @@ def run_ours(args, w):
              "e2e": e2e, "clocks": clocks, "gpu_launches": KERNELS_PER_STEP * args.steps,
              "gpu": torch.cuda.get_device_name(dev)}
     extra["int8_peak"] = i8
+    # compact forms of the same index on the device (not part of the step): CSR rows and the
+    # per-(KV head, query block) union lists with head masks
+    rp = torch.empty(w.Hq * ((w.S + w.b - 1) // w.b) + 1, dtype=torch.int32, device=dev)
+    col = torch.empty(max(1, int(exp["nnz"])), dtype=torch.int32, device=dev)
+    gp = torch.empty(w.Hkv * ((w.S + w.b - 1) // w.b) + 1, dtype=torch.int32, device=dev)
+    fp.fp_index_group_lists(idx, gp, None, None, stream)
+    torch.cuda.synchronize(dev)
+    gtot = int(gp[-1])
+    gc = torch.empty(max(1, gtot), dtype=torch.int32, device=dev)
+    gm = torch.empty(max(1, gtot), dtype=torch.int32, device=dev)
+    ct = []
+    for _ in range(5):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        fp.fp_index_csr(idx, rp, col, stream)
+        e1.record(stream)
+        fp.fp_index_group_lists(idx, gp, gc, gm, stream)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        ct.append((e0.elapsed_time(e1), e1.elapsed_time(e2)))
+    extra["compact_lists"] = {"csr_ms": float(np.median([a for a, _ in ct])),
+                              "group_lists_ms": float(np.median([b for _, b in ct])),
+                              "nnz": int(exp["nnz"]), "group_entries": gtot,
+                              "note": "device CSR and per-group union lists of the timed index; the attention "
+                                      "reads the padded rows, so neither is part of the step"}
+    del rp, col, gp, gc, gm
     if not w.int8 and not args.no_w8a8:
         # the W8A8 variant of the same layer: Q and K quantised per head from these bf16 tensors
         del q, k, qq, kk
@@ -526,9 +552,16 @@ def run_ours(args, w):
     return 0
 
 
+SHARE_EPS = 0.05  # head-pattern sharing threshold reported in the sweep (half of tau)
+
+
 def run_sweep(args):
     """The S x b x gamma sweep on the 128K generator (Hq=32, Hkv=8): one JSON
-    line per point with density next to time (not the headline line)."""
+    line per point with density next to time (not the headline line).  At
+    b = 128 each line also carries the block size the content rule chooses
+    from that index (fp_choose_block_size) and the layer with head-pattern
+    sharing (fp_index_share, eps = SHARE_EPS): its density, sharing time and
+    attention time."""
     from dynamic_block_sparse_last_b200 import fp
     dev = torch.device("cuda", 0)
     cache = {}
@@ -540,13 +573,17 @@ def run_sweep(args):
         q, k, v = cache[w.S]
         out = torch.empty_like(q)
         idx = fp.fp_index_create(w.S, w.Hq, w.Hkv, w.d, w.b)
-        for _ in range(args.warmup):
+
+        def build():
             fp.fp_build_index(q, k, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, fp.FP_QK_BF16, None, None, idx)
+
+        for _ in range(args.warmup):
+            build()
             fp.fp_sparse_attn(q, k, v, None, None, idx, out)
         ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
         for e in ev:
             e[0].record()
-            fp.fp_build_index(q, k, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, fp.FP_QK_BF16, None, None, idx)
+            build()
             e[1].record()
             fp.fp_sparse_attn(q, k, v, None, None, idx, out)
             e[2].record()
@@ -557,11 +594,30 @@ def run_sweep(args):
         idx_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
         attn_ms = float(np.median([e[1].elapsed_time(e[2]) for e in ev]))
         layer = idx_ms + attn_ms
-        print(json.dumps({"sweep": w.name, "S": w.S, "b": w.b, "gamma": w.gamma,
-                          "density": nnz / (w.Hq * n * (n + 1) / 2), "index_ms": idx_ms, "attn_ms": attn_ms,
-                          "ms_per_layer": layer,
-                          "dense_equiv_tflops": synth.dense_equiv_flops(w.S, w.Hq, w.d) / (layer / 1e3) / 1e12}),
-              flush=True)
+        line = {"sweep": w.name, "S": w.S, "b": w.b, "gamma": w.gamma,
+                "density": nnz / (w.Hq * n * (n + 1) / 2), "index_ms": idx_ms, "attn_ms": attn_ms,
+                "ms_per_layer": layer,
+                "dense_equiv_tflops": synth.dense_equiv_flops(w.S, w.Hq, w.d) / (layer / 1e3) / 1e12}
+        if w.b == 128:
+            bsel, rho = fp.fp_choose_block_size(idx, w.gamma)
+            line["adaptive_block"] = {"b": bsel, "rho": rho}
+            # head-pattern sharing on the same index: lists replaced by class unions
+            sh = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+            for e in sh:
+                build()
+                e[0].record()
+                fp.fp_index_share(idx, SHARE_EPS)
+                e[1].record()
+                fp.fp_sparse_attn(q, k, v, None, None, idx, out)
+                e[2].record()
+            torch.cuda.synchronize()
+            assert fp.fp_get_device_error() == fp.FP_OK
+            cls = fp.fp_index_classes(idx)
+            line["shared"] = {"eps": SHARE_EPS, "classes": int(len(set(cls.tolist()))),
+                              "density": fp.fp_index_nnz(idx) / (w.Hq * n * (n + 1) / 2),
+                              "share_ms": float(np.median([e[0].elapsed_time(e[1]) for e in sh])),
+                              "attn_ms": float(np.median([e[1].elapsed_time(e[2]) for e in sh]))}
+        print(json.dumps(line), flush=True)
         idx.free()
     return 0
 

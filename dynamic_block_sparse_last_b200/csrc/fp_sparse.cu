@@ -17,6 +17,7 @@
 #include "fp_sparse.h"
 #include "index_kernels.cuh"
 #include "rope_pool.cuh"
+#include "share_kernels.cuh"
 
 using namespace fpk;
 
@@ -35,6 +36,7 @@ struct fp_index {
   bool slab_pooled;        // slab from the stream-ordered allocator (else cudaMalloc)
   cudaStream_t own;        // the index's own stream: allocation and release of the slab
   cudaEvent_t last_use;    // recorded on the caller's stream at the end of every build / attention call
+  cudaEvent_t ev_fork, ev_join;  // Q pooling on `own` beside the score kernel on the caller's stream
   float *pm, *plo, *phi;   // [Hq][npart][b]
   float *ksum;             // [Hkv][npart][128]
   float *kbar;             // [Hkv][n][128]
@@ -43,6 +45,10 @@ struct fp_index {
   float *jsd;              // [Hq]
   int *pattern;            // [Hq]
   int *counts;             // [Hq][n]
+  int *cls;                // [Hq] head-sharing class representatives (fp_index_share)
+  int *cover;              // [Hq] blocks covering gamma of vhat (fp_choose_block_size)
+  int *gcount;             // [Hkv][n] union sizes of the group lists (fp_index_group_lists)
+  int shared;              // the lists are class unions (fp_index_share ran on this build)
   int *cols;               // [Hq][n(n+1)/2]
   float *zlog;             // [Hq][n(n+1)/2] q-bar . k-bar logits (query-aware heads)
 };
@@ -215,9 +221,9 @@ struct StatsJob {
   const float *ext_kbar;  // K block means given by the caller (then ksum/kbar are not computed), or null
 };
 
-// k_score_last and k_head_stats on `st`.
+// k_score_last on `st`.
 template <bool I8>
-int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
+int launch_score(const StatsJob &J, int *err, cudaStream_t st) {
   int rc;
   CUtensorMap tq, tk;
   if (!make_map(&tq, J.q, I8, map_rows(J.Hq, J.ld, J.S)) || !make_map(&tk, J.k, I8, map_rows(J.Hkv, J.ld, J.S)))
@@ -252,7 +258,13 @@ int launch_pattern_stats(const StatsJob &J, int *err, cudaStream_t st) {
     sp.cap_h = c.s_h; sp.cap_slice = c.s_slice; sp.cap_ch = c.s_ch;
   }
   k_score_last<I8><<<dim3(R, tgroups, J.Hkv), ScoreCfg<I8>::kThreads, ScoreCfg<I8>::kSmem, st>>>(tq, tk, sp);
-  if ((rc = launch_status())) return rc;
+  return launch_status();
+}
+
+// k_head_stats on `st` (after launch_score).
+template <bool I8>
+int launch_head_stats(const StatsJob &J, cudaStream_t st) {
+  const int nlast = J.S - (J.n - 1) * J.b;
   HeadStatsParams hp;
   hp.S = J.S; hp.b = J.b; hp.n = J.n; hp.npart = J.npart; hp.g = J.g; hp.ld = J.ld; hp.nlast = nlast;
   hp.pm = J.pm; hp.plo = J.plo; hp.phi = J.phi;
@@ -286,14 +298,24 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   J.ksum = I->ksum; J.kbar = I->kbar;
   J.vhat = I->vhat; J.shat = I->shat; J.pest = I->pest; J.jsd = I->jsd; J.pattern = I->pattern;
   J.ext_kbar = ext_kbar;
-  if ((rc = launch_pattern_stats<I8>(J, err, st))) return rc;
-  const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
-  const float *qbar = ext_qbar, *kbar = ext_kbar ? ext_kbar : I->kbar;
+  // Q block means of every head on the index's own stream, beside the score
+  // kernel (which is bound by its exponentials and leaves HBM mostly idle).
+  // The fork point precedes the score kernel; the pooling kernel is queued
+  // after it, so the score kernel's CTAs are dispatched first.
+  const float *qbar = ext_qbar;
+  if (!qbar && cudaEventRecord(I->ev_fork, st) != cudaSuccess) return FP_ERR_CUDA;
+  if ((rc = launch_score<I8>(J, err, st))) return rc;
   if (!qbar) {
-    k_qbar<I8><<<dim3(I->n, I->Hq), 256, 0, st>>>(q, q_scale, I->pattern, I->S, I->ld, I->b, I->n, I->qbar);
+    if (cudaStreamWaitEvent(I->own, I->ev_fork, 0) != cudaSuccess) return FP_ERR_CUDA;
+    k_qpool<I8><<<dim3(I->n, I->Hq), 256, 0, I->own>>>(q, q_scale, I->S, I->ld, I->b, I->n, I->qbar);
     if ((rc = launch_status())) return rc;
+    if (cudaEventRecord(I->ev_join, I->own) != cudaSuccess) return FP_ERR_CUDA;
     qbar = I->qbar;
   }
+  if ((rc = launch_head_stats<I8>(J, st))) return rc;
+  const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
+  const float *kbar = ext_kbar ? ext_kbar : I->kbar;
+  if (!ext_qbar && cudaStreamWaitEvent(st, I->ev_join, 0) != cudaSuccess) return FP_ERR_CUDA;
   const int nt = (I->n + kLgTile - 1) / kLgTile;
   k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, qbar, kbar, I->g, I->n,
                                                                inv_sqrt_d, I->zlog);
@@ -360,6 +382,9 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   add((size_t)Hq * 4);
   add((size_t)Hq * 4);
   add((size_t)Hq * n * 4);
+  add((size_t)Hq * 4);
+  add((size_t)Hq * 4);
+  add((size_t)Hkv * n * 4);
   add((size_t)Hq * tri * 4);
   add((size_t)Hq * tri * 4);
   if (cudaStreamCreateWithFlags(&I->own, cudaStreamNonBlocking) != cudaSuccess) {
@@ -367,6 +392,19 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
     return FP_ERR_CUDA;
   }
   if (cudaEventCreateWithFlags(&I->last_use, cudaEventDisableTiming) != cudaSuccess) {
+    cudaStreamDestroy(I->own);
+    free(I);
+    return FP_ERR_CUDA;
+  }
+  if (cudaEventCreateWithFlags(&I->ev_fork, cudaEventDisableTiming) != cudaSuccess) {
+    cudaEventDestroy(I->last_use);
+    cudaStreamDestroy(I->own);
+    free(I);
+    return FP_ERR_CUDA;
+  }
+  if (cudaEventCreateWithFlags(&I->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+    cudaEventDestroy(I->ev_fork);
+    cudaEventDestroy(I->last_use);
     cudaStreamDestroy(I->own);
     free(I);
     return FP_ERR_CUDA;
@@ -379,6 +417,8 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
     cudaGetLastError();
     I->slab = nullptr;
     if (cudaMalloc(&I->slab, need) != cudaSuccess) {
+      cudaEventDestroy(I->ev_join);
+      cudaEventDestroy(I->ev_fork);
       cudaEventDestroy(I->last_use);
       cudaStreamDestroy(I->own);
       free(I);
@@ -399,6 +439,9 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   I->jsd = carve<float>(cur, (size_t)Hq);
   I->pattern = carve<int>(cur, (size_t)Hq);
   I->counts = carve<int>(cur, (size_t)Hq * n);
+  I->cls = carve<int>(cur, (size_t)Hq);
+  I->cover = carve<int>(cur, (size_t)Hq);
+  I->gcount = carve<int>(cur, (size_t)Hkv * n);
   I->cols = carve<int>(cur, (size_t)Hq * tri);
   I->zlog = carve<float>(cur, (size_t)Hq * tri);
   *out = I;
@@ -426,6 +469,8 @@ void fp_index_free(fp_index *I) {
     cudaEventSynchronize(I->last_use);
     cudaFree(I->slab);
   }
+  cudaEventDestroy(I->ev_join);
+  cudaEventDestroy(I->ev_fork);
   cudaEventDestroy(I->last_use);
   cudaStreamDestroy(I->own);  // returns at once; the stream's pending free still completes
   if (prev >= 0) cudaSetDevice(prev);
@@ -445,6 +490,7 @@ int fp_build_index(const void *q, const void *k, int S, int Hq, int Hkv, int d, 
   if (!aligned16(q) || !aligned16(k)) return FP_ERR_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   idx->built = 0;
+  idx->shared = 0;
   const int rc = qk_dtype == FP_QK_INT8 ? build_index_impl<true>(q, k, gamma, tau, q_scale, k_scale, idx, st)
                                         : build_index_impl<false>(q, k, gamma, tau, nullptr, nullptr, idx, st);
   if (rc == FP_OK) {
@@ -570,6 +616,89 @@ int fp_debug_qk_tile_i8(const int8_t *q8, const int8_t *k8, int S, int Hq, int H
   return launch_status();
 }
 
+int fp_index_share(fp_index *idx, float eps, void *stream) {
+  if (!idx || !(eps >= 0.f) || std::isnan(eps)) return FP_ERR_ARG;
+  if (!idx->built) return FP_ERR_STATE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem = (size_t)idx->g * idx->g * sizeof(float);
+  if (smem > 48 * 1024) return FP_ERR_ARG;
+  k_share_classes<<<idx->Hkv, 256, smem, st>>>(idx->vhat, idx->n, idx->g, eps, idx->cls);
+  int rc = launch_status();
+  if (rc) return rc;
+  k_share_union<<<(idx->Hq * idx->n + 7) / 8, 256, 0, st>>>(idx->cls, idx->Hq, idx->n, idx->g, idx->counts,
+                                                            idx->cols);
+  if ((rc = launch_status())) return rc;
+  idx->shared = 1;
+  return cudaEventRecord(idx->last_use, st) == cudaSuccess ? FP_OK : FP_ERR_CUDA;
+}
+
+int fp_index_csr(const fp_index *idx, int32_t *row_ptr, int32_t *col, void *stream) {
+  if (!idx || !row_ptr) return FP_ERR_ARG;
+  if (!idx->built) return FP_ERR_STATE;
+  if (((uintptr_t)row_ptr & 3u) || ((uintptr_t)col & 3u)) return FP_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int N = idx->Hq * idx->n;
+  k_scan_counts<<<1, 1024, 0, st>>>(idx->counts, N, row_ptr);
+  int rc = launch_status();
+  if (rc || !col) return rc;
+  k_compact_rows<<<(N + 7) / 8, 256, 0, st>>>(idx->counts, idx->cols, row_ptr, idx->Hq, idx->n, col);
+  return launch_status();
+}
+
+int fp_index_group_lists(const fp_index *idx, int32_t *grp_ptr, int32_t *grp_col, uint32_t *grp_mask,
+                         void *stream) {
+  if (!idx || !grp_ptr || (grp_col == nullptr) != (grp_mask == nullptr)) return FP_ERR_ARG;
+  if (!idx->built) return FP_ERR_STATE;
+  if (idx->g > 32) return FP_ERR_ARG;
+  if (((uintptr_t)grp_ptr & 3u) || ((uintptr_t)grp_col & 3u) || ((uintptr_t)grp_mask & 3u)) return FP_ERR_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int N = idx->Hkv * idx->n;
+  const size_t smem = (size_t)8 * idx->g * 32 * sizeof(uint32_t);
+  // sizes of the unions (into the index's own counts scratch for the groups), their scan, then the lists
+  k_group_lists<<<(N + 7) / 8, 256, smem, st>>>(idx->counts, idx->cols, idx->Hkv, idx->n, idx->g, nullptr,
+                                                idx->gcount, nullptr, nullptr);
+  int rc = launch_status();
+  if (rc) return rc;
+  k_scan_counts<<<1, 1024, 0, st>>>(idx->gcount, N, grp_ptr);
+  if ((rc = launch_status()) || !grp_col) return rc;
+  k_group_lists<<<(N + 7) / 8, 256, smem, st>>>(idx->counts, idx->cols, idx->Hkv, idx->n, idx->g, grp_ptr,
+                                                nullptr, grp_col, grp_mask);
+  return launch_status();
+}
+
+int fp_index_classes(const fp_index *idx, int32_t *cls, void *stream) {
+  if (!idx || !cls) return FP_ERR_ARG;
+  if (!idx->built) return FP_ERR_STATE;
+  if (!idx->shared) {
+    for (int h = 0; h < idx->Hq; ++h) cls[h] = h;
+    return FP_OK;
+  }
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP_ERR_CUDA;
+  return cudaMemcpy(cls, idx->cls, (size_t)idx->Hq * 4, cudaMemcpyDeviceToHost) == cudaSuccess ? FP_OK
+                                                                                                : FP_ERR_CUDA;
+}
+
+int fp_choose_block_size(const fp_index *idx, float gamma, int *b, float *rho, void *stream) {
+  if (!idx || !b || !(gamma > 0.f && gamma <= 1.f) || std::isnan(gamma)) return FP_ERR_ARG;
+  if (!idx->built || idx->b != 128 || idx->ld != idx->S) return FP_ERR_STATE;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  k_cover_count<<<(idx->Hq + 7) / 8, 256, 0, st>>>(idx->vhat, idx->Hq, idx->n, gamma, idx->cover);
+  const int rc = launch_status();
+  if (rc) return rc;
+  std::vector<int> cover(idx->Hq);
+  if (cudaStreamSynchronize(st) != cudaSuccess ||
+      cudaMemcpy(cover.data(), idx->cover, cover.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return FP_ERR_CUDA;
+  double r = 0.0;
+  for (int h = 0; h < idx->Hq; ++h) r += (double)cover[h] / idx->n;
+  r /= idx->Hq;
+  if (rho) *rho = (float)r;
+  if (r < 0.1 && (idx->S + 63) / 64 <= kSelMaxN) *b = 64;
+  else if (r >= 0.5) *b = 256;
+  else *b = 128;
+  return FP_OK;
+}
+
 int fp_debug_capture_i8(int which, int h, int tile, int chunk, int32_t *out) {
   if (which != 0 && which != 1) return FP_ERR_ARG;
   if (out && (!aligned16(out) || h < 0 || tile < 0 || chunk < 0)) return FP_ERR_ARG;
@@ -640,7 +769,8 @@ int stats_noalloc_impl(const void *q, const void *k, int S, int Hq, int Hkv, int
   J.pm = pm; J.plo = plo; J.phi = phi;
   J.ksum = ksum; J.kbar = kbar;
   J.vhat = vhat; J.shat = shat; J.pest = pest; J.jsd = jsd; J.pattern = pattern;
-  return launch_pattern_stats<I8>(J, err, st);
+  if ((rc = launch_score<I8>(J, err, st))) return rc;
+  return launch_head_stats<I8>(J, st);
 }
 
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }

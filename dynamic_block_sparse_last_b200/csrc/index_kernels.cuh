@@ -16,7 +16,8 @@
 //   k_head_stats   one cluster per head: row max / sum, row-normalised
 //                  block masses, vhat, shat, block means of K, P_est, JSD,
 //                  pattern.
-//   k_qbar         block means of Q for query-aware heads only.
+//   k_qpool        block means of Q of every head, on a second stream
+//                  beside k_score_last.
 //   k_qa_logits    q-bar . k-bar logits of query-aware heads (tiled fp32).
 //   k_cut          per (head, query block): scores, gamma cut, sorted list.
 #pragma once
@@ -73,7 +74,9 @@ struct ScoreParams {
 
 template <bool I8>
 struct ScoreCfg {
-  static constexpr int kStages = I8 ? 4 : 3;
+  // two 32 KB K stages for bf16 keep the CTA at 193 KB of shared memory, so a
+  // Q-pooling CTA (k_qpool) fits beside it on the same SM
+  static constexpr int kStages = I8 ? 4 : 2;
   static constexpr int kTileBytes = I8 ? 16384 : 32768;  // 128 rows x 128 elements
   static constexpr int kTiles = 4;       // row tiles per CTA
   static constexpr int kSumWarps = 2;
@@ -277,22 +280,23 @@ __global__ void __launch_bounds__(736, 1)
         if (I8) scale2 *= P.q_scale[hh] * P.k_scale[kvh];
         const uint32_t taddr = tmem + t * 128 + (((warp & 3) * 32) << 16);
         const bool cap_on = I8 && P.cap != nullptr && hh == P.cap_h && (tile % tiles_per_head) == P.cap_slice;
+        const uint64_t sc2 = f2_pack(scale2, scale2);
         bool ok = true;
         float m = -INFINITY;
-        float lo4[4] = {0.f, 0.f, 0.f, 0.f}, hi4[4] = {0.f, 0.f, 0.f, 0.f};
+        uint64_t lo2 = 0ull, hi2 = 0ull;  // the part's lo / hi sums as packed fp32 pairs
         for (int u = 0; u < U && ok; ++u) {
           const int ch = ch0 + u;
           // One pass over the chunk in 32-column pieces with an online max:
           // lo/hi are kept relative to the running max m and rescaled when a
           // piece raises it.  Columns t <= i (block-relative) go to lo, the
-          // rest to hi; in the last block columns t > i are causally masked.
-          // With b = 64 each 64-column half is a block of its own and gets
-          // its own (max, lo, hi) part; otherwise the chunk is one part.
+          // rest to hi; in the last block columns t > i are causally masked
+          // (their exponentials are 0).  With b = 64 each 64-column half is a
+          // block of its own and gets its own (max, lo, hi) part; otherwise
+          // the chunk is one part.
           for (int hf = 0; hf < 2; ++hf) {
             if (hf == 0 || P.nsub == 2) {
               m = -INFINITY;
-#pragma unroll
-              for (int w4 = 0; w4 < 4; ++w4) lo4[w4] = hi4[w4] = 0.f;
+              lo2 = hi2 = 0ull;
             }
             if (!mbar_wait(smem_u32(&bar_sfull[t][hf]), u & 1, abort_flag, P.err)) { ok = false; break; }
             tc_fence_after();
@@ -312,64 +316,72 @@ __global__ void __launch_bounds__(736, 1)
               const int key0 = ch * 128 + hf * 64 + qq * 32;  // first key of the piece
               const int blk = key0 / P.b;
               if (blk > P.n - 1) continue;                    // past the last block: masked
-              const bool last_block = blk == P.n - 1;
-              const int t0 = key0 - blk * P.b;                // block-relative column of the piece
-              const int dlt = i - t0;  // columns e <= dlt are on the lo side
-              float pm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+              const int dlt = i - (key0 - blk * P.b);         // columns e <= dlt are on the lo side
+              float s[32];
 #pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const float s = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
-                const bool valid = !last_block || (e <= dlt);
-                pm4[e & 3] = valid ? fmaxf(pm4[e & 3], s) : pm4[e & 3];
+              for (int e = 0; e < 32; ++e) s[e] = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
+              if (blk == P.n - 1 && dlt < 31) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s[e] = (e <= dlt) ? s[e] : -INFINITY;
               }
-              const float pmx = fmaxf(fmaxf(pm4[0], pm4[1]), fmaxf(pm4[2], pm4[3]));
+              // piece max: eight chains of three-input max, then a short tree
+              float m8[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) m8[e] = fmax3(s[e], s[8 + e], s[16 + e]);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[24 + e]);
+              const float pmx =
+                  fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
               if (pmx == -INFINITY) continue;  // whole piece masked
               if (pmx > m) {
                 const float f = (m == -INFINITY) ? 0.f : ex2((m - pmx) * scale2);
-#pragma unroll
-                for (int w4 = 0; w4 < 4; ++w4) {
-                  lo4[w4] *= f;
-                  hi4[w4] *= f;
-                }
+                const uint64_t f2 = f2_pack(f, f);
+                lo2 = f2_mul(lo2, f2);
+                hi2 = f2_mul(hi2, f2);
                 m = pmx;
               }
-              const float m2p = m * scale2;
-              if (dlt >= 31) {
+              const float nm = -m * scale2;
+              const uint64_t nm2 = f2_pack(nm, nm);
+              // exponent arguments two at a time (packed fp32 FMA), ex2, packed adds
+              if (dlt >= 31 || dlt < 0) {
+                uint64_t a0 = 0ull, a1 = 0ull;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  const float s = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
-                  lo4[e & 3] += ex2(fmaf(s, scale2, -m2p));
+                for (int e = 0; e < 32; e += 4) {
+                  float x0, x1, x2, x3;
+                  f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+                  f2_unpack(f2_fma(f2_pack(s[e + 2], s[e + 3]), sc2, nm2), x2, x3);
+                  a0 = f2_add(a0, f2_pack(ex2(x0), ex2(x1)));
+                  a1 = f2_add(a1, f2_pack(ex2(x2), ex2(x3)));
                 }
-              } else if (dlt < 0) {
-                if (!last_block) {
-#pragma unroll
-                  for (int e = 0; e < 32; ++e) {
-                    const float s = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
-                    hi4[e & 3] += ex2(fmaf(s, scale2, -m2p));
-                  }
-                }
+                if (dlt >= 31) lo2 = f2_add(lo2, f2_add(a0, a1));
+                else hi2 = f2_add(hi2, f2_add(a0, a1));
               } else {
+                uint64_t l0 = 0ull, h0 = 0ull;
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                  const float s = I8 ? i32_to_f32_small(r[e]) : __uint_as_float(r[e]);
-                  const float p = ex2(fmaf(s, scale2, -m2p));
-                  if (e <= dlt) lo4[e & 3] += p;
-                  else if (!last_block) hi4[e & 3] += p;
+                for (int e = 0; e < 32; e += 2) {
+                  float x0, x1;
+                  f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+                  const float p0 = ex2(x0), p1 = ex2(x1);
+                  const bool q0 = e <= dlt, q1 = e + 1 <= dlt;
+                  l0 = f2_add(l0, f2_pack(q0 ? p0 : 0.f, q1 ? p1 : 0.f));
+                  h0 = f2_add(h0, f2_pack(q0 ? 0.f : p0, q1 ? 0.f : p1));
                 }
+                lo2 = f2_add(lo2, l0);
+                hi2 = f2_add(hi2, h0);
               }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&bar_sfree[t][hf]));
             if ((hf == 1 || P.nsub == 2) && i < P.nlast) {
-              const float m2 = m * scale2;
-              const float lo = (lo4[0] + lo4[1]) + (lo4[2] + lo4[3]);
-              const float hi = (hi4[0] + hi4[1]) + (hi4[2] + hi4[3]);
+              float l_a, l_b, h_a, h_b;
+              f2_unpack(lo2, l_a, l_b);
+              f2_unpack(hi2, h_a, h_b);
               const int part = ch * P.nsub + (P.nsub == 2 ? hf : 0);
               const size_t o = ((size_t)hh * P.nch * P.nsub + part) * P.b + i;
-              P.pm[o] = m2;
-              P.plo[o] = lo;
-              P.phi[o] = hi;
+              P.pm[o] = m * scale2;
+              P.plo[o] = l_a + l_b;
+              P.phi[o] = h_a + h_b;
             }
           }
           if (!ok) break;
@@ -668,19 +680,38 @@ __global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads)
 }
 
 // ---------------------------------------------------------------------------
-// k_qbar: grid (n, Hq), block 256: qbar[h][r][t] = mean of the Q rows of
-// block r (b rows, or S - (n-1)b for a partial last block), only for heads
-// whose pattern is query-aware (others exit).
+// k_qpool: grid (n, Hq), block 256, at most 48 registers per thread (one CTA
+// fits beside a k_score_last CTA on the same SM, so the two overlap: the
+// score kernel is bound by its exponentials and leaves HBM mostly idle).
+// qbar[h][r][t] = mean of the Q rows of block r (b rows, or S - (n-1)b for a
+// partial last block), for every head: which heads are query-aware is known
+// only after the scores.  Thread (c8 = tid & 15, rr = tid >> 4) owns columns
+// 8 c8 .. 8 c8 + 7 and rows rr, rr + 16, ...; the block kPoolAhead blocks
+// ahead is prefetched into L2 (bulk prefetch, no registers held).
 // ---------------------------------------------------------------------------
+constexpr int kPoolAhead = 4;
+
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
 template <bool I8>
-__global__ void __launch_bounds__(256)
-    k_qbar(const void *__restrict__ q, const float *__restrict__ q_scale,
-           const int *__restrict__ pattern, int S, int ld, int b, int n, float *__restrict__ qbar) {
+__global__ void __maxnreg__(48)
+    k_qpool(const void *__restrict__ q, const float *__restrict__ q_scale, int S, int ld, int b, int n,
+            float *__restrict__ qbar) {
   const int r = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-  if (pattern[h] != 1) return;
   __shared__ float red[16][128];
   const size_t row0 = (size_t)h * ld + (size_t)r * b;
   const int rows = min(b, S - r * b);
+  const int esz = I8 ? 1 : 2;
+  if (tid == 0 && r + kPoolAhead < n) {
+    const int ra = r + kPoolAhead;
+    const int arows = min(b, S - ra * b);
+    // 16-byte multiples: a row is 128 (int8) or 256 (bf16) bytes
+    prefetch_l2(reinterpret_cast<const char *>(q) + ((size_t)h * ld + (size_t)ra * b) * 128 * esz,
+                (uint32_t)arows * 128u * esz);
+  }
   if (I8) {
     // 8 threads per 128-byte row, 32 rows per pass; thread owns 16 columns
     const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
@@ -688,13 +719,13 @@ __global__ void __launch_bounds__(256)
     int acc[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) acc[e] = 0;
+#pragma unroll 2
     for (int p = rr; p < rows; p += 32) {
       const int4 v = *reinterpret_cast<const int4 *>(q8 + (row0 + p) * 128 + c16 * 16);
       const int w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 16; ++e) acc[e] += (int)(int8_t)((w[e >> 2] >> (8 * (e & 3))) & 0xff);
     }
-    // reduce over rr (32 groups) via shuffles within the 4 groups of a warp then smem
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       int a = acc[e];
@@ -709,26 +740,32 @@ __global__ void __launch_bounds__(256)
     }
     __syncthreads();
     if (tid < 128) {
-      float s = 0.f;
-      for (int w = 0; w < 8; ++w) s += red[w][tid];
-      qbar[((size_t)h * n + r) * 128 + tid] = s * q_scale[h] / (float)rows;
+      float s2 = 0.f;
+      for (int w = 0; w < 8; ++w) s2 += red[w][tid];
+      qbar[((size_t)h * n + r) * 128 + tid] = s2 * q_scale[h] / (float)rows;
     }
   } else {
-    // 16 threads per 256-byte row, 16 rows per pass; thread owns 8 columns
+    // 16 threads per 256-byte row, 16 rows per pass; thread owns 8 columns;
+    // four rows' loads in flight before they are added
     const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(q);
     const int c8 = tid & 15, rr = tid >> 4;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 4
-    for (int p = rr; p < rows; p += 16) {
-      const uint4 v = *reinterpret_cast<const uint4 *>(qh + (row0 + p) * 128 + c8 * 8);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int p = rr; p < rows; p += 64) {
+      uint4 v[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
-        acc[2 * e] += f.x;
-        acc[2 * e + 1] += f.y;
+      for (int j = 0; j < 4; ++j)
+        v[j] = (p + 16 * j < rows) ? *reinterpret_cast<const uint4 *>(qh + (row0 + p + 16 * j) * 128 + c8 * 8)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[2 * e] += __uint_as_float(w[e] << 16);
+          acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+        }
       }
     }
 #pragma unroll
@@ -740,9 +777,9 @@ __global__ void __launch_bounds__(256)
     }
     __syncthreads();
     if (tid < 128) {
-      float s = 0.f;
-      for (int w = 0; w < 8; ++w) s += red[w][tid];
-      qbar[((size_t)h * n + r) * 128 + tid] = s / (float)rows;
+      float s2 = 0.f;
+      for (int w = 0; w < 8; ++w) s2 += red[w][tid];
+      qbar[((size_t)h * n + r) * 128 + tid] = s2 / (float)rows;
     }
   }
 }
@@ -752,8 +789,10 @@ __global__ void __launch_bounds__(256)
 // query-aware heads only (others exit): the lower triangle of
 // Z = qbar kbar^T / sqrt(d), z[h][r][c] for c <= r, in the padded triangular
 // layout (row r at h*n(n+1)/2 + r(r+1)/2).  Tiled fp32 product: 64 x 64
-// output tile per CTA, 4 x 4 outputs per thread, d staged through shared
-// memory 32 at a time.
+// output tile per CTA, 4 x 4 outputs per thread held as column pairs and
+// updated with packed fp32 FMAs; d is staged through shared memory 32 at a
+// time, double-buffered (the next slice is loaded into registers while the
+// current one is multiplied).
 // ---------------------------------------------------------------------------
 constexpr int kLgTile = 64;
 constexpr int kLgK = 32;
@@ -764,8 +803,8 @@ __global__ void __launch_bounds__(256)
                 const float *__restrict__ kbar, int g, int n, float inv_sqrt_d, float *__restrict__ z) {
   const int h = blockIdx.y;
   if (pattern[h] != 1) return;
-  __shared__ __align__(16) float As[kLgK][kLgStride];  // [k][row]
-  __shared__ __align__(16) float Bs[kLgK][kLgStride];  // [k][col]
+  __shared__ __align__(16) float As[2][kLgK][kLgStride];  // [buffer][k][row]
+  __shared__ __align__(16) float Bs[2][kLgK][kLgStride];  // [buffer][k][col]
   // lower-triangular tile (tr, tc), tc <= tr, from the linear index
   const int x = blockIdx.x;
   int tr = (int)((sqrtf(8.f * (float)x + 1.f) - 1.f) * 0.5f);
@@ -777,44 +816,67 @@ __global__ void __launch_bounds__(256)
   const int row0 = tr * kLgTile, col0 = tc * kLgTile;
   const float *qh = qbar + (size_t)h * n * 128;
   const float *kh = kbar + (size_t)kvh * n * 128;
-  float acc[4][4];
-#pragma unroll
-  for (int a = 0; a < 4; ++a)
-#pragma unroll
-    for (int b2 = 0; b2 < 4; ++b2) acc[a][b2] = 0.f;
-  for (int k0 = 0; k0 < 128; k0 += kLgK) {
-    __syncthreads();
+  // this thread's share of a k-slice: rows rr0, rr0 + 32 of q-bar and k-bar, 4 consecutive k
+  const int rr0 = tid >> 3, k4 = (tid & 7) * 4;
+  float4 qa[2], kb[2];
+  auto load = [&](int k0) {
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int f = tid + u * 256, rr = f >> 3, k4 = (f & 7) * 4;
-      const float4 qa = (row0 + rr < n) ? *reinterpret_cast<const float4 *>(qh + (size_t)(row0 + rr) * 128 + k0 + k4)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 kb = (col0 + rr < n) ? *reinterpret_cast<const float4 *>(kh + (size_t)(col0 + rr) * 128 + k0 + k4)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-      As[k4 + 0][rr] = qa.x; As[k4 + 1][rr] = qa.y; As[k4 + 2][rr] = qa.z; As[k4 + 3][rr] = qa.w;
-      Bs[k4 + 0][rr] = kb.x; Bs[k4 + 1][rr] = kb.y; Bs[k4 + 2][rr] = kb.z; Bs[k4 + 3][rr] = kb.w;
+      const int rr = rr0 + 32 * u;
+      qa[u] = (row0 + rr < n) ? *reinterpret_cast<const float4 *>(qh + (size_t)(row0 + rr) * 128 + k0 + k4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      kb[u] = (col0 + rr < n) ? *reinterpret_cast<const float4 *>(kh + (size_t)(col0 + rr) * 128 + k0 + k4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    __syncthreads();
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int rr = rr0 + 32 * u;
+      As[buf][k4 + 0][rr] = qa[u].x; As[buf][k4 + 1][rr] = qa[u].y;
+      As[buf][k4 + 2][rr] = qa[u].z; As[buf][k4 + 3][rr] = qa[u].w;
+      Bs[buf][k4 + 0][rr] = kb[u].x; Bs[buf][k4 + 1][rr] = kb[u].y;
+      Bs[buf][k4 + 2][rr] = kb[u].z; Bs[buf][k4 + 3][rr] = kb[u].w;
+    }
+  };
+  uint64_t acc[4][2];  // rows ty*4 + a, column pairs tx*4 + 2p, +1
+#pragma unroll
+  for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0ull;
+  load(0);
+  store(0);
+  __syncthreads();
+#pragma unroll 1
+  for (int kt = 0; kt < 128 / kLgK; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < 128 / kLgK) load((kt + 1) * kLgK);
 #pragma unroll 8
     for (int k = 0; k < kLgK; ++k) {
-      const float4 a4 = *reinterpret_cast<const float4 *>(&As[k][ty * 4]);
-      const float4 b4 = *reinterpret_cast<const float4 *>(&Bs[k][tx * 4]);
-      const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+      const float4 a4 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 4]);
+      const float4 b4 = *reinterpret_cast<const float4 *>(&Bs[buf][k][tx * 4]);
+      const uint64_t b01 = f2_pack(b4.x, b4.y), b23 = f2_pack(b4.z, b4.w);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b2 = 0; b2 < 4; ++b2) acc[a][b2] = fmaf(av[a], bv[b2], acc[a][b2]);
+      for (int a = 0; a < 4; ++a) {
+        const uint64_t aa = f2_pack(av[a], av[a]);
+        acc[a][0] = f2_fma(aa, b01, acc[a][0]);
+        acc[a][1] = f2_fma(aa, b23, acc[a][1]);
+      }
     }
+    if (kt + 1 < 128 / kLgK) store(buf ^ 1);
+    __syncthreads();
   }
   float *zh = z + (size_t)h * ((size_t)n * (n + 1) / 2);
 #pragma unroll
   for (int a = 0; a < 4; ++a) {
     const int r = row0 + ty * 4 + a;
     if (r >= n) continue;
+    float v[4];
+    f2_unpack(acc[a][0], v[0], v[1]);
+    f2_unpack(acc[a][1], v[2], v[3]);
 #pragma unroll
     for (int b2 = 0; b2 < 4; ++b2) {
       const int c = col0 + tx * 4 + b2;
-      if (c <= r) zh[(size_t)r * (r + 1) / 2 + c] = acc[a][b2] * inv_sqrt_d;
+      if (c <= r) zh[(size_t)r * (r + 1) / 2 + c] = v[b2] * inv_sqrt_d;
     }
   }
 }

@@ -21,6 +21,8 @@ FP_PATTERN_VS, FP_PATTERN_QA = 0, 1
 SYMBOLS = ("fp_index_create", "fp_index_free", "fp_build_index", "fp_sparse_attn", "fp_index_info",
            "fp_index_nnz", "fp_index_export", "fp_get_device_error", "fp_debug_wait_timeout",
            "fp_debug_qk_tile_i8", "fp_debug_capture_i8", "fp_pattern_stats_noalloc", "fp_strerror",
+           "fp_index_share", "fp_index_classes", "fp_choose_block_size", "fp_index_csr",
+           "fp_index_group_lists",
            "fp_prefill_create", "fp_prefill_free", "fp_prefill_enqueue", "fp_prefill_wait", "fp_prefill_run",
            "fp_prefill_group_index", "fp_varlen_create", "fp_varlen_free", "fp_varlen_build_index",
            "fp_varlen_sparse_attn", "fp_varlen_index", "fp_rope_pool", "fp_build_index_pooled")
@@ -50,6 +52,11 @@ def _load():
     L.fp_debug_wait_timeout.argtypes = [i, vp]
     L.fp_debug_qk_tile_i8.argtypes = [vp, vp, i, i, i, i, i, i, i, vp, vp]
     L.fp_debug_capture_i8.argtypes = [i, i, i, i, vp]
+    L.fp_index_share.argtypes = [vp, f, vp]
+    L.fp_index_csr.argtypes = [vp, vp, vp, vp]
+    L.fp_index_group_lists.argtypes = [vp, vp, vp, vp, vp]
+    L.fp_index_classes.argtypes = [vp, vp, vp]
+    L.fp_choose_block_size.argtypes = [vp, f, ctypes.POINTER(i), ctypes.POINTER(f), vp]
     L.fp_pattern_stats_noalloc.argtypes = [vp, vp, i, i, i, i, i, f, i, vp, vp, vp, vp, vp, vp, vp, vp]
     L.fp_strerror.argtypes = [i]
     L.fp_strerror.restype = ctypes.c_char_p
@@ -204,6 +211,41 @@ def fp_debug_wait_timeout(timeout_us: int, stream=None):
 def fp_debug_qk_tile_i8(q8, k8, S, Hq, Hkv, d, h, p0, j0, out, stream=None):
     _check(_lib.fp_debug_qk_tile_i8(_ptr(q8), _ptr(k8), S, Hq, Hkv, d, h, p0, j0, _ptr(out), _stream(stream)),
            "fp_debug_qk_tile_i8")
+
+
+def fp_index_share(idx, eps, stream=None):
+    """Head-pattern sharing on a built index: classes by JSD of vhat < eps
+    within each GQA group, every member's lists replaced by the class union."""
+    _check(_lib.fp_index_share(idx.handle, float(eps), _stream(stream)), "fp_index_share")
+
+
+def fp_index_csr(idx, row_ptr, col=None, stream=None):
+    """Device CSR of the index into caller-owned device int32 tensors
+    (row_ptr [Hq*n + 1], col [nnz] or None for the offsets only)."""
+    _check(_lib.fp_index_csr(idx.handle, _ptr(row_ptr), _ptr(col), _stream(stream)), "fp_index_csr")
+
+
+def fp_index_group_lists(idx, grp_ptr, grp_col=None, grp_mask=None, stream=None):
+    """Per-(KV head, query block) union lists with head masks into caller-owned
+    device tensors (grp_ptr int32 [Hkv*n + 1]; grp_col int32, grp_mask int32
+    bit patterns [total], or both None for the offsets only)."""
+    _check(_lib.fp_index_group_lists(idx.handle, _ptr(grp_ptr), _ptr(grp_col), _ptr(grp_mask), _stream(stream)),
+           "fp_index_group_lists")
+
+
+def fp_index_classes(idx, stream=None):
+    import numpy as np
+    cls = np.zeros(idx.Hq, dtype=np.int32)
+    _check(_lib.fp_index_classes(idx.handle, cls.ctypes.data, _stream(stream)), "fp_index_classes")
+    return cls
+
+
+def fp_choose_block_size(idx, gamma, stream=None):
+    """Block size chosen by the content rule from an index built at b = 128: (b, rho)."""
+    b, rho = ctypes.c_int(0), ctypes.c_float(0.0)
+    _check(_lib.fp_choose_block_size(idx.handle, float(gamma), ctypes.byref(b), ctypes.byref(rho), _stream(stream)),
+           "fp_choose_block_size")
+    return b.value, rho.value
 
 
 def fp_debug_capture_i8(which, h, tile, chunk, out):

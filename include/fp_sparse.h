@@ -125,6 +125,56 @@ int fp_index_nnz(const fp_index *idx, int64_t *nnz, void *stream);
 int fp_index_export(const fp_index *idx, int32_t *row_ptr, int32_t *col, uint8_t *pattern,
                     float *jsd, float *vhat, float *shat, float *pest, void *stream);
 
+/* Head-pattern sharing (second article, section 5: similar heads share one
+ * sparse pattern; the articles give no rule, so this is the written
+ * convention).  Within each GQA group, in head order, head a joins the class
+ * of the earliest earlier class representative b with JSD(vhat_a, vhat_b) <
+ * eps (natural log, the divergence of the pattern decision); a head that
+ * joins none represents its own class.  Every head of a class then attends to
+ * the union of the class members' block lists for each query block, so every
+ * head keeps at least its own gamma-coverage, and heads of one class walk the
+ * same key blocks in fp_sparse_attn.  Rewrites the lists of a built index in
+ * place (asynchronous on `stream`); eps >= 0 (eps = 0 shares nothing).
+ * Returns FP_ERR_STATE before a build, FP_ERR_ARG for a negative or NaN eps
+ * or more than 110 query heads per KV head. */
+int fp_index_share(fp_index *idx, float eps, void *stream);
+
+/* Compact block lists on the device (first article, section 3.2: compact
+ * job lists).  row_ptr: device int32[Hq*n + 1] receives the CSR row offsets
+ * over rows h*n + r (row_ptr[Hq*n] = nnz); col (device int32[nnz], or NULL
+ * to get only row_ptr) the ascending key blocks of every row.  Both
+ * caller-owned, 4-byte aligned; asynchronous on `stream`.  The attention
+ * kernel itself reads the index's padded per-row lists (row (h, r) at a
+ * fixed offset, written by the selection without a scan); this call
+ * produces the compact form for other consumers. */
+int fp_index_csr(const fp_index *idx, int32_t *row_ptr, int32_t *col, void *stream);
+
+/* Per-(KV head, query block) union lists with head masks (first article,
+ * section 2.2: a KV block loaded once serves the query heads of its GQA
+ * group).  Rows j*n + r for KV head j: grp_ptr device int32[Hkv*n + 1]
+ * (offsets), grp_col device int32[total] the ascending union of the g
+ * query heads' blocks, grp_mask device uint32[total] with bit m set when
+ * query head j*g + m lists that block.  grp_col and grp_mask both NULL to get
+ * only grp_ptr (the total is grp_ptr[Hkv*n]).  g <= 32.  Caller-owned, 4-byte
+ * aligned; asynchronous on `stream`. */
+int fp_index_group_lists(const fp_index *idx, int32_t *grp_ptr, int32_t *grp_col, uint32_t *grp_mask,
+                         void *stream);
+
+/* Synchronises `stream` and copies the class representative of every query
+ * head (absolute head index; h itself when not shared) to HOST cls[Hq]. */
+int fp_index_classes(const fp_index *idx, int32_t *cls, void *stream);
+
+/* Adaptive block size (second article, section 5: block size adjusted to the
+ * complexity of the content; section 4.3: 64, 128, 256; the articles give no
+ * rule, so this is the written convention).  From an index built with
+ * b = 128: k_h = fewest key blocks whose vhat (the exact pooled last-block
+ * attention of head h) sums to at least gamma, taken by descending vhat;
+ * rho = mean over heads of k_h / n.  *b = 64 when rho < 0.1 and S/64 <= 1024
+ * blocks, 256 when rho >= 0.5, else 128; *rho (may be NULL) receives rho.
+ * The counts run on the device; synchronises `stream`.  Returns
+ * FP_ERR_STATE unless idx is built with b = 128. */
+int fp_choose_block_size(const fp_index *idx, float gamma, int *b, float *rho, void *stream);
+
 /* Synchronises `stream`, returns FP_OK or the sticky device error recorded by
  * a kernel on the current device (FP_ERR_TIMEOUT), and clears it. */
 int fp_get_device_error(void *stream);
