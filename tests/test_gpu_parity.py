@@ -269,7 +269,7 @@ def sampled_tiles(w, count, seed):
     return sorted(tiles)
 
 
-@pytest.mark.parametrize("name,ntiles", [("llama3b", 24), ("llama8b", 64), ("llama8b_w8a8", 64)])
+@pytest.mark.parametrize("name,ntiles", [("llama3b", 64), ("llama8b", 64), ("llama8b_w8a8", 64)])
 def test_full_size_layers(fp, name, ntiles):
     w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
