@@ -507,6 +507,20 @@ def run_ours(args, w):
                               "note": "device CSR and per-group union lists of the timed index; the attention "
                                       "reads the padded rows, so neither is part of the step"}
     del rp, col, gp, gc, gm
+    if not w.int8 and not args.no_w8a8 and w.b == 128 and w.S % 256 == 0:
+        # the same layer at b = 256 (two 128-row halves per block share one list)
+        wb = synth.Workload(w.name + "_b256", S=w.S, Hq=w.Hq, Hkv=w.Hkv, d=w.d, b=256, gamma=w.gamma, tau=w.tau,
+                            n_vertical=w.n_vertical, n_topics=w.n_topics, seed=w.seed)
+        Lb = time_layer(fp, wb, qq, kk, v, qs, ks, dt, args, dev, stream, world)
+        msb = max_over_ranks(Lb["total_ms"], dev) / args.steps
+        achb = Lb["attn_flops"] / (Lb["attn_ms"] / 1e3) / 1e12
+        extra["b256"] = {"workload": wb.name, "ms_per_layer": msb, "index_ms": Lb["index_ms"],
+                         "attn_ms": Lb["attn_ms"], "value": world * dense / (msb / 1e3) / 1e12, "unit": UNIT,
+                         "density": Lb["density"], "chunks": Lb["chunks"],
+                         "roofline": {"kernel": "k_sparse_attn", "bound": "tensor", "achieved": achb,
+                                      "peak": peak, "unit": "TFLOP/s", "frac": achb / peak, "peak_source": src},
+                         "clocks": Lb["clocks"], "gpu_launches": KERNELS_PER_STEP * args.steps}
+        Lb["idx"].free()
     if not w.int8 and not args.no_w8a8:
         # the W8A8 variant of the same layer: Q and K quantised per head from these bf16 tensors
         del q, k, qq, kk
