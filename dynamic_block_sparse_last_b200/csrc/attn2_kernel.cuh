@@ -305,6 +305,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(608, 1)
       uint32_t rr[64];
       tmem_ld64(s_tm, rr);
       tmem_ld_wait64(rr);
+      if constexpr (I8) {
+        if (P.cap != nullptr && me.h == P.cap_h && qc == P.cap_qc && kc == P.cap_kc) {
+          int4 *dst = reinterpret_cast<int4 *>(P.cap + (size_t)row * 128 + ch * 64);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            dst[e] = make_int4((int)rr[4 * e], (int)rr[4 * e + 1], (int)rr[4 * e + 2], (int)rr[4 * e + 3]);
+        }
+      }
       float s[64];
 #pragma unroll
       for (int e = 0; e < 64; ++e) s[e] = I8 ? i32_to_f32_small(rr[e]) : __uint_as_float(rr[e]);
@@ -345,8 +353,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(608, 1)
         f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
         pk[e >> 1] = pack_bf16x2(ex2(x0), ex2(x1));
       }
+      uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int e = 0; e < 32; ++e) add_bf16x2_f32(pk[e], r8[(2 * e) & 7], r8[(2 * e + 1) & 7]);
+      for (int e = 0; e < 32; ++e)
+        a2[e & 3] = f2_add(a2[e & 3], f2_pack(__uint_as_float(pk[e] << 16), __uint_as_float(pk[e] & 0xFFFF0000u)));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f2_unpack(a2[e], r8[2 * e], r8[2 * e + 1]);
       const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l = l * alpha + rs;
       m_ref = m_new;

@@ -489,10 +489,13 @@ __global__ void __launch_bounds__(608, 1)
           pk[e >> 1] = pack_bf16x2(ex2(x0), ex2(x1));
         }
       }
-      // row sum of the rounded P: each bf16 added to an fp32 chain as it is
-      // (mixed-precision add), eight chains
+      // row sum of the rounded P, two at a time (packed fp32 add)
+      uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int e = 0; e < 32; ++e) add_bf16x2_f32(pk[e], r8[(2 * e) & 7], r8[(2 * e + 1) & 7]);
+      for (int e = 0; e < 32; ++e)
+        a2[e & 3] = f2_add(a2[e & 3], f2_pack(__uint_as_float(pk[e] << 16), __uint_as_float(pk[e] & 0xFFFF0000u)));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) f2_unpack(a2[e], r8[2 * e], r8[2 * e + 1]);
       const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l = l * alpha + rs;
       m_ref = m_new;

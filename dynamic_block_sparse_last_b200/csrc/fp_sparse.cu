@@ -206,6 +206,12 @@ int set_smem_attrs() {
   if (cudaFuncSetAttribute(k_sparse_attn2<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Attn2Cfg<I8>::kSmem) != cudaSuccess)
     return FP_ERR_CUDA;
+  // the Q pooling runs beside k_score_last on the same SMs: same (largest) shared-memory carveout
+  if (cudaFuncSetAttribute(k_qpool<I8>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
+      cudaFuncSetAttribute(k_score_last<I8>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+    return FP_ERR_CUDA;
   d->attrs[I8] = true;
   return FP_OK;
 }

@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(736, 1)
 // the K block means (ext_kbar) they are read instead of the column sums.
 // ---------------------------------------------------------------------------
 constexpr int kStatCta = 8;
-constexpr int kStatThreads = 256;
+constexpr int kStatThreads = 1024;
 constexpr int kStatMaxOwnParts = 256;   // npart <= 2048
 constexpr int kStatMaxOwnBlocks = 128;  // n <= 1024
 
@@ -449,6 +449,7 @@ __global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads)
   __shared__ float rowM[256], rowL[256];                     // this rank's row partials (shared)
   __shared__ float gM[256], gInvL[256];                      // cluster row statistics
   __shared__ float qpart[128], qb[128];                      // last-block query column sums / mean
+  __shared__ float qgrp[kStatThreads / 128][128];            // per row group, before qpart
   __shared__ float LOp[kStatMaxOwnParts], HIp[kStatMaxOwnParts];
   __shared__ float LOb[kStatMaxOwnBlocks], HIb[kStatMaxOwnBlocks];  // owned blocks (shared)
   __shared__ float vh[kStatMaxOwnBlocks], zc[kStatMaxOwnBlocks];
@@ -469,37 +470,55 @@ __global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads)
     const int G = kStatThreads / b, i = tid % b, j = tid / b;
     float M = -INFINITY, L = 0.f;
     if (i < nlast) {
-      for (int p = p0 + j; p < p1; p += G) {
-        const size_t o = hoff + (size_t)p * b + i;
-        const float m = P.pm[o];
-        if (m == -INFINITY) continue;
-        const float sv = P.plo[o] + P.phi[o];
-        if (m > M) {
-          L = L * ex2(M - m) + sv;
-          M = m;
-        } else {
-          L += sv * ex2(m - M);
+      // four parts' partials in flight, then the running combine in part order
+      for (int p = p0 + j; p < p1; p += 4 * G) {
+        float mv[4], sv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int pp = p + u * G;
+          const size_t o = hoff + (size_t)pp * b + i;
+          const bool in = pp < p1;
+          mv[u] = in ? P.pm[o] : -INFINITY;
+          sv[u] = in ? P.plo[o] + P.phi[o] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float m = mv[u];
+          if (m == -INFINITY) continue;
+          if (m > M) {
+            L = L * ex2(M - m) + sv[u];
+            M = m;
+          } else {
+            L += sv[u] * ex2(m - M);
+          }
         }
       }
     }
     grpM[tid] = M;
     grpL[tid] = L;
-    if (tid < 128) {
+    {
+      // rows r0 .. r1-1 of the last block, column tid % 128, row group tid / 128
       const int r0 = (k * nlast) / kStatCta, r1 = ((k + 1) * nlast) / kStatCta;
-      const size_t base = ((size_t)h * P.ld + (size_t)(n - 1) * b) * 128 + tid;
+      const int c = tid & 127, rg = tid >> 7, RG = kStatThreads / 128;
+      const size_t base = ((size_t)h * P.ld + (size_t)(n - 1) * b) * 128 + c;
       float acc = 0.f;
       if (I8) {
         const int8_t *q8 = reinterpret_cast<const int8_t *>(P.q);
         int ia = 0;
-        for (int r = r0; r < r1; ++r) ia += q8[base + (size_t)r * 128];
+        for (int r = r0 + rg; r < r1; r += RG) ia += q8[base + (size_t)r * 128];
         acc = (float)ia;
       } else {
         const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(P.q);
-        for (int r = r0; r < r1; ++r) acc += __bfloat162float(qh[base + (size_t)r * 128]);
+        for (int r = r0 + rg; r < r1; r += RG) acc += __bfloat162float(qh[base + (size_t)r * 128]);
       }
-      qpart[tid] = acc;
+      qgrp[rg][c] = acc;
     }
     __syncthreads();
+    if (tid < 128) {
+      float a = 0.f;
+      for (int rg = 0; rg < kStatThreads / 128; ++rg) a += qgrp[rg][tid];
+      qpart[tid] = a;
+    }
     if (tid < b) {
       float Mi = -INFINITY, Li = 0.f;
       for (int jj = 0; jj < G; ++jj) {
@@ -539,13 +558,22 @@ __global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads)
   // ---- 2. part masses (warp per part, lanes over rows), block masses, kbar and logits
   for (int p = p0 + warp; p < p1; p += nwarp) {
     float a = 0.f, c = 0.f;
-    for (int i = lane; i < b; i += 32) {
-      if (i >= nlast) break;
+    float mv[8], lv[8], hv[8];  // the lane's rows i = lane + 32 t of the part (b <= 256)
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int i = lane + 32 * t;
+      const bool in = i < b && i < nlast;
       const size_t o = hoff + (size_t)p * b + i;
-      const float m = P.pm[o];
-      const float w = (m == -INFINITY) ? 0.f : ex2(m - gM[i]) * gInvL[i];
-      a += P.plo[o] * w;
-      c += P.phi[o] * w;
+      mv[t] = in ? P.pm[o] : -INFINITY;
+      lv[t] = in ? P.plo[o] : 0.f;
+      hv[t] = in ? P.phi[o] : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int i = lane + 32 * t;
+      const float w = (mv[t] == -INFINITY) ? 0.f : ex2(mv[t] - gM[i]) * gInvL[i];
+      a += lv[t] * w;
+      c += hv[t] * w;
     }
 #pragma unroll
     for (int sft = 16; sft > 0; sft >>= 1) {
@@ -884,7 +912,8 @@ __global__ void __launch_bounds__(256)
 // ---------------------------------------------------------------------------
 // k_cut: one warp per (head, query block r), heavy rows first; block 256.
 // Scores over c <= r:  VS: w_c = vhat[c] + shat[r - c];  QA: w_c = exp(z_c -
-// max); normalised to sum 1.  The diagonal is kept; the others are kept in
+// max) (as 2^((z_c - max) log2 e)); normalised to sum 1 (times the reciprocal
+// of the sum).  The diagonal is kept; the others are kept in
 // order of descending score (ties: lower index) while the kept sum is below
 // gamma.  The cut is found by bisection on the fp32 bit pattern of the
 // scores (monotone for positive floats), between the smallest and the
@@ -921,7 +950,7 @@ __device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const floa
     }
     mx = redux_max_f32(mx);
 #pragma unroll
-    for (int i = 0; i < NL; ++i) v[i] = (lane + 32 * i <= r) ? expf(v[i] - mx) : 0.f;
+    for (int i = 0; i < NL; ++i) v[i] = (lane + 32 * i <= r) ? ex2((v[i] - mx) * kLog2e) : 0.f;
   } else {
     const float *vh = vhat + (size_t)h * n, *sh = shat + (size_t)h * n;
 #pragma unroll
@@ -937,8 +966,9 @@ __device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const floa
   for (int i = 0; i < NL; ++i) zs += v[i];
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, s);
+  const float inv_zs = __frcp_rn(zs);
 #pragma unroll
-  for (int i = 0; i < NL; ++i) v[i] = v[i] / zs;
+  for (int i = 0; i < NL; ++i) v[i] = v[i] * inv_zs;
   // diagonal score w_r from lane r % 32, slot r / 32; then that slot is zeroed
   float wr_l = 0.f;
 #pragma unroll
