@@ -206,6 +206,8 @@ int set_smem_attrs() {
   if (cudaFuncSetAttribute(k_sparse_attn2<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            Attn2Cfg<I8>::kSmem) != cudaSuccess)
     return FP_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_qa_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, kLgSmem) != cudaSuccess)
+    return FP_ERR_CUDA;
   // the Q pooling runs beside k_score_last on the same SMs: same (largest) shared-memory carveout
   if (cudaFuncSetAttribute(k_qpool<I8>, cudaFuncAttributePreferredSharedMemoryCarveout,
                            cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
@@ -327,8 +329,8 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   const float *kbar = ext_kbar ? ext_kbar : I->kbar;
   if (!ext_qbar && cudaStreamWaitEvent(st, I->ev_join, 0) != cudaSuccess) return FP_ERR_CUDA;
   const int nt = (I->n + kLgTile - 1) / kLgTile;
-  k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, qbar, kbar, I->g, I->n,
-                                                               inv_sqrt_d, I->zlog);
+  k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 128, kLgSmem, st>>>(I->pattern, qbar, kbar, I->g, I->n,
+                                                                     inv_sqrt_d, err, I->zlog);
   if ((rc = launch_status())) return rc;
   k_cut<<<(I->Hq * I->n + 7) / 8, 256, 0, st>>>(I->pattern, I->vhat, I->shat, I->zlog, I->Hq, I->n, gamma,
                                                I->counts, I->cols);
