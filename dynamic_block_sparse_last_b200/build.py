@@ -11,7 +11,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRCS = [os.path.join(PKG, "csrc", f) for f in ("fp_sparse.cu", "fp_prefill.cpp")]
 DEPS = SRCS + [os.path.join(PKG, "csrc", f) for f in ("ptx.cuh", "index_kernels.cuh", "attn_kernel.cuh",
-                                                      "rope_pool.cuh", "share_kernels.cuh", "attn2_kernel.cuh")] \
+                                                      "rope_pool.cuh", "share_kernels.cuh")] \
     + [os.path.join(ROOT, "include", f) for f in ("fp_sparse.h", "fp_prefill.h")]
 LIB = os.path.join(PKG, "_lib", "libfpsparse.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc" if os.path.exists("/usr/local/cuda/bin/nvcc") else "nvcc")

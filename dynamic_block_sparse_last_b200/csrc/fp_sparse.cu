@@ -14,7 +14,6 @@
 #include <vector>
 
 #include "attn_kernel.cuh"
-#include "attn2_kernel.cuh"
 #include "fp_sparse.h"
 #include "index_kernels.cuh"
 #include "rope_pool.cuh"
@@ -144,16 +143,16 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D map over a [rows][128] tensor: boxes of box_rows rows x 128 bytes
+// 2-D map over a [rows][128] tensor: boxes of 128 rows x 128 bytes
 // (64 bf16 or 128 int8 columns), 128-byte swizzle.  For H heads of S rows
 // spaced ld rows apart the map covers (H-1)*ld + S rows from the first head's
 // first row, so no box reads past the last head's last row.
-bool make_map(CUtensorMap *m, const void *ptr, bool i8, uint64_t rows, uint32_t box_rows = 128) {
+bool make_map(CUtensorMap *m, const void *ptr, bool i8, uint64_t rows) {
   auto enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {128, rows};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(128 * (i8 ? 1 : 2))};
-  const cuuint32_t box[2] = {i8 ? 128u : 64u, box_rows};
+  const cuuint32_t box[2] = {i8 ? 128u : 64u, 128u};
   const cuuint32_t estr[2] = {1u, 1u};
   CUresult r = enc(m, i8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -202,11 +201,6 @@ int set_smem_attrs() {
     return FP_ERR_CUDA;
   if (cudaFuncSetAttribute(k_sparse_attn<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            AttnCfg<I8>::kSmem) != cudaSuccess)
-    return FP_ERR_CUDA;
-  if (cudaFuncSetAttribute(k_sparse_attn2<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           Attn2Cfg<I8>::kSmem) != cudaSuccess)
-    return FP_ERR_CUDA;
-  if (cudaFuncSetAttribute(k_qa_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, kLgSmem) != cudaSuccess)
     return FP_ERR_CUDA;
   // the Q pooling runs beside k_score_last on the same SMs: same (largest) shared-memory carveout
   if (cudaFuncSetAttribute(k_qpool<I8>, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -319,7 +313,7 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   if ((rc = launch_score<I8>(J, err, st))) return rc;
   if (!qbar) {
     if (cudaStreamWaitEvent(I->own, I->ev_fork, 0) != cudaSuccess) return FP_ERR_CUDA;
-    k_qpool<I8><<<dim3(I->n, I->Hq), 256, 0, I->own>>>(q, q_scale, I->S, I->ld, I->b, I->n, I->qbar);
+    k_qpool<I8><<<dim3(I->n, I->Hq), 128, 0, I->own>>>(q, q_scale, I->S, I->ld, I->b, I->n, I->qbar);
     if ((rc = launch_status())) return rc;
     if (cudaEventRecord(I->ev_join, I->own) != cudaSuccess) return FP_ERR_CUDA;
     qbar = I->qbar;
@@ -329,8 +323,8 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   const float *kbar = ext_kbar ? ext_kbar : I->kbar;
   if (!ext_qbar && cudaStreamWaitEvent(st, I->ev_join, 0) != cudaSuccess) return FP_ERR_CUDA;
   const int nt = (I->n + kLgTile - 1) / kLgTile;
-  k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 128, kLgSmem, st>>>(I->pattern, qbar, kbar, I->g, I->n,
-                                                                     inv_sqrt_d, err, I->zlog);
+  k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, qbar, kbar, I->g, I->n,
+                                                               inv_sqrt_d, I->zlog);
   if ((rc = launch_status())) return rc;
   k_cut<<<(I->Hq * I->n + 7) / 8, 256, 0, st>>>(I->pattern, I->vhat, I->shat, I->zlog, I->Hq, I->n, gamma,
                                                I->counts, I->cols);
@@ -365,16 +359,8 @@ int attn_impl(const void *q, const void *k, const void *v, const float *q_scale,
     ap.cap = c.attn;
     ap.cap_h = c.a_h; ap.cap_qc = c.a_qc; ap.cap_kc = c.a_kc;
   }
-  if (I->b == 256) {
-    // CTA pairs (M = 256 MMAs across two SMs): each CTA loads 64-row halves of the K chunks
-    CUtensorMap tkh;
-    if (!make_map(&tkh, k, I8, map_rows(I->Hkv, I->ld, I->S), 64)) return FP_ERR_CUDA;
-    const unsigned grid = 2u * (unsigned)attn2_units(I->Hq, I->Hkv, I->S);
-    k_sparse_attn2<I8><<<grid, Attn2Cfg<I8>::kThreads, Attn2Cfg<I8>::kSmem, st>>>(tq, tkh, tv, ap);
-  } else {
-    const unsigned grid = (unsigned)attn_pairs(I->Hq, I->Hkv, I->S, I->b);
-    k_sparse_attn<I8><<<grid, AttnCfg<I8>::kThreads, AttnCfg<I8>::kSmem, st>>>(tq, tk, tv, ap);
-  }
+  const unsigned grid = (unsigned)attn_pairs(I->Hq, I->Hkv, I->S, I->b);
+  k_sparse_attn<I8><<<grid, AttnCfg<I8>::kThreads, AttnCfg<I8>::kSmem, st>>>(tq, tk, tv, ap);
   if ((rc = launch_status())) return rc;
   return cudaEventRecord(I->last_use, st) == cudaSuccess ? FP_OK : FP_ERR_CUDA;
 }

@@ -708,14 +708,15 @@ __global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads)
 }
 
 // ---------------------------------------------------------------------------
-// k_qpool: grid (n, Hq), block 256, at most 48 registers per thread (one CTA
-// fits beside a k_score_last CTA on the same SM, so the two overlap: the
-// score kernel is bound by its exponentials and leaves HBM mostly idle).
-// qbar[h][r][t] = mean of the Q rows of block r (b rows, or S - (n-1)b for a
-// partial last block), for every head: which heads are query-aware is known
-// only after the scores.  Thread (c8 = tid & 15, rr = tid >> 4) owns columns
-// 8 c8 .. 8 c8 + 7 and rows rr, rr + 16, ...; the block kPoolAhead blocks
-// ahead is prefetched into L2 (bulk prefetch, no registers held).
+// k_qpool: grid (n, Hq), block 128, at most 64 registers per thread: one warp
+// per SM sub-partition, so a CTA fits beside a k_score_last CTA (6 warps x 72
+// registers per sub-partition) and the two overlap; the score kernel is bound
+// by its exponentials and leaves HBM mostly idle.  qbar[h][r][t] = mean of
+// the Q rows of block r (b rows, or S - (n-1)b for a partial last block), for
+// every head: which heads are query-aware is known only after the scores.
+// Eight rows' 16-byte loads per thread are in flight before they are added;
+// the block kPoolAhead blocks ahead is prefetched into L2 (bulk prefetch, no
+// registers held).
 // ---------------------------------------------------------------------------
 constexpr int kPoolAhead = 4;
 
@@ -725,11 +726,11 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
 }
 
 template <bool I8>
-__global__ void __maxnreg__(48)
+__global__ void __maxnreg__(64)
     k_qpool(const void *__restrict__ q, const float *__restrict__ q_scale, int S, int ld, int b, int n,
             float *__restrict__ qbar) {
   const int r = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-  __shared__ float red[16][128];
+  __shared__ float red[4][128];
   const size_t row0 = (size_t)h * ld + (size_t)r * b;
   const int rows = min(b, S - r * b);
   const int esz = I8 ? 1 : 2;
@@ -740,19 +741,26 @@ __global__ void __maxnreg__(48)
     prefetch_l2(reinterpret_cast<const char *>(q) + ((size_t)h * ld + (size_t)ra * b) * 128 * esz,
                 (uint32_t)arows * 128u * esz);
   }
+  const int warp = tid >> 5, lane = tid & 31;
   if (I8) {
-    // 8 threads per 128-byte row, 32 rows per pass; thread owns 16 columns
+    // 8 threads per 128-byte row, 16 rows per pass; thread owns 16 columns
     const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
     const int c16 = tid & 7, rr = tid >> 3;
     int acc[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) acc[e] = 0;
-#pragma unroll 2
-    for (int p = rr; p < rows; p += 32) {
-      const int4 v = *reinterpret_cast<const int4 *>(q8 + (row0 + p) * 128 + c16 * 16);
-      const int w[4] = {v.x, v.y, v.z, v.w};
+    for (int p = rr; p < rows; p += 16 * 8) {
+      int4 v[8];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) acc[e] += (int)(int8_t)((w[e >> 2] >> (8 * (e & 3))) & 0xff);
+      for (int j = 0; j < 8; ++j)
+        v[j] = (p + 16 * j < rows) ? *reinterpret_cast<const int4 *>(q8 + (row0 + p + 16 * j) * 128 + c16 * 16)
+                                   : make_int4(0, 0, 0, 0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] += (int)(int8_t)((w[e >> 2] >> (8 * (e & 3))) & 0xff);
+      }
     }
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
@@ -761,33 +769,29 @@ __global__ void __maxnreg__(48)
       a += __shfl_xor_sync(0xffffffffu, a, 16);
       acc[e] = a;
     }
-    const int warp = tid >> 5, lane = tid & 31;
     if (lane < 8) {
 #pragma unroll
       for (int e = 0; e < 16; ++e) red[warp][lane * 16 + e] = (float)acc[e];
     }
     __syncthreads();
-    if (tid < 128) {
-      float s2 = 0.f;
-      for (int w = 0; w < 8; ++w) s2 += red[w][tid];
-      qbar[((size_t)h * n + r) * 128 + tid] = s2 * q_scale[h] / (float)rows;
-    }
+    float s2 = 0.f;
+    for (int w = 0; w < 4; ++w) s2 += red[w][tid];
+    qbar[((size_t)h * n + r) * 128 + tid] = s2 * q_scale[h] / (float)rows;
   } else {
-    // 16 threads per 256-byte row, 16 rows per pass; thread owns 8 columns;
-    // four rows' loads in flight before they are added
+    // 16 threads per 256-byte row, 8 rows per pass; thread owns 8 columns
     const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(q);
     const int c8 = tid & 15, rr = tid >> 4;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-    for (int p = rr; p < rows; p += 64) {
-      uint4 v[4];
+    for (int p = rr; p < rows; p += 8 * 8) {
+      uint4 v[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        v[j] = (p + 16 * j < rows) ? *reinterpret_cast<const uint4 *>(qh + (row0 + p + 16 * j) * 128 + c8 * 8)
-                                   : make_uint4(0u, 0u, 0u, 0u);
+      for (int j = 0; j < 8; ++j)
+        v[j] = (p + 8 * j < rows) ? *reinterpret_cast<const uint4 *>(qh + (row0 + p + 8 * j) * 128 + c8 * 8)
+                                  : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 8; ++j) {
         const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -798,48 +802,38 @@ __global__ void __maxnreg__(48)
     }
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
-    const int warp = tid >> 5, lane = tid & 31;
     if (lane < 16) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
     }
     __syncthreads();
-    if (tid < 128) {
-      float s2 = 0.f;
-      for (int w = 0; w < 8; ++w) s2 += red[w][tid];
-      qbar[((size_t)h * n + r) * 128 + tid] = s2 / (float)rows;
-    }
+    float s2 = 0.f;
+    for (int w = 0; w < 4; ++w) s2 += red[w][tid];
+    qbar[((size_t)h * n + r) * 128 + tid] = s2 / (float)rows;
   }
 }
 
 // ---------------------------------------------------------------------------
-// k_qa_logits: grid (nt(nt+1)/2, Hq) with nt = ceil(n/128), block 128.  For
+// k_qa_logits: grid (nt(nt+1)/2, Hq) with nt = ceil(n/64), block 256.  For
 // query-aware heads only (others exit): the lower triangle of
 // Z = qbar kbar^T / sqrt(d), z[h][r][c] for c <= r, in the padded triangular
-// layout (row r at h*n(n+1)/2 + r(r+1)/2), one 128 x 128 tile per CTA on the
-// tensor cores.  Every fp32 operand is split as x = x_hi + x_lo with x_hi =
-// tf32(x) and x_lo = tf32(x - x_hi); the tile accumulates hi.hi + hi.lo +
-// lo.hi in fp32 in tensor memory (the dropped lo.lo term and the rounding of
-// x_lo are below 2^-21 of each product, the order of fp32 rounding).  d is
-// staged 32 at a time: thread t converts row t of the q-bar tile and of the
-// k-bar tile into four 128-byte-swizzled K-major slabs (q_hi, q_lo, k_hi,
-// k_lo), thread 0 issues the 12 MMAs (M = N = 128, K = 8 each) and commits;
-// the slabs are refilled once those MMAs have completed.  Epilogue: thread t
-// reads row t of the accumulator from tensor memory.
+// layout (row r at h*n(n+1)/2 + r(r+1)/2).  Tiled fp32 product: 64 x 64
+// output tile per CTA, 4 x 4 outputs per thread held as column pairs and
+// updated with packed fp32 FMAs; d is staged through shared memory 32 at a
+// time, double-buffered (the next slice is loaded into registers while the
+// current one is multiplied).
 // ---------------------------------------------------------------------------
-constexpr int kLgTile = 128;
-constexpr int kLgSmem = 4 * 16384 + 1024;
+constexpr int kLgTile = 64;
+constexpr int kLgK = 32;
+constexpr int kLgStride = kLgTile + 4;  // float4-aligned rows
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
     k_qa_logits(const int *__restrict__ pattern, const float *__restrict__ qbar,
-                const float *__restrict__ kbar, int g, int n, float inv_sqrt_d, int *__restrict__ err,
-                float *__restrict__ z) {
+                const float *__restrict__ kbar, int g, int n, float inv_sqrt_d, float *__restrict__ z) {
   const int h = blockIdx.y;
   if (pattern[h] != 1) return;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_mma;
-  __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_sh;
+  __shared__ __align__(16) float As[2][kLgK][kLgStride];  // [buffer][k][row]
+  __shared__ __align__(16) float Bs[2][kLgK][kLgStride];  // [buffer][k][col]
   // lower-triangular tile (tr, tc), tc <= tr, from the linear index
   const int x = blockIdx.x;
   int tr = (int)((sqrtf(8.f * (float)x + 1.f) - 1.f) * 0.5f);
@@ -847,94 +841,72 @@ __global__ void __launch_bounds__(128)
   while (tr * (tr + 1) / 2 > x) --tr;
   const int tc = x - tr * (tr + 1) / 2;
   const int kvh = h / g;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
-  uint8_t *const gbase = smem_raw + (base - smem_u32(smem_raw));
-  if (tid == 0) {
-    abort_sh = 0;
-    mbar_init(smem_u32(&bar_mma), 1);
-    fence_mbar_init();
-  }
-  if (warp == 0) {
-    tmem_alloc(smem_u32(&tmem_base_sh), 128);
-    tmem_relinquish();
-  }
-  tc_fence_before();
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int row0 = tr * kLgTile, col0 = tc * kLgTile;
+  const float *qh = qbar + (size_t)h * n * 128;
+  const float *kh = kbar + (size_t)kvh * n * 128;
+  // this thread's share of a k-slice: rows rr0, rr0 + 32 of q-bar and k-bar, 4 consecutive k
+  const int rr0 = tid >> 3, k4 = (tid & 7) * 4;
+  float4 qa[2], kb[2];
+  auto load = [&](int k0) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int rr = rr0 + 32 * u;
+      qa[u] = (row0 + rr < n) ? *reinterpret_cast<const float4 *>(qh + (size_t)(row0 + rr) * 128 + k0 + k4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      kb[u] = (col0 + rr < n) ? *reinterpret_cast<const float4 *>(kh + (size_t)(col0 + rr) * 128 + k0 + k4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  auto store = [&](int buf) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int rr = rr0 + 32 * u;
+      As[buf][k4 + 0][rr] = qa[u].x; As[buf][k4 + 1][rr] = qa[u].y;
+      As[buf][k4 + 2][rr] = qa[u].z; As[buf][k4 + 3][rr] = qa[u].w;
+      Bs[buf][k4 + 0][rr] = kb[u].x; Bs[buf][k4 + 1][rr] = kb[u].y;
+      Bs[buf][k4 + 2][rr] = kb[u].z; Bs[buf][k4 + 3][rr] = kb[u].w;
+    }
+  };
+  uint64_t acc[4][2];  // rows ty*4 + a, column pairs tx*4 + 2p, +1
+#pragma unroll
+  for (int a = 0; a < 4; ++a) acc[a][0] = acc[a][1] = 0ull;
+  load(0);
+  store(0);
   __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = tmem_base_sh;
-  volatile int *abort_flag = &abort_sh;
-  const int rq = tr * kLgTile + tid, rk = tc * kLgTile + tid;  // this thread's q-bar and k-bar rows
-  const float *qrow = qbar + ((size_t)h * n + rq) * 128;
-  const float *krow = kbar + ((size_t)kvh * n + rk) * 128;
-  const uint32_t idesc = idesc_tf32(128, 128);
-  const uint32_t swz = (uint32_t)((tid >> 3) * 1024 + (tid & 7) * 128);
-  bool ok = true;
-  for (int qd = 0; qd < 4 && ok; ++qd) {
-    if (qd > 0) ok = mbar_wait(smem_u32(&bar_mma), (qd - 1) & 1, abort_flag, err);
-    if (!ok) break;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const float4 qv = rq < n ? *reinterpret_cast<const float4 *>(qrow + qd * 32 + 4 * j)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float4 kv = rk < n ? *reinterpret_cast<const float4 *>(krow + qd * 32 + 4 * j)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float qa[4] = {qv.x, qv.y, qv.z, qv.w}, ka[4] = {kv.x, kv.y, kv.z, kv.w};
-      uint32_t qh[4], ql[4], kh[4], kl[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        qh[e] = tf32_rna(qa[e]);
-        ql[e] = tf32_rna(qa[e] - __uint_as_float(qh[e]));
-        kh[e] = tf32_rna(ka[e]);
-        kl[e] = tf32_rna(ka[e] - __uint_as_float(kh[e]));
-      }
-      const uint32_t off = swz + (uint32_t)(((j ^ (tid & 7)) << 4));
-      *reinterpret_cast<uint4 *>(gbase + 0 * 16384 + off) = make_uint4(qh[0], qh[1], qh[2], qh[3]);
-      *reinterpret_cast<uint4 *>(gbase + 1 * 16384 + off) = make_uint4(ql[0], ql[1], ql[2], ql[3]);
-      *reinterpret_cast<uint4 *>(gbase + 2 * 16384 + off) = make_uint4(kh[0], kh[1], kh[2], kh[3]);
-      *reinterpret_cast<uint4 *>(gbase + 3 * 16384 + off) = make_uint4(kl[0], kl[1], kl[2], kl[3]);
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t a_hi = umma_desc_sw128(base + 0 * 16384 + kk * 32, 16, 1024);
-        const uint64_t a_lo = umma_desc_sw128(base + 1 * 16384 + kk * 32, 16, 1024);
-        const uint64_t b_hi = umma_desc_sw128(base + 2 * 16384 + kk * 32, 16, 1024);
-        const uint64_t b_lo = umma_desc_sw128(base + 3 * 16384 + kk * 32, 16, 1024);
-        mma_tf32_ss(tmem, a_hi, b_hi, idesc, (qd > 0 || kk > 0));
-        mma_tf32_ss(tmem, a_hi, b_lo, idesc, 1);
-        mma_tf32_ss(tmem, a_lo, b_hi, idesc, 1);
-      }
-      tc_commit(smem_u32(&bar_mma));
-    }
-    __syncwarp();
-  }
-  if (ok && mbar_wait(smem_u32(&bar_mma), 1, abort_flag, err)) {
-    tc_fence_after();
-    float *zh = z + (size_t)h * ((size_t)n * (n + 1) / 2);
-    const size_t roff = (size_t)rq * (rq + 1) / 2;
 #pragma unroll 1
-    for (int q4 = 0; q4 < 4; ++q4) {
-      uint32_t v[32];
-      tmem_ld32(tmem + (((uint32_t)(warp * 32)) << 16) + q4 * 32, v);
-      tmem_ld_wait(v);
-      if (rq < n) {
+  for (int kt = 0; kt < 128 / kLgK; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < 128 / kLgK) load((kt + 1) * kLgK);
+#pragma unroll 8
+    for (int k = 0; k < kLgK; ++k) {
+      const float4 a4 = *reinterpret_cast<const float4 *>(&As[buf][k][ty * 4]);
+      const float4 b4 = *reinterpret_cast<const float4 *>(&Bs[buf][k][tx * 4]);
+      const uint64_t b01 = f2_pack(b4.x, b4.y), b23 = f2_pack(b4.z, b4.w);
+      const float av[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c = tc * kLgTile + q4 * 32 + e;
-          if (c <= rq) zh[roff + c] = __uint_as_float(v[e]) * inv_sqrt_d;
-        }
+      for (int a = 0; a < 4; ++a) {
+        const uint64_t aa = f2_pack(av[a], av[a]);
+        acc[a][0] = f2_fma(aa, b01, acc[a][0]);
+        acc[a][1] = f2_fma(aa, b23, acc[a][1]);
       }
     }
+    if (kt + 1 < 128 / kLgK) store(buf ^ 1);
+    __syncthreads();
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 128);
+  float *zh = z + (size_t)h * ((size_t)n * (n + 1) / 2);
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    const int r = row0 + ty * 4 + a;
+    if (r >= n) continue;
+    float v[4];
+    f2_unpack(acc[a][0], v[0], v[1]);
+    f2_unpack(acc[a][1], v[2], v[3]);
+#pragma unroll
+    for (int b2 = 0; b2 < 4; ++b2) {
+      const int c = col0 + tx * 4 + b2;
+      if (c <= r) zh[(size_t)r * (r + 1) / 2 + c] = v[b2] * inv_sqrt_d;
+    }
   }
 }
 
