@@ -426,7 +426,7 @@ __global__ void __launch_bounds__(608, 1)
       }
       float s[64];
 #pragma unroll
-      for (int e = 0; e < 64; ++e) s[e] = I8 ? i32_to_f32_small(rr[e]) : __uint_as_float(rr[e]);
+      for (int e = 0; e < 64; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
       if (P.b < 128) {
         // the warp's quadrant is one (query block, key block 2kc + ch) pair
         const int kb = 2 * kc + ch;
@@ -489,13 +489,10 @@ __global__ void __launch_bounds__(608, 1)
           pk[e >> 1] = pack_bf16x2(ex2(x0), ex2(x1));
         }
       }
-      // row sum of the rounded P, two at a time (packed fp32 add)
-      uint64_t a2[4] = {0ull, 0ull, 0ull, 0ull};
+      // row sum of the rounded P: each bf16 added to an fp32 chain as it is
+      // (mixed-precision add, no unpacking), eight chains
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        a2[e & 3] = f2_add(a2[e & 3], f2_pack(__uint_as_float(pk[e] << 16), __uint_as_float(pk[e] & 0xFFFF0000u)));
-#pragma unroll
-      for (int e = 0; e < 4; ++e) f2_unpack(a2[e], r8[2 * e], r8[2 * e + 1]);
+      for (int e = 0; e < 32; ++e) add_bf16x2_f32(pk[e], r8[(2 * e) & 7], r8[(2 * e + 1) & 7]);
       const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l = l * alpha + rs;
       m_ref = m_new;

@@ -34,9 +34,10 @@ struct fp_index {
   void *slab;
   size_t slab_bytes;
   bool slab_pooled;        // slab from the stream-ordered allocator (else cudaMalloc)
-  cudaStream_t own;        // the index's own stream: allocation and release of the slab
+  cudaStream_t own;        // the index's own stream: allocation and release of the slab, Q pooling
+  cudaStream_t own_hi;     // highest-priority stream of the index: the score kernel
   cudaEvent_t last_use;    // recorded on the caller's stream at the end of every build / attention call
-  cudaEvent_t ev_fork, ev_join;  // Q pooling on `own` beside the score kernel on the caller's stream
+  cudaEvent_t ev_fork, ev_join, ev_score;  // fork before the pass; Q pooling done; scores done
   float *pm, *plo, *phi;   // [Hq][npart][b]
   float *ksum;             // [Hkv][npart][128]
   float *kbar;             // [Hkv][n][128]
@@ -306,17 +307,24 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   J.ext_kbar = ext_kbar;
   // Q block means of every head on the index's own stream, beside the score
   // kernel (which is bound by its exponentials and leaves HBM mostly idle).
-  // The fork point precedes the score kernel; the pooling kernel is queued
-  // after it, so the score kernel's CTAs are dispatched first.
+  // Both start from one fork point on the caller's stream; the score kernel
+  // runs on the index's highest-priority stream, so its CTAs (one per SM) are
+  // dispatched before the many small pooling CTAs, which then fill the room
+  // left beside them.
   const float *qbar = ext_qbar;
-  if (!qbar && cudaEventRecord(I->ev_fork, st) != cudaSuccess) return FP_ERR_CUDA;
-  if ((rc = launch_score<I8>(J, err, st))) return rc;
   if (!qbar) {
-    if (cudaStreamWaitEvent(I->own, I->ev_fork, 0) != cudaSuccess) return FP_ERR_CUDA;
+    if (cudaEventRecord(I->ev_fork, st) != cudaSuccess || cudaStreamWaitEvent(I->own_hi, I->ev_fork, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(I->own, I->ev_fork, 0) != cudaSuccess)
+      return FP_ERR_CUDA;
+    if ((rc = launch_score<I8>(J, err, I->own_hi))) return rc;
+    if (cudaEventRecord(I->ev_score, I->own_hi) != cudaSuccess) return FP_ERR_CUDA;
     k_qpool<I8><<<dim3(I->n, I->Hq), 128, 0, I->own>>>(q, q_scale, I->S, I->ld, I->b, I->n, I->qbar);
     if ((rc = launch_status())) return rc;
-    if (cudaEventRecord(I->ev_join, I->own) != cudaSuccess) return FP_ERR_CUDA;
+    if (cudaEventRecord(I->ev_join, I->own) != cudaSuccess || cudaStreamWaitEvent(st, I->ev_score, 0) != cudaSuccess)
+      return FP_ERR_CUDA;
     qbar = I->qbar;
+  } else if ((rc = launch_score<I8>(J, err, st))) {
+    return rc;
   }
   if ((rc = launch_head_stats<I8>(J, st))) return rc;
   const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
@@ -408,7 +416,13 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
     free(I);
     return FP_ERR_CUDA;
   }
-  if (cudaEventCreateWithFlags(&I->ev_join, cudaEventDisableTiming) != cudaSuccess) {
+  int prio_lo = 0, prio_hi = 0;
+  cudaDeviceGetStreamPriorityRange(&prio_lo, &prio_hi);
+  if (cudaEventCreateWithFlags(&I->ev_join, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&I->ev_score, cudaEventDisableTiming) != cudaSuccess ||
+      cudaStreamCreateWithPriority(&I->own_hi, cudaStreamNonBlocking, prio_hi) != cudaSuccess) {
+    if (I->ev_join) cudaEventDestroy(I->ev_join);
+    if (I->ev_score) cudaEventDestroy(I->ev_score);
     cudaEventDestroy(I->ev_fork);
     cudaEventDestroy(I->last_use);
     cudaStreamDestroy(I->own);
@@ -423,6 +437,8 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
     cudaGetLastError();
     I->slab = nullptr;
     if (cudaMalloc(&I->slab, need) != cudaSuccess) {
+      cudaStreamDestroy(I->own_hi);
+      cudaEventDestroy(I->ev_score);
       cudaEventDestroy(I->ev_join);
       cudaEventDestroy(I->ev_fork);
       cudaEventDestroy(I->last_use);
@@ -475,9 +491,11 @@ void fp_index_free(fp_index *I) {
     cudaEventSynchronize(I->last_use);
     cudaFree(I->slab);
   }
+  cudaEventDestroy(I->ev_score);
   cudaEventDestroy(I->ev_join);
   cudaEventDestroy(I->ev_fork);
   cudaEventDestroy(I->last_use);
+  cudaStreamDestroy(I->own_hi);
   cudaStreamDestroy(I->own);  // returns at once; the stream's pending free still completes
   if (prev >= 0) cudaSetDevice(prev);
   free(I);

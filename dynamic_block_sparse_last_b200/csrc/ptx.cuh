@@ -350,6 +350,15 @@ __device__ __forceinline__ float i32_to_f32_small(uint32_t x) {
   return __uint_as_float(x + 0x4B400000u) - 12582912.f;
 }
 
+// a0 += float(low bf16 of pk), a1 += float(high bf16 of pk): mixed-precision
+// adds (the bf16 operand is widened exactly), no unpacking instructions.
+__device__ __forceinline__ void add_bf16x2_f32(uint32_t pk, float &a0, float &a1) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(pk));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t *>(&v);
