@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(736, 1)
 // the K block means (ext_kbar) they are read instead of the column sums.
 // ---------------------------------------------------------------------------
 constexpr int kStatCta = 8;
-constexpr int kStatThreads = 1024;
+constexpr int kStatThreads = 512;  // two CTAs per SM: 256 clustered CTAs (32 heads) run in one wave
 constexpr int kStatMaxOwnParts = 256;   // npart <= 2048
 constexpr int kStatMaxOwnBlocks = 128;  // n <= 1024
 
@@ -441,7 +441,7 @@ struct HeadStatsParams {
 __device__ __forceinline__ int stat_block0(int k, int n) { return (k * n) / kStatCta; }
 
 template <bool I8>
-__global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads)
+__global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads, 2)
     k_head_stats(HeadStatsParams P) {
   namespace cg = cooperative_groups;
   cg::cluster_group cl = cg::this_cluster();
@@ -708,15 +708,17 @@ __global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads)
 }
 
 // ---------------------------------------------------------------------------
-// k_qpool: grid (n, Hq), block 128, at most 64 registers per thread: one warp
-// per SM sub-partition, so a CTA fits beside a k_score_last CTA (6 warps x 72
-// registers per sub-partition) and the two overlap; the score kernel is bound
-// by its exponentials and leaves HBM mostly idle.  qbar[h][r][t] = mean of
-// the Q rows of block r (b rows, or S - (n-1)b for a partial last block), for
+// k_qpool: grid (n, Hq), block 128, at most 64 registers per thread and no
+// shared memory: one warp per SM sub-partition, so a CTA fits beside a
+// k_score_last CTA (6 warps x 72 registers per sub-partition, ~198 KB of
+// shared memory) and the two overlap; the score kernel is bound by its
+// exponentials and leaves HBM mostly idle.  qbar[h][r][t] = mean of the Q
+// rows of block r (b rows, or S - (n-1)b for a partial last block), for
 // every head: which heads are query-aware is known only after the scores.
-// Eight rows' 16-byte loads per thread are in flight before they are added;
-// the block kPoolAhead blocks ahead is prefetched into L2 (bulk prefetch, no
-// registers held).
+// Warp w owns columns 32w .. 32w+31; lane (c = lane & 3, rr = lane >> 2)
+// loads 16 bytes of rows rr, rr + 8, ..., eight rows' loads in flight, and
+// the rows are summed across lanes with shuffles.  The block kPoolAhead
+// blocks ahead is prefetched into L2 (bulk prefetch, no registers held).
 // ---------------------------------------------------------------------------
 constexpr int kPoolAhead = 4;
 
@@ -730,7 +732,6 @@ __global__ void __maxnreg__(64)
     k_qpool(const void *__restrict__ q, const float *__restrict__ q_scale, int S, int ld, int b, int n,
             float *__restrict__ qbar) {
   const int r = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
-  __shared__ float red[4][128];
   const size_t row0 = (size_t)h * ld + (size_t)r * b;
   const int rows = min(b, S - r * b);
   const int esz = I8 ? 1 : 2;
@@ -742,10 +743,11 @@ __global__ void __maxnreg__(64)
                 (uint32_t)arows * 128u * esz);
   }
   const int warp = tid >> 5, lane = tid & 31;
+  float *out = qbar + ((size_t)h * n + r) * 128 + warp * 32;
   if (I8) {
-    // 8 threads per 128-byte row, 16 rows per pass; thread owns 16 columns
+    // warp's 32 columns = 32 bytes per row: lane (c = lane & 1, rr = lane >> 1) owns 16 columns, 16 rows per pass
     const int8_t *q8 = reinterpret_cast<const int8_t *>(q);
-    const int c16 = tid & 7, rr = tid >> 3;
+    const int c = lane & 1, rr = lane >> 1;
     int acc[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) acc[e] = 0;
@@ -753,34 +755,31 @@ __global__ void __maxnreg__(64)
       int4 v[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        v[j] = (p + 16 * j < rows) ? *reinterpret_cast<const int4 *>(q8 + (row0 + p + 16 * j) * 128 + c16 * 16)
-                                   : make_int4(0, 0, 0, 0);
+        v[j] = (p + 16 * j < rows)
+                   ? *reinterpret_cast<const int4 *>(q8 + (row0 + p + 16 * j) * 128 + warp * 32 + c * 16)
+                   : make_int4(0, 0, 0, 0);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+        const int w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[e] += (int)(int8_t)((w[e >> 2] >> (8 * (e & 3))) & 0xff);
+        for (int e = 0; e < 16; ++e) acc[e] += (int)(int8_t)((w4[e >> 2] >> (8 * (e & 3))) & 0xff);
       }
     }
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       int a = acc[e];
-      a += __shfl_xor_sync(0xffffffffu, a, 8);
-      a += __shfl_xor_sync(0xffffffffu, a, 16);
+#pragma unroll
+      for (int sft = 2; sft < 32; sft <<= 1) a += __shfl_xor_sync(0xffffffffu, a, sft);
       acc[e] = a;
     }
-    if (lane < 8) {
+    if (lane < 2) {
 #pragma unroll
-      for (int e = 0; e < 16; ++e) red[warp][lane * 16 + e] = (float)acc[e];
+      for (int e = 0; e < 16; ++e) out[c * 16 + e] = (float)acc[e] * q_scale[h] / (float)rows;
     }
-    __syncthreads();
-    float s2 = 0.f;
-    for (int w = 0; w < 4; ++w) s2 += red[w][tid];
-    qbar[((size_t)h * n + r) * 128 + tid] = s2 * q_scale[h] / (float)rows;
   } else {
-    // 16 threads per 256-byte row, 8 rows per pass; thread owns 8 columns
+    // warp's 32 columns = 64 bytes per row: lane (c = lane & 3, rr = lane >> 2) owns 8 columns, 8 rows per pass
     const __nv_bfloat16 *qh = reinterpret_cast<const __nv_bfloat16 *>(q);
-    const int c8 = tid & 15, rr = tid >> 4;
+    const int c = lane & 3, rr = lane >> 2;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -788,28 +787,28 @@ __global__ void __maxnreg__(64)
       uint4 v[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        v[j] = (p + 8 * j < rows) ? *reinterpret_cast<const uint4 *>(qh + (row0 + p + 8 * j) * 128 + c8 * 8)
-                                  : make_uint4(0u, 0u, 0u, 0u);
+        v[j] = (p + 8 * j < rows)
+                   ? *reinterpret_cast<const uint4 *>(qh + (row0 + p + 8 * j) * 128 + warp * 32 + c * 8)
+                   : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+        const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          acc[2 * e] += __uint_as_float(w[e] << 16);
-          acc[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+          acc[2 * e] += __uint_as_float(w4[e] << 16);
+          acc[2 * e + 1] += __uint_as_float(w4[e] & 0xFFFF0000u);
         }
       }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
-    if (lane < 16) {
+    for (int e = 0; e < 8; ++e) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = acc[e];
+      for (int sft = 4; sft < 32; sft <<= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], sft);
     }
-    __syncthreads();
-    float s2 = 0.f;
-    for (int w = 0; w < 4; ++w) s2 += red[w][tid];
-    qbar[((size_t)h * n + r) * 128 + tid] = s2 / (float)rows;
+    if (lane < 4) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) out[c * 8 + e] = acc[e] / (float)rows;
+    }
   }
 }
 
@@ -1047,39 +1046,30 @@ __device__ __forceinline__ void cut_row(int pat, int h, int r, int n, const floa
       s_gt = f_hi;  // every candidate above T has key >= hi
     }
   }
-  // emit ascending; ties at T in index order until the target is reached
+  // Ties at T are taken in index order while the kept sum is below the
+  // target: the count taken is the smallest k with s_gt + k t_fx >= need
+  // (all of them if the target is not reached, or if T is below the fixed
+  // point's resolution).  A tie's rank is its position among the ties in
+  // index order (slot-major, then lane).
+  uint32_t take_ties = 0u;
+  if (mode == 2 && s_gt < need_fx) {
+    const uint32_t t_fx = __float2uint_rn(__uint_as_float(T) * kCutFx);
+    take_ties = t_fx ? (need_fx - s_gt + t_fx - 1u) / t_fx : 0xFFFFFFFFu;
+  }
+  const uint32_t lt_mask = (1u << lane) - 1u;
   int written = 0;
-  uint32_t tie_acc = s_gt;
-  const uint32_t t_fx = __float2uint_rn(__uint_as_float(T) * kCutFx);
-  bool ties_done = false;
+  uint32_t ties_before = 0u;
 #pragma unroll
   for (int i = 0; i < NL; ++i) {
     const int c = lane + 32 * i;
-    bool keep = false, is_tie = false;
-    if (c <= r) {
-      if (mode == 0 || c == r) keep = true;
-      else if (mode == 2) {
-        const uint32_t key = __float_as_uint(v[i]);
-        keep = key > T;
-        is_tie = (key == T);
-      }
-    }
-    if (mode == 2) {
-      uint32_t tmask = __ballot_sync(0xffffffffu, is_tie);
-      uint32_t take = 0u;
-      while (tmask && !ties_done) {
-        if (tie_acc >= need_fx) {
-          ties_done = true;
-          break;
-        }
-        take |= 1u << (__ffs(tmask) - 1);
-        tie_acc += t_fx;
-        tmask &= tmask - 1u;
-      }
-      if (take & (1u << lane)) keep = true;
-    }
+    const uint32_t key = __float_as_uint(v[i]);
+    const bool is_tie = mode == 2 && c < r && key == T;
+    const uint32_t tm = __ballot_sync(0xffffffffu, is_tie);
+    const bool keep = c <= r && (mode == 0 || c == r || (mode == 2 && key > T) ||
+                                 (is_tie && ties_before + __popc(tm & lt_mask) < take_ties));
+    ties_before += __popc(tm);
     const uint32_t km = __ballot_sync(0xffffffffu, keep);
-    if (keep) out[written + __popc(km & ((1u << lane) - 1u))] = c;
+    if (keep) out[written + __popc(km & lt_mask)] = c;
     written += __popc(km);
   }
   if (lane == 0) *count_out = written;
