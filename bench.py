@@ -462,13 +462,11 @@ def run_ours(args, w):
             "peak_source": src,
             "algorithmic_flops_per_launch": attn_flops,
             "note": "algorithmic FLOPs = 4*128^3 per computed 128x128 query-key chunk tile"}
-    # index pass against HBM: K once, Q of every head once (pooled beside the scores: which heads are
-    # query-aware is known only after them), the last query block.  The bytes a pass that pooled only
-    # the query-aware heads would need are reported beside it.
+    # index pass against HBM: K once, Q of the query-aware heads once (pooled after the pattern
+    # decision), the last query block of every head
     elt = 1 if w.int8 else 2
     qa_heads = int((exp["pattern"] == 1).sum())
-    idx_bytes = (w.Hkv * w.S * w.d + w.Hq * w.S * w.d + w.Hq * w.b * w.d) * elt
-    qa_only_bytes = (w.Hkv * w.S * w.d + qa_heads * w.S * w.d + w.Hq * w.b * w.d) * elt
+    idx_bytes = (w.Hkv * w.S * w.d + qa_heads * w.S * w.d + w.Hq * w.b * w.d) * elt
     idx_gbs = idx_bytes / (index_ms / 1e3) / 1e9
     # the pass's floors: its bytes at the HBM copy bandwidth, and its exponentials at the MUFU
     # rate and the SM clock sampled during the run
@@ -478,9 +476,7 @@ def run_ours(args, w):
     extra = {"roofline": roof,
              "index_pass": {"ms": index_ms, "algorithmic_bytes": idx_bytes, "achieved_gbs": idx_gbs,
                             "frac_of_hbm": idx_gbs / peaks["hbm_gbs"], "qa_heads": qa_heads,
-                            "bytes_note": "K + Q of every head + the last query block, each read once",
-                            "qa_only_bytes": qa_only_bytes,
-                            "frac_of_hbm_qa_only_bytes": qa_only_bytes / (index_ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                            "bytes_note": "K + Q of the query-aware heads + the last query block, each read once",
                             "hbm_floor_ms": hbm_floor_ms,
                             "exponentials": n_exp, "mufu_floor_ms": mufu_floor_ms},
              "attn_ms": attn_ms, "density": density, "chunks": chunks,

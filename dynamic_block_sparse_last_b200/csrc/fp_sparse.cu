@@ -34,10 +34,8 @@ struct fp_index {
   void *slab;
   size_t slab_bytes;
   bool slab_pooled;        // slab from the stream-ordered allocator (else cudaMalloc)
-  cudaStream_t own;        // the index's own stream: allocation and release of the slab, Q pooling
-  cudaStream_t own_hi;     // highest-priority stream of the index: the score kernel
+  cudaStream_t own;        // the index's own stream: allocation and release of the slab
   cudaEvent_t last_use;    // recorded on the caller's stream at the end of every build / attention call
-  cudaEvent_t ev_fork, ev_join, ev_score;  // fork before the pass; Q pooling done; scores done
   float *pm, *plo, *phi;   // [Hq][npart][b]
   float *ksum;             // [Hkv][npart][128]
   float *kbar;             // [Hkv][n][128]
@@ -203,12 +201,6 @@ int set_smem_attrs() {
   if (cudaFuncSetAttribute(k_sparse_attn<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            AttnCfg<I8>::kSmem) != cudaSuccess)
     return FP_ERR_CUDA;
-  // the Q pooling runs beside k_score_last on the same SMs: same (largest) shared-memory carveout
-  if (cudaFuncSetAttribute(k_qpool<I8>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared) != cudaSuccess ||
-      cudaFuncSetAttribute(k_score_last<I8>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-    return FP_ERR_CUDA;
   d->attrs[I8] = true;
   return FP_OK;
 }
@@ -231,7 +223,6 @@ struct StatsJob {
 // k_score_last on `st`.
 template <bool I8>
 int launch_score(const StatsJob &J, int *err, cudaStream_t st) {
-  int rc;
   CUtensorMap tq, tk;
   if (!make_map(&tq, J.q, I8, map_rows(J.Hq, J.ld, J.S)) || !make_map(&tk, J.k, I8, map_rows(J.Hkv, J.ld, J.S)))
     return FP_ERR_CUDA;
@@ -305,31 +296,17 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   J.ksum = I->ksum; J.kbar = I->kbar;
   J.vhat = I->vhat; J.shat = I->shat; J.pest = I->pest; J.jsd = I->jsd; J.pattern = I->pattern;
   J.ext_kbar = ext_kbar;
-  // Q block means of every head on the index's own stream, beside the score
-  // kernel (which is bound by its exponentials and leaves HBM mostly idle).
-  // Both start from one fork point on the caller's stream; the score kernel
-  // runs on the index's highest-priority stream, so its CTAs (one per SM) are
-  // dispatched before the many small pooling CTAs, which then fill the room
-  // left beside them.
+  if ((rc = launch_score<I8>(J, err, st))) return rc;
+  if ((rc = launch_head_stats<I8>(J, st))) return rc;
+  // Q block means of the query-aware heads only, now that the pattern is known
   const float *qbar = ext_qbar;
   if (!qbar) {
-    if (cudaEventRecord(I->ev_fork, st) != cudaSuccess || cudaStreamWaitEvent(I->own_hi, I->ev_fork, 0) != cudaSuccess ||
-        cudaStreamWaitEvent(I->own, I->ev_fork, 0) != cudaSuccess)
-      return FP_ERR_CUDA;
-    if ((rc = launch_score<I8>(J, err, I->own_hi))) return rc;
-    if (cudaEventRecord(I->ev_score, I->own_hi) != cudaSuccess) return FP_ERR_CUDA;
-    k_qpool<I8><<<dim3(I->n, I->Hq), 128, 0, I->own>>>(q, q_scale, I->S, I->ld, I->b, I->n, I->qbar);
+    k_qpool<I8><<<dim3(I->n, I->Hq), 128, 0, st>>>(I->pattern, q, q_scale, I->S, I->ld, I->b, I->n, I->qbar);
     if ((rc = launch_status())) return rc;
-    if (cudaEventRecord(I->ev_join, I->own) != cudaSuccess || cudaStreamWaitEvent(st, I->ev_score, 0) != cudaSuccess)
-      return FP_ERR_CUDA;
     qbar = I->qbar;
-  } else if ((rc = launch_score<I8>(J, err, st))) {
-    return rc;
   }
-  if ((rc = launch_head_stats<I8>(J, st))) return rc;
   const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
   const float *kbar = ext_kbar ? ext_kbar : I->kbar;
-  if (!ext_qbar && cudaStreamWaitEvent(st, I->ev_join, 0) != cudaSuccess) return FP_ERR_CUDA;
   const int nt = (I->n + kLgTile - 1) / kLgTile;
   k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, qbar, kbar, I->g, I->n,
                                                                inv_sqrt_d, I->zlog);
@@ -410,25 +387,6 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
     free(I);
     return FP_ERR_CUDA;
   }
-  if (cudaEventCreateWithFlags(&I->ev_fork, cudaEventDisableTiming) != cudaSuccess) {
-    cudaEventDestroy(I->last_use);
-    cudaStreamDestroy(I->own);
-    free(I);
-    return FP_ERR_CUDA;
-  }
-  int prio_lo = 0, prio_hi = 0;
-  cudaDeviceGetStreamPriorityRange(&prio_lo, &prio_hi);
-  if (cudaEventCreateWithFlags(&I->ev_join, cudaEventDisableTiming) != cudaSuccess ||
-      cudaEventCreateWithFlags(&I->ev_score, cudaEventDisableTiming) != cudaSuccess ||
-      cudaStreamCreateWithPriority(&I->own_hi, cudaStreamNonBlocking, prio_hi) != cudaSuccess) {
-    if (I->ev_join) cudaEventDestroy(I->ev_join);
-    if (I->ev_score) cudaEventDestroy(I->ev_score);
-    cudaEventDestroy(I->ev_fork);
-    cudaEventDestroy(I->last_use);
-    cudaStreamDestroy(I->own);
-    free(I);
-    return FP_ERR_CUDA;
-  }
   // stream-ordered allocation, so that freeing waits for this index's work
   // only; plain cudaMalloc where the device has no memory pools
   I->slab_pooled = cudaMallocAsync(&I->slab, need, I->own) == cudaSuccess &&
@@ -437,10 +395,6 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
     cudaGetLastError();
     I->slab = nullptr;
     if (cudaMalloc(&I->slab, need) != cudaSuccess) {
-      cudaStreamDestroy(I->own_hi);
-      cudaEventDestroy(I->ev_score);
-      cudaEventDestroy(I->ev_join);
-      cudaEventDestroy(I->ev_fork);
       cudaEventDestroy(I->last_use);
       cudaStreamDestroy(I->own);
       free(I);
@@ -491,11 +445,7 @@ void fp_index_free(fp_index *I) {
     cudaEventSynchronize(I->last_use);
     cudaFree(I->slab);
   }
-  cudaEventDestroy(I->ev_score);
-  cudaEventDestroy(I->ev_join);
-  cudaEventDestroy(I->ev_fork);
   cudaEventDestroy(I->last_use);
-  cudaStreamDestroy(I->own_hi);
   cudaStreamDestroy(I->own);  // returns at once; the stream's pending free still completes
   if (prev >= 0) cudaSetDevice(prev);
   free(I);

@@ -16,8 +16,7 @@
 //   k_head_stats   one cluster per head: row max / sum, row-normalised
 //                  block masses, vhat, shat, block means of K, P_est, JSD,
 //                  pattern.
-//   k_qpool        block means of Q of every head, on a second stream
-//                  beside k_score_last.
+//   k_qpool        block means of Q of the query-aware heads.
 //   k_qa_logits    q-bar . k-bar logits of query-aware heads (tiled fp32).
 //   k_cut          per (head, query block): scores, gamma cut, sorted list.
 #pragma once
@@ -74,8 +73,7 @@ struct ScoreParams {
 
 template <bool I8>
 struct ScoreCfg {
-  // two 32 KB K stages for bf16 keep the CTA at 193 KB of shared memory, so a
-  // Q-pooling CTA (k_qpool) fits beside it on the same SM
+  // two bf16 K stages: a third measured no faster (the kernel is bound by its exponentials)
   static constexpr int kStages = I8 ? 4 : 2;
   static constexpr int kTileBytes = I8 ? 16384 : 32768;  // 128 rows x 128 elements
   static constexpr int kTiles = 4;       // row tiles per CTA
@@ -708,13 +706,15 @@ __global__ void __cluster_dims__(kStatCta, 1, 1) __launch_bounds__(kStatThreads,
 }
 
 // ---------------------------------------------------------------------------
-// k_qpool: grid (n, Hq), block 128, at most 64 registers per thread and no
-// shared memory: one warp per SM sub-partition, so a CTA fits beside a
-// k_score_last CTA (6 warps x 72 registers per sub-partition, ~198 KB of
-// shared memory) and the two overlap; the score kernel is bound by its
-// exponentials and leaves HBM mostly idle.  qbar[h][r][t] = mean of the Q
-// rows of block r (b rows, or S - (n-1)b for a partial last block), for
-// every head: which heads are query-aware is known only after the scores.
+// k_qpool: grid (n, Hq), block 128, at most 64 registers per thread, no
+// shared memory, so that 8 CTAs (32 warps, 256 loads of 16 bytes in flight
+// per SM sub-partition) share an SM.  For the query-aware heads only (the
+// CTAs of the others exit at once): qbar[h][r][t] = mean of the Q rows of
+// block r (b rows, or S - (n-1)b for a partial last block).  Runs after the
+// pattern decision.  (Pooling every head beside k_score_last instead, on a
+// second stream or in extra warps of that kernel, measured slower: the
+// score kernel holds the register file and almost all shared memory of its
+// SM, which leaves the pooling too few bytes in flight.)
 // Warp w owns columns 32w .. 32w+31; lane (c = lane & 3, rr = lane >> 2)
 // loads 16 bytes of rows rr, rr + 8, ..., eight rows' loads in flight, and
 // the rows are summed across lanes with shuffles.  The block kPoolAhead
@@ -729,9 +729,10 @@ __device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
 
 template <bool I8>
 __global__ void __maxnreg__(64)
-    k_qpool(const void *__restrict__ q, const float *__restrict__ q_scale, int S, int ld, int b, int n,
-            float *__restrict__ qbar) {
+    k_qpool(const int *__restrict__ pattern, const void *__restrict__ q, const float *__restrict__ q_scale, int S,
+            int ld, int b, int n, float *__restrict__ qbar) {
   const int r = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+  if (pattern[h] != 1) return;
   const size_t row0 = (size_t)h * ld + (size_t)r * b;
   const int rows = min(b, S - r * b);
   const int esz = I8 ? 1 : 2;
