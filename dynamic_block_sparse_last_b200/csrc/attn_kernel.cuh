@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(608, 1)
 #pragma unroll
         for (int e = 0; e < 64; ++e) s[e] = (ch * 64 + e <= row) ? s[e] : -INFINITY;
       }
-      // row max: eight chains of three-input max, then a short tree
+      // row max: eight chains of maxima, then a short tree
       float m8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) m8[e] = s[e];

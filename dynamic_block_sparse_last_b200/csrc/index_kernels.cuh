@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(736, 1)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) s[e] = (e <= dlt) ? s[e] : -INFINITY;
               }
-              // piece max: eight chains of three-input max, then a short tree
+              // piece max: eight chains of maxima, then a short tree
               float m8[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) m8[e] = fmax3(s[e], s[8 + e], s[16 + e]);
