@@ -41,9 +41,12 @@
 //
 // MMA issue order per union entry u: for each tile t, PV_t(u-1) then
 // QK_t(u).  While softmax t works on S_t(u), the tensor pipe runs the other
-// tile's PV and QK.  The reference max of a row is raised lazily (only when
-// the row max exceeds it by more than 2^8); the correction O *= 2^(m_old -
-// m_new) runs in TMEM after PV_t(u-1) has completed.
+// tile's PV and QK.  The exponentials of a chunk are taken against the
+// row's current reference max at once; the reference moves (to the row max)
+// only when the chunk's row sum exceeds 2^8 or the row has none yet, and
+// the chunk is then recomputed, so no row max is formed in the common case.
+// The correction O *= 2^(m_old - m_new) runs in TMEM after PV_t(u-1) has
+// completed.
 #pragma once
 
 #include "ptx.cuh"
@@ -399,6 +402,7 @@ __global__ void __launch_bounds__(608, 1)
     float scale2 = P.scale2;
     if (I8 && me.valid) scale2 *= P.q_scale[me.h] * P.k_scale[kvh];
     float m_ref = -INFINITY, l = 0.f;
+    int nx = 0;  // exchanges with the partner half so far (phase and buffer parity)
     bool ok = true;
     // this tile's chunks, ascending: the entries its S tile receives
     int L = 0;
@@ -424,81 +428,110 @@ __global__ void __launch_bounds__(608, 1)
             dst[e] = make_int4((int)rr[4 * e], (int)rr[4 * e + 1], (int)rr[4 * e + 2], (int)rr[4 * e + 3]);
         }
       }
+      // S (this warp's 64 keys) as fp32 with the masks applied; -inf where
+      // a key is not visible.  Called again when the reference must move.
       float s[64];
-#pragma unroll
-      for (int e = 0; e < 64; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
-      if (P.b < 128) {
-        // the warp's quadrant is one (query block, key block 2kc + ch) pair
-        const int kb = 2 * kc + ch;
-        if (!((vis_bm[kb >> 5] >> (kb & 31)) & 1u)) {
-#pragma unroll
-          for (int e = 0; e < 64; ++e) s[e] = -INFINITY;
+      auto load_s = [&](bool reload) {
+        if (reload) {
+          tmem_ld64(s_tm, rr);
+          tmem_ld_wait64(rr);
         }
-      }
-      if (j == L - 1) {
-        // diagonal chunk: key 64ch+e of the chunk is visible iff it is <= row
 #pragma unroll
-        for (int e = 0; e < 64; ++e) s[e] = (ch * 64 + e <= row) ? s[e] : -INFINITY;
-      }
-      // row max: eight chains of maxima, then a short tree
-      float m8[8];
+        for (int e = 0; e < 64; ++e) s[e] = I8 ? (float)(int)rr[e] : __uint_as_float(rr[e]);
+        if (P.b < 128) {
+          // the warp's quadrant is one (query block, key block 2kc + ch) pair
+          const int kb = 2 * kc + ch;
+          if (!((vis_bm[kb >> 5] >> (kb & 31)) & 1u)) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) m8[e] = s[e];
+            for (int e = 0; e < 64; ++e) s[e] = -INFINITY;
+          }
+        }
+        if (j == L - 1) {
+          // diagonal chunk: key 64ch+e of the chunk is visible iff it is <= row
 #pragma unroll
-      for (int c = 8; c < 64; c += 16)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
-      const float pmx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      // exchange with the partner half (also orders both halves' S reads
-      // before either writes P over the first 64 columns of S)
-      xmax[j & 1][t][ch][row] = pmx;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(xbar);
-      if (!mbar_wait(xbar, j & 1, abort_flag, P.err)) { ok = false; break; }
-      tc_fence_after();
-      const float mx = fmaxf(pmx, xmax[j & 1][t][ch ^ 1][row]);
-      const float rmax2 = mx * scale2;
-      const bool raise = rmax2 > m_ref + 8.f;
-      const float m_new = raise ? rmax2 : m_ref;
-      const float alpha = raise ? ex2(m_ref - m_new) : 1.f;
-      // a row that has seen no visible key yet keeps m = -inf and P = 0
-      const float m_sub = (m_new == -INFINITY) ? 0.f : m_new;
-      // P in bf16 (the P.V operand); the row sum adds the same rounded values
+          for (int e = 0; e < 64; ++e) s[e] = (ch * 64 + e <= row) ? s[e] : -INFINITY;
+        }
+      };
+      // P in bf16 (the P.V operand) against reference m (log2 units; 0
+      // stands for "none yet"), and the row sum of the same rounded values:
+      // each bf16 added to an fp32 chain as it is (mixed-precision add), eight chains
       uint32_t pk[32];
-      float r8[8];
+      auto make_p = [&](float m) -> float {
+        float r8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) r8[e] = 0.f;
-      // Off the diagonal chunk every kExpFmaEvery-th exponential may run on
-      // the FMA pipe (ex2_fma); the diagonal chunk has masked (-inf) entries
-      // and uses MUFU only, which maps them to exactly 0.
-      if (C::kExpFmaEvery > 0 && j != L - 1) {
+        for (int e = 0; e < 8; ++e) r8[e] = 0.f;
+        if (C::kExpFmaEvery > 0 && j != L - 1) {
+          // every kExpFmaEvery-th exponential on the FMA pipe (ex2_fma); the
+          // diagonal chunk has masked (-inf) entries and uses MUFU only
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const float x0 = fmaf(s[e], scale2, -m_sub), x1 = fmaf(s[e + 1], scale2, -m_sub);
-          const bool f1 = ((e + 1) % (C::kExpFmaEvery > 0 ? C::kExpFmaEvery : 1)) == 0;
-          pk[e >> 1] = pack_bf16x2(ex2(x0), f1 ? ex2_fma(x1) : ex2(x1));
+          for (int e = 0; e < 64; e += 2) {
+            const float x0 = fmaf(s[e], scale2, -m), x1 = fmaf(s[e + 1], scale2, -m);
+            const bool f1 = ((e + 1) % (C::kExpFmaEvery > 0 ? C::kExpFmaEvery : 1)) == 0;
+            pk[e >> 1] = pack_bf16x2(ex2(x0), f1 ? ex2_fma(x1) : ex2(x1));
+          }
+        } else {
+          // exponent arguments two at a time (packed fp32 FMA), then MUFU ex2
+          const uint64_t sc2 = f2_pack(scale2, scale2), nm2 = f2_pack(-m, -m);
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+            pk[e >> 1] = pack_bf16x2(ex2(x0), ex2(x1));
+          }
         }
-      } else {
-        // exponent arguments two at a time (packed fp32 FMA), then MUFU ex2
-        const uint64_t sc2 = f2_pack(scale2, scale2), nm2 = f2_pack(-m_sub, -m_sub);
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
-          pk[e >> 1] = pack_bf16x2(ex2(x0), ex2(x1));
-        }
+        for (int e = 0; e < 32; ++e) add_bf16x2_f32(pk[e], r8[(2 * e) & 7], r8[(2 * e + 1) & 7]);
+        return ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
+      };
+      // one exchange with the partner half through shared memory; also
+      // orders both halves' S reads before either writes P over the first
+      // 64 columns of S
+      auto exchange = [&](float v, float &partner) -> bool {
+        xmax[nx & 1][t][ch][row] = v;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(xbar);
+        if (!mbar_wait(xbar, nx & 1, abort_flag, P.err)) return false;
+        tc_fence_after();
+        partner = xmax[nx & 1][t][ch ^ 1][row];
+        ++nx;
+        return true;
+      };
+      load_s(false);
+      // Exponentials first, against the current reference m_ref.  The
+      // reference moves only when the row's chunk sum (both halves) exceeds
+      // 2^8, which bounds every P of the chunk by 2^8, or when the row has no
+      // reference yet; then the row max is taken, S is read again (P has
+      // not been written over it yet) and P is recomputed.  In the common
+      // case no row max is computed at all.
+      float rs = make_p(m_ref == -INFINITY ? 0.f : m_ref);
+      float rs_other;
+      if (!exchange(rs, rs_other)) { ok = false; break; }
+      const bool trig = !(rs + rs_other <= 256.f) || m_ref == -INFINITY;
+      float alpha = 1.f;
+      bool moved = false;
+      if (__any_sync(0xffffffffu, trig)) {
+        load_s(true);
+        float m8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m8[e] = s[e];
+#pragma unroll
+        for (int c = 8; c < 64; c += 16)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) m8[e] = fmax3(m8[e], s[c + e], s[c + 8 + e]);
+        const float pmx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+        float pmx_other;
+        if (!exchange(pmx, pmx_other)) { ok = false; break; }
+        const float m_new = trig ? fmaxf(m_ref, fmaxf(pmx, pmx_other) * scale2) : m_ref;
+        moved = m_new > m_ref;
+        alpha = moved ? ex2(m_ref - m_new) : 1.f;  // 0 when there was no reference
+        m_ref = m_new;
+        rs = make_p(m_ref == -INFINITY ? 0.f : m_ref);
       }
-      // row sum of the rounded P: each bf16 added to an fp32 chain as it is
-      // (mixed-precision add, no unpacking), eight chains
-#pragma unroll
-      for (int e = 0; e < 32; ++e) add_bf16x2_f32(pk[e], r8[(2 * e) & 7], r8[(2 * e + 1) & 7]);
-      const float rs = ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       l = l * alpha + rs;
-      m_ref = m_new;
       // The commit that signalled S(j) also covers PV(j-1), issued before
       // QK(j): O is stable here and may be rescaled in place.
-      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+      if (j > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll 1
         for (int qq = 0; qq < 2; ++qq) {
           uint32_t o[32];
@@ -521,7 +554,7 @@ __global__ void __launch_bounds__(608, 1)
       xl[t][ch][row] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(xbar);
-      if (mbar_wait(xbar, L & 1, abort_flag, P.err)) {
+      if (mbar_wait(xbar, nx & 1, abort_flag, P.err)) {
         const float inv = 1.f / (l + xl[t][ch ^ 1][row]);
         const bool store = me.qc * 128 + row < P.S;  // rows past S belong to a neighbour
         __nv_bfloat16 *orow = P.out + ((size_t)me.h * P.ld + (size_t)me.qc * 128 + row) * 128 + ch * 64;
