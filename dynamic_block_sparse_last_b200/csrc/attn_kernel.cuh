@@ -43,7 +43,7 @@
 // QK_t(u).  While softmax t works on S_t(u), the tensor pipe runs the other
 // tile's PV and QK.  The exponentials of a chunk are taken against the
 // row's current reference max at once; the reference moves (to the row max)
-// only when the chunk's row sum exceeds 2^8 or the row has none yet, and
+// only when the chunk's row sum exceeds kRefSum or the row has none yet, and
 // the chunk is then recomputed, so no row max is formed in the common case.
 // The correction O *= 2^(m_old - m_new) runs in TMEM after PV_t(u-1) has
 // completed.
@@ -83,6 +83,10 @@ struct AttnCfg {
   // FMA pipe (ex2_fma) instead of MUFU; 0 keeps all on MUFU.  A share of 1/4
   // measured no faster on the 128K layer (power-capped clocks), so it is off.
   static constexpr int kExpFmaEvery = 0;
+  // The reference max of a row moves when a chunk's row sum of P exceeds
+  // this bound, so no P exceeds it (bf16 keeps its relative precision at any
+  // magnitude; the sums and O accumulate in fp32).
+  static constexpr float kRefSum = 256.f;
 };
 
 // Number of CTAs (tile pairs) for a layer shape.
@@ -500,14 +504,14 @@ __global__ void __launch_bounds__(608, 1)
       load_s(false);
       // Exponentials first, against the current reference m_ref.  The
       // reference moves only when the row's chunk sum (both halves) exceeds
-      // 2^8, which bounds every P of the chunk by 2^8, or when the row has no
+      // kRefSum, which bounds every P of the chunk by it, or when the row has no
       // reference yet; then the row max is taken, S is read again (P has
       // not been written over it yet) and P is recomputed.  In the common
       // case no row max is computed at all.
       float rs = make_p(m_ref == -INFINITY ? 0.f : m_ref);
       float rs_other;
       if (!exchange(rs, rs_other)) { ok = false; break; }
-      const bool trig = !(rs + rs_other <= 256.f) || m_ref == -INFINITY;
+      const bool trig = !(rs + rs_other <= C::kRefSum) || m_ref == -INFINITY;
       float alpha = 1.f;
       bool moved = false;
       if (__any_sync(0xffffffffu, trig)) {

@@ -56,6 +56,10 @@ class Workload:
     seed: int = 0
     int8: bool = False
     kinds: list = field(default_factory=list)
+    # > 0: key row j is scaled by 1 + key_ramp * j / S after the structure is
+    # planted, so the scores (and each row's running maximum) grow along the
+    # key axis; 0 leaves the keys as generated
+    key_ramp: float = 0.0
 
     def head_kinds(self):
         if self.kinds:
@@ -163,6 +167,8 @@ def make_inputs(w: Workload):
         extra = torch.randperm(max(S - 4, 0), generator=gen)[: min(w.n_vertical, max(S - 4, 0))] + 4
         pos = torch.cat([torch.arange(min(4, S)), extra])
         k[h // g, pos] += 3.0 * mu
+    if w.key_ramp:
+        k *= (1.0 + w.key_ramp * torch.arange(S, dtype=torch.float32) / S)[None, :, None]
     out = {
         "q": q.to(torch.bfloat16).contiguous(),
         "k": k.to(torch.bfloat16).contiguous(),

@@ -360,3 +360,54 @@ def test_sweep_b256_gammas(fp, name):
     tiles = [(h, qc) for h in range(w.Hq) for qc in range(nq)] if w.S <= 16384 else \
         sampled_tiles(w, 64, seed=w.seed + w.S)
     check_tiles(P, exp, out, w, tiles)
+
+
+def reference_moves(x, w, heads):
+    """How often the softmax's reference max must move after a row's first
+    chunk, by the rule the attention kernel applies (chunk row sum of
+    2^(x - m) above 2^8, x = q.k log2(e) / sqrt(d)), evaluated in fp64 on the
+    bf16 inputs at gamma = 1 (every causal key).  Used to show that a case
+    exercises the recompute path; the kernel's own sums are of bf16-rounded
+    exponentials, so its count can differ slightly."""
+    g = w.Hq // w.Hkv
+    c = math.log2(math.e) / math.sqrt(w.d)
+    moves = 0
+    for h in heads:
+        q = x["q"][h].double().numpy()
+        k = x["k"][h // g].double().numpy()
+        sc = (q @ k.T) * c
+        for i in range(w.S):
+            m = -math.inf
+            for c0 in range(0, i + 1, 128):
+                xs = sc[i, c0:min(i + 1, c0 + 128)]
+                if m == -math.inf:
+                    m = float(xs.max())
+                    continue
+                if float(np.exp2(xs - m).sum()) > 256.0:
+                    m = max(m, float(xs.max()))
+                    moves += 1
+    return moves
+
+
+RAMP = [synth.Workload("ramp_b128", S=2048, Hq=4, Hkv=1, b=128, gamma=1.0, key_ramp=15.0, seed=31),
+        synth.Workload("ramp_int8", S=2048, Hq=4, Hkv=1, b=128, gamma=1.0, key_ramp=15.0, int8=True, seed=31),
+        synth.Workload("ramp_b64_ragged", S=1500, Hq=4, Hkv=2, b=64, gamma=1.0, key_ramp=15.0, seed=32),
+        synth.Workload("ramp_b256", S=2048, Hq=4, Hkv=2, b=256, gamma=1.0, key_ramp=15.0, seed=32)]
+
+
+@pytest.mark.parametrize("w", RAMP, ids=[w.name for w in RAMP])
+def test_rising_scores_move_the_reference(fp, w):
+    """Keys scaled up along the sequence make every row's maximum grow from
+    chunk to chunk, so the softmax's reference has to move (and its chunk be
+    recomputed, and O rescaled) many times per row; every tile is compared
+    with the oracle on the GPU's index (gamma = 1: all causal blocks)."""
+    x = synth.make_inputs(w)
+    exp, out, idx = run_gpu(fp, x, w)
+    n = nblocks(w.S, w.b)
+    assert exp["nnz"] == w.Hq * n * (n + 1) // 2
+    moves = reference_moves(x, w, [0])
+    print(f"[{w.name}] reference moves after the first chunk, head 0: {moves} over {w.S} rows")
+    assert moves >= w.S  # more than one per row on average
+    P = oracle_problem(x, w)
+    tiles = [(h, qc) for h in range(w.Hq) for qc in range(nblocks(w.S, 128))]
+    check_tiles(P, exp, out, w, tiles)

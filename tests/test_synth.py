@@ -82,3 +82,19 @@ def test_prerope_inputs_are_seeded_and_shaped():
         assert torch.equal(a[key], b[key]), key
     c = synth.make_prerope_inputs(synth.Workload("pr", S=200, Hq=4, Hkv=2, b=64, seed=8))
     assert not torch.equal(a["q_in"], c["q_in"])
+
+
+def test_key_ramp_scales_key_rows():
+    """key_ramp multiplies key row j by 1 + key_ramp * j / S and touches nothing else."""
+    base = synth.Workload("r0", S=256, Hq=2, Hkv=1, seed=5)
+    ramp = synth.Workload("r1", S=256, Hq=2, Hkv=1, seed=5, key_ramp=3.0)
+    a, b = synth.make_inputs(base), synth.make_inputs(ramp)
+    assert torch.equal(a["q"], b["q"]) and torch.equal(a["v"], b["v"])
+    fac = 1.0 + 3.0 * torch.arange(256, dtype=torch.float32) / 256
+    want = (a["k"].float() * fac[None, :, None]).to(torch.bfloat16)
+    # both sides round the same fp32 product once; the generator scales before its
+    # single bf16 rounding, so allow one bf16 step
+    diff = (b["k"].float() - want.float()).abs()
+    assert float(diff.max()) <= float(want.float().abs().max()) * 2 ** -7
+    norms = b["k"][0].float().norm(dim=1)
+    assert float(norms[-32:].mean()) > 3.0 * float(norms[:32].mean())
