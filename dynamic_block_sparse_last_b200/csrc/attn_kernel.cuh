@@ -35,9 +35,11 @@
 //   warp 17          TMEM owner and MMA issuer (one thread)
 //   warp 18          TMA producer of V chunks (2-stage ring)
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
-// The softmax writes P (bf16, two per column) over the first 64 columns of
-// its S tile and the P.V product reads it from TMEM (tcgen05.mma A operand
-// in tensor memory), so P never touches shared memory.
+// Each softmax warp writes the P of its 64 keys (bf16, two per column) over
+// the first 32 of its own 64 S columns, so P occupies columns 0-31 and 64-95
+// of the S tile and no warp writes where another still reads. The P.V
+// product reads P from TMEM (tcgen05.mma A operand in tensor memory), so P
+// never touches shared memory.
 //
 // MMA issue order per union entry u: for each tile t, PV_t(u-1) then
 // QK_t(u).  While softmax t works on S_t(u), the tensor pipe runs the other
@@ -341,7 +343,8 @@ __global__ void __launch_bounds__(608, 1)
         const uint64_t dv = vst ? dv1 : dv0;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + kk * 8, dv + (uint64_t)((kk * 2048) >> 4), id_pv,
+          mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + (kk >> 2) * 64 + (kk & 3) * 8,
+                      dv + (uint64_t)((kk * 2048) >> 4), id_pv,
                       (npv[t] > 0 || kk > 0));
         tc_commit(smem_u32(&bar_odone[t]));
         ++npv[t];
@@ -400,7 +403,7 @@ __global__ void __launch_bounds__(608, 1)
     const int row = lq * 32 + lane;
     const uint32_t lane_off = ((uint32_t)(lq * 32)) << 16;
     const uint32_t s_tm = tmem + t * 128 + ch * 64 + lane_off;    // this warp's S columns
-    const uint32_t p_tm = tmem + t * 128 + ch * 32 + lane_off;    // packed P of its 64 keys
+    const uint32_t p_tm = tmem + t * 128 + ch * 64 + lane_off;    // packed P of its 64 keys, over its own S
     const uint32_t o_tm = tmem + 256 + t * 128 + ch * 64 + lane_off;
     const uint32_t xbar = smem_u32(&bar_xchg[t][lq]);
     float scale2 = P.scale2;
@@ -487,16 +490,14 @@ __global__ void __launch_bounds__(608, 1)
         for (int e = 0; e < 32; ++e) add_bf16x2_f32(pk[e], r8[(2 * e) & 7], r8[(2 * e + 1) & 7]);
         return ((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7]));
       };
-      // one exchange with the partner half through shared memory; also
-      // orders both halves' S reads before either writes P over the first
-      // 64 columns of S
+      // one exchange with the partner half through shared memory (each warp
+      // writes P only over its own S columns, so no tensor-memory ordering
+      // between the two is needed here)
       auto exchange = [&](float v, float &partner) -> bool {
         xmax[nx & 1][t][ch][row] = v;
-        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(xbar);
         if (!mbar_wait(xbar, nx & 1, abort_flag, P.err)) return false;
-        tc_fence_after();
         partner = xmax[nx & 1][t][ch ^ 1][row];
         ++nx;
         return true;
