@@ -44,8 +44,9 @@
 // MMA issue order per union entry u: for each tile t, PV_t(u-1) then
 // QK_t(u).  While softmax t works on S_t(u), the tensor pipe runs the other
 // tile's PV and QK.  The exponentials of a chunk are taken against the
-// row's current reference max at once; the reference moves (to the row max)
-// only when the chunk's row sum exceeds kRefSum or the row has none yet, and
+// row's current reference max at once; the reference moves (to the row max
+// plus a headroom) only when the chunk's row sum exceeds kRefSum or the row
+// has none yet, and
 // the chunk is then recomputed, so no row max is formed in the common case.
 // The correction O *= 2^(m_old - m_new) runs in TMEM after PV_t(u-1) has
 // completed.
@@ -89,6 +90,14 @@ struct AttnCfg {
   // this bound, so no P exceeds it (bf16 keeps its relative precision at any
   // magnitude; the sums and O accumulate in fp32).
   static constexpr float kRefSum = 256.f;
+  // A moved reference is set this far (log2 units) above the row max, so the
+  // next move needs the scores to rise about log2(kRefSum) + kRefHeadroom
+  // above it.  Scores near the diagonal often exceed those of the first
+  // chunks by tens of log2 units; with this headroom such rows rarely move
+  // again.  P then starts near 2^-kRefHeadroom: bf16 keeps its relative
+  // precision there, and only keys more than 126 - kRefHeadroom below the
+  // row max flush to zero, whose weight relative to it is below 2^-62.
+  static constexpr float kRefHeadroom = 64.f;
 };
 
 // Number of CTAs (tile pairs) for a layer shape.
@@ -527,7 +536,7 @@ __global__ void __launch_bounds__(608, 1)
         const float pmx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
         float pmx_other;
         if (!exchange(pmx, pmx_other)) { ok = false; break; }
-        const float m_new = trig ? fmaxf(m_ref, fmaxf(pmx, pmx_other) * scale2) : m_ref;
+        const float m_new = trig ? fmaxf(m_ref, fmaxf(pmx, pmx_other) * scale2 + C::kRefHeadroom) : m_ref;
         moved = m_new > m_ref;
         alpha = moved ? ex2(m_ref - m_new) : 1.f;  // 0 when there was no reference
         m_ref = m_new;
