@@ -10,7 +10,7 @@
 //
 // Kernels, in launch order:
 //   k_score_last   tcgen05 Q_last.K^T per 128-key chunk, K streamed once per
-//                  KV group through a TMA ring; per (row, chunk) max and the
+//                  KV group through a TMA ring; per (row, chunk) reference and the
 //                  two offset-half sums; per-chunk K column sums.  Nothing of
 //                  size S x b reaches global memory.
 //   k_head_stats   one cluster per head: row max / sum, row-normalised
@@ -28,6 +28,9 @@
 namespace fpk {
 
 constexpr float kLog2e = 1.4426950408889634f;
+// headroom (log2 units) above the piece max when the statistics loop of
+// k_score_last moves a row's reference
+constexpr float kScoreHeadroom = 64.f;
 
 // ---------------------------------------------------------------------------
 // k_score_last
@@ -284,18 +287,15 @@ __global__ void __launch_bounds__(736, 1)
         uint64_t lo2 = 0ull, hi2 = 0ull;  // the part's lo / hi sums as packed fp32 pairs
         for (int u = 0; u < U && ok; ++u) {
           const int ch = ch0 + u;
-          // One pass over the chunk in 32-column pieces with an online max:
-          // lo/hi are kept relative to the running max m and rescaled when a
-          // piece raises it.  Columns t <= i (block-relative) go to lo, the
+          // One pass over the chunk in 32-column pieces: lo/hi are kept
+          // relative to the row's reference m (see below) and rescaled when
+          // it moves.  Columns t <= i (block-relative) go to lo, the
           // rest to hi; in the last block columns t > i are causally masked
           // (their exponentials are 0).  With b = 64 each 64-column half is a
-          // block of its own and gets its own (max, lo, hi) part; otherwise
+          // block of its own and gets its own (reference, lo, hi) part; otherwise
           // the chunk is one part.
           for (int hf = 0; hf < 2; ++hf) {
-            if (hf == 0 || P.nsub == 2) {
-              m = -INFINITY;
-              lo2 = hi2 = 0ull;
-            }
+            if (hf == 0 || P.nsub == 2) lo2 = hi2 = 0ull;  // the reference m carries over
             if (!mbar_wait(smem_u32(&bar_sfull[t][hf]), u & 1, abort_flag, P.err)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll 1
@@ -322,51 +322,73 @@ __global__ void __launch_bounds__(736, 1)
 #pragma unroll
                 for (int e = 0; e < 32; ++e) s[e] = (e <= dlt) ? s[e] : -INFINITY;
               }
-              // piece max: eight chains of maxima, then a short tree
-              float m8[8];
+              // the piece's lo / hi sums of 2^((s - m) scale2), exponent
+              // arguments two at a time (packed fp32 FMA), ex2, packed adds
+              auto piece = [&](uint64_t &pl, uint64_t &ph) {
+                const float nm = -m * scale2;
+                const uint64_t nm2 = f2_pack(nm, nm);
+                pl = ph = 0ull;
+                if (dlt >= 31 || dlt < 0) {
+                  uint64_t a0 = 0ull, a1 = 0ull;
 #pragma unroll
-              for (int e = 0; e < 8; ++e) m8[e] = fmax3(s[e], s[8 + e], s[16 + e]);
+                  for (int e = 0; e < 32; e += 4) {
+                    float x0, x1, x2, x3;
+                    f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+                    f2_unpack(f2_fma(f2_pack(s[e + 2], s[e + 3]), sc2, nm2), x2, x3);
+                    a0 = f2_add(a0, f2_pack(ex2(x0), ex2(x1)));
+                    a1 = f2_add(a1, f2_pack(ex2(x2), ex2(x3)));
+                  }
+                  if (dlt >= 31) pl = f2_add(a0, a1);
+                  else ph = f2_add(a0, a1);
+                } else {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[24 + e]);
-              const float pmx =
-                  fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-              if (pmx == -INFINITY) continue;  // whole piece masked
-              if (pmx > m) {
-                const float f = (m == -INFINITY) ? 0.f : ex2((m - pmx) * scale2);
-                const uint64_t f2 = f2_pack(f, f);
-                lo2 = f2_mul(lo2, f2);
-                hi2 = f2_mul(hi2, f2);
-                m = pmx;
-              }
-              const float nm = -m * scale2;
-              const uint64_t nm2 = f2_pack(nm, nm);
-              // exponent arguments two at a time (packed fp32 FMA), ex2, packed adds
-              if (dlt >= 31 || dlt < 0) {
-                uint64_t a0 = 0ull, a1 = 0ull;
-#pragma unroll
-                for (int e = 0; e < 32; e += 4) {
-                  float x0, x1, x2, x3;
-                  f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
-                  f2_unpack(f2_fma(f2_pack(s[e + 2], s[e + 3]), sc2, nm2), x2, x3);
-                  a0 = f2_add(a0, f2_pack(ex2(x0), ex2(x1)));
-                  a1 = f2_add(a1, f2_pack(ex2(x2), ex2(x3)));
+                  for (int e = 0; e < 32; e += 2) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+                    const float p0 = ex2(x0), p1 = ex2(x1);
+                    const bool q0 = e <= dlt, q1 = e + 1 <= dlt;
+                    pl = f2_add(pl, f2_pack(q0 ? p0 : 0.f, q1 ? p1 : 0.f));
+                    ph = f2_add(ph, f2_pack(q0 ? 0.f : p0, q1 ? 0.f : p1));
+                  }
                 }
-                if (dlt >= 31) lo2 = f2_add(lo2, f2_add(a0, a1));
-                else hi2 = f2_add(hi2, f2_add(a0, a1));
-              } else {
-                uint64_t l0 = 0ull, h0 = 0ull;
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                  float x0, x1;
-                  f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
-                  const float p0 = ex2(x0), p1 = ex2(x1);
-                  const bool q0 = e <= dlt, q1 = e + 1 <= dlt;
-                  l0 = f2_add(l0, f2_pack(q0 ? p0 : 0.f, q1 ? p1 : 0.f));
-                  h0 = f2_add(h0, f2_pack(q0 ? 0.f : p0, q1 ? 0.f : p1));
-                }
-                lo2 = f2_add(lo2, l0);
-                hi2 = f2_add(hi2, h0);
+              };
+              // Exponentials first, against the row's reference m (raw score
+              // units).  The reference moves -- to the piece max plus
+              // kScoreHeadroom (log2 units) -- only when the piece's sum
+              // exceeds 2^8 or the row has no reference yet; the piece is then
+              // recomputed and the part's sums so far rescaled.  The per-part
+              // partials carry the reference in place of a maximum, which the
+              // statistics kernel's log-sum-exp combination allows.
+              uint64_t pl, ph;
+              bool move = (m == -INFINITY);
+              if (!move) {
+                piece(pl, ph);
+                float a, b2, c, d2;
+                f2_unpack(pl, a, b2);
+                f2_unpack(ph, c, d2);
+                move = !((a + b2) + (c + d2) <= 256.f);
               }
+              if (move) {
+                float m8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m8[e] = fmax3(s[e], s[8 + e], s[16 + e]);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) m8[e] = fmaxf(m8[e], s[24 + e]);
+                const float pmx =
+                    fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+                if (pmx == -INFINITY) continue;  // whole piece masked and no reference yet
+                const float nmv = fmaxf(m, pmx + kScoreHeadroom / scale2);
+                if (nmv > m) {
+                  const float f = (m == -INFINITY) ? 0.f : ex2((m - nmv) * scale2);
+                  const uint64_t f2 = f2_pack(f, f);
+                  lo2 = f2_mul(lo2, f2);
+                  hi2 = f2_mul(hi2, f2);
+                  m = nmv;
+                }
+                piece(pl, ph);
+              }
+              lo2 = f2_add(lo2, pl);
+              hi2 = f2_add(hi2, ph);
             }
             tc_fence_before();
             __syncwarp();
@@ -400,7 +422,9 @@ __global__ void __launch_bounds__(736, 1)
 // kStatCta CTAs per query head h (grid (kStatCta, Hq), 256 threads).  Rank
 // k of the cluster owns the key blocks [k n / C, (k+1) n / C) and their
 // column parts.  With nlast = S - (n-1)b rows in the last block and the
-// score kernel's per-(row, part) partials (m in log2 units, lo, hi):
+// score kernel's per-(row, part) partials (m, the reference the part's sums
+// are taken against, in log2 units; lo; hi -- any reference gives the same
+// combined statistics):
 //   1. row statistics over the owned parts, combined over the cluster
 //      through distributed shared memory (in rank order):
 //        M_i = max_p m_ip,  L_i = sum_p (lo_ip + hi_ip) 2^(m_ip - M_i);
