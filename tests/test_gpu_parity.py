@@ -398,22 +398,27 @@ def reference_moves(x, w, heads):
 RAMP = [synth.Workload("ramp_b128", S=2048, Hq=4, Hkv=1, b=128, gamma=1.0, key_ramp=80.0, seed=31),
         synth.Workload("ramp_int8", S=2048, Hq=4, Hkv=1, b=128, gamma=1.0, key_ramp=80.0, int8=True, seed=31),
         synth.Workload("ramp_b64_ragged", S=1500, Hq=4, Hkv=2, b=64, gamma=1.0, key_ramp=80.0, seed=32),
-        synth.Workload("ramp_b256", S=2048, Hq=4, Hkv=2, b=256, gamma=1.0, key_ramp=80.0, seed=32)]
+        synth.Workload("ramp_b256", S=2048, Hq=4, Hkv=2, b=256, gamma=1.0, key_ramp=80.0, seed=32),
+        # gamma < 1: the selection itself depends on the statistics the moved references produce
+        synth.Workload("ramp_b128_gamma09", S=2048, Hq=4, Hkv=2, b=128, gamma=0.9, key_ramp=80.0, seed=33)]
 
 
 @pytest.mark.parametrize("w", RAMP, ids=[w.name for w in RAMP])
 def test_rising_scores_move_the_reference(fp, w):
     """Keys scaled up along the sequence make every row's maximum grow from
     chunk to chunk, so the softmax's reference has to move (and its chunk be
-    recomputed, and O rescaled) many times per row; every tile is compared
-    with the oracle on the GPU's index (gamma = 1: all causal blocks)."""
+    recomputed, and O rescaled) many times per row, and so does the score
+    kernel's per-row reference.  The index (statistics, pattern and block
+    sets) is compared with the oracle, and every tile on the GPU's index."""
     x = synth.make_inputs(w)
     exp, out, idx = run_gpu(fp, x, w)
     n = nblocks(w.S, w.b)
-    assert exp["nnz"] == w.Hq * n * (n + 1) // 2
+    if w.gamma >= 1.0:
+        assert exp["nnz"] == w.Hq * n * (n + 1) // 2
     moves = reference_moves(x, w, [0])
     print(f"[{w.name}] reference moves after the first chunk, head 0: {moves} over {w.S} rows")
     assert moves >= w.S  # more than one per row on average
     P = oracle_problem(x, w)
+    check_index(P, exp, w)
     tiles = [(h, qc) for h in range(w.Hq) for qc in range(nblocks(w.S, 128))]
     check_tiles(P, exp, out, w, tiles)
