@@ -35,8 +35,17 @@ from dynamic_block_sparse_last_b200 import synth  # noqa: E402
 
 METRIC = "sparse-prefill ms/layer & dense-equiv TFLOPS at S=128K; % of HBM/TC roofline"
 UNIT = "dense-equiv TFLOP/s"
-# k_score_last, k_head_stats, k_qbar, k_qa_logits, k_cut, k_sparse_attn
-KERNELS_PER_STEP = 6
+# the library's switch of the q-bar . k-bar logits to the tensor cores (kLgTensorMinN in
+# index_kernels.cuh): from n = 960 blocks two k_split_tf32 launches precede k_qa_logits
+LOGITS_TENSOR_MIN_N = 960
+
+
+def kernels_per_step(S: int, b: int) -> int:
+    """Launches of the library's kernels per layer step: k_score_last, k_head_stats,
+    k_qpool, k_qa_logits (plus two k_split_tf32 on the tensor-core path), k_cut,
+    k_sparse_attn."""
+    n = (S + b - 1) // b
+    return 6 + (2 if n >= LOGITS_TENSOR_MIN_N else 0)
 ATTN_SRC = os.path.join(ROOT, "dynamic_block_sparse_last_b200", "csrc", "attn_kernel.cuh")
 
 
@@ -480,7 +489,7 @@ def run_ours(args, w):
                             "hbm_floor_ms": hbm_floor_ms,
                             "exponentials": n_exp, "mufu_floor_ms": mufu_floor_ms},
              "attn_ms": attn_ms, "density": density, "chunks": chunks,
-             "e2e": e2e, "clocks": clocks, "gpu_launches": KERNELS_PER_STEP * args.steps,
+             "e2e": e2e, "clocks": clocks, "gpu_launches": kernels_per_step(w.S, w.b) * args.steps,
              "gpu": torch.cuda.get_device_name(dev)}
     extra["int8_peak"] = i8
     # compact forms of the same index on the device (not part of the step): CSR rows and the
@@ -521,7 +530,7 @@ def run_ours(args, w):
                          "density": Lb["density"], "chunks": Lb["chunks"],
                          "roofline": {"kernel": "k_sparse_attn", "bound": "tensor", "achieved": achb,
                                       "peak": peak, "unit": "TFLOP/s", "frac": achb / peak, "peak_source": src},
-                         "clocks": Lb["clocks"], "gpu_launches": KERNELS_PER_STEP * args.steps}
+                         "clocks": Lb["clocks"], "gpu_launches": kernels_per_step(wb.S, wb.b) * args.steps}
         Lb["idx"].free()
     if not w.int8 and not args.no_w8a8:
         # the W8A8 variant of the same layer: Q and K quantised per head from these bf16 tensors
@@ -545,7 +554,7 @@ def run_ours(args, w):
                                                       "at the bf16 sustained peak: 2/(1/P_i8 + 1/P_bf16)"
                                                       if i8_sus else "int8 at the nominal 2x of bf16")},
                          "clocks": L8["clocks"]}
-        extra["w8a8"]["gpu_launches"] = KERNELS_PER_STEP * args.steps
+        extra["w8a8"]["gpu_launches"] = kernels_per_step(wq.S, wq.b) * args.steps
         L8["idx"].free()
         del q8, k8
         idx = None

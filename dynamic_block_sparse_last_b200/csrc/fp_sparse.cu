@@ -40,6 +40,7 @@ struct fp_index {
   float *ksum;             // [Hkv][npart][128]
   float *kbar;             // [Hkv][n][128]
   float *qbar;             // [Hq][n][128]
+  float *qsplit, *ksplit;  // [Hq][n][256], [Hkv][n][256]: tf32 hi | lo of the block means (logits operands)
   float *vhat, *shat, *pest;  // [Hq][n]
   float *jsd;              // [Hq]
   int *pattern;            // [Hq]
@@ -160,6 +161,21 @@ bool make_map(CUtensorMap *m, const void *ptr, bool i8, uint64_t rows) {
   return r == CUDA_SUCCESS;
 }
 
+// Rows of 256 fp32 (a block mean split as tf32 hi | lo), 32-column x 128-row
+// boxes with the 128-byte swizzle: the operands of k_qa_logits.
+bool make_map_split(CUtensorMap *m, const float *ptr, uint64_t rows) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {256, rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(256 * 4)};
+  const cuuint32_t box[2] = {32u, 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 uint64_t map_rows(int H, int ld, int S) { return (uint64_t)(H - 1) * (uint64_t)ld + (uint64_t)S; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -200,6 +216,8 @@ int set_smem_attrs() {
     return FP_ERR_CUDA;
   if (cudaFuncSetAttribute(k_sparse_attn<I8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            AttnCfg<I8>::kSmem) != cudaSuccess)
+    return FP_ERR_CUDA;
+  if (cudaFuncSetAttribute(k_qa_logits, cudaFuncAttributeMaxDynamicSharedMemorySize, kLgSmem) != cudaSuccess)
     return FP_ERR_CUDA;
   d->attrs[I8] = true;
   return FP_OK;
@@ -307,9 +325,26 @@ int build_index_impl(const void *q, const void *k, float gamma, float tau, const
   }
   const float inv_sqrt_d = 1.0f / sqrtf((float)I->d);
   const float *kbar = ext_kbar ? ext_kbar : I->kbar;
-  const int nt = (I->n + kLgTile - 1) / kLgTile;
-  k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, qbar, kbar, I->g, I->n,
-                                                               inv_sqrt_d, I->zlog);
+  if (I->n >= kLgTensorMinN) {
+    // tensor cores: the logits' operands as tf32 hi | lo pairs (q-bar of the
+    // query-aware heads only), 128 x 128 tiles
+    const int qrows = I->Hq * I->n, krows = I->Hkv * I->n;
+    k_split_tf32<<<(qrows + 7) / 8, 256, 0, st>>>(qbar, I->qsplit, qrows, I->n, I->pattern);
+    if ((rc = launch_status())) return rc;
+    k_split_tf32<<<(krows + 7) / 8, 256, 0, st>>>(kbar, I->ksplit, krows, I->n, nullptr);
+    if ((rc = launch_status())) return rc;
+    CUtensorMap tmq, tmk;
+    if (!make_map_split(&tmq, I->qsplit, (uint64_t)qrows) || !make_map_split(&tmk, I->ksplit, (uint64_t)krows))
+      return FP_ERR_CUDA;
+    const int nt = (I->n + kLgTile - 1) / kLgTile;
+    k_qa_logits<<<dim3(nt * (nt + 1) / 2, I->Hq), 128, kLgSmem, st>>>(tmq, tmk, I->pattern, I->g, I->n,
+                                                                      inv_sqrt_d, err, I->zlog);
+  } else {
+    // too few 128 x 128 tiles to fill the GPU: 64 x 64 tiles on the FMA pipe
+    const int nt = (I->n + kLgFmaTile - 1) / kLgFmaTile;
+    k_qa_logits_fma<<<dim3(nt * (nt + 1) / 2, I->Hq), 256, 0, st>>>(I->pattern, qbar, kbar, I->g, I->n,
+                                                                     inv_sqrt_d, I->zlog);
+  }
   if ((rc = launch_status())) return rc;
   k_cut<<<(I->Hq * I->n + 7) / 8, 256, 0, st>>>(I->pattern, I->vhat, I->shat, I->zlog, I->Hq, I->n, gamma,
                                                I->counts, I->cols);
@@ -369,6 +404,9 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   add((size_t)Hkv * nch * 128 * 4);
   add((size_t)Hkv * n * 128 * 4);
   add((size_t)Hq * n * 128 * 4);
+  const size_t nsplit = n >= (size_t)kLgTensorMinN ? n : 0;  // tf32 operands only where the tensor-core logits run
+  add((size_t)Hq * nsplit * 256 * 4);
+  add((size_t)Hkv * nsplit * 256 * 4);
   for (int i = 0; i < 3; ++i) add((size_t)Hq * n * 4);
   add((size_t)Hq * 4);
   add((size_t)Hq * 4);
@@ -409,6 +447,8 @@ int index_create(int S, int ld, int Hq, int Hkv, int d, int b, fp_index **out) {
   I->ksum = carve<float>(cur, (size_t)Hkv * nch * 128);
   I->kbar = carve<float>(cur, (size_t)Hkv * n * 128);
   I->qbar = carve<float>(cur, (size_t)Hq * n * 128);
+  I->qsplit = carve<float>(cur, (size_t)Hq * nsplit * 256);
+  I->ksplit = carve<float>(cur, (size_t)Hkv * nsplit * 256);
   I->vhat = carve<float>(cur, (size_t)Hq * n);
   I->shat = carve<float>(cur, (size_t)Hq * n);
   I->pest = carve<float>(cur, (size_t)Hq * n);

@@ -17,7 +17,9 @@
 //                  block masses, vhat, shat, block means of K, P_est, JSD,
 //                  pattern.
 //   k_qpool        block means of Q of the query-aware heads.
-//   k_qa_logits    q-bar . k-bar logits of query-aware heads (tiled fp32).
+//   k_qa_logits    q-bar . k-bar logits of query-aware heads: tf32 hi/lo split
+//                  on the tensor cores (k_split_tf32 prepares the operands), or
+//                  tiled fp32 FMAs (k_qa_logits_fma) when n is small.
 //   k_cut          per (head, query block): scores, gamma cut, sorted list.
 #pragma once
 
@@ -838,7 +840,9 @@ __global__ void __maxnreg__(64)
 }
 
 // ---------------------------------------------------------------------------
-// k_qa_logits: grid (nt(nt+1)/2, Hq) with nt = ceil(n/64), block 256.  For
+// k_qa_logits_fma: grid (nt(nt+1)/2, Hq) with nt = ceil(n/64), block 256.  The
+// form for small n, where k_qa_logits (tensor cores, 128 x 128 tiles) has too
+// few tiles to fill the GPU; same output.  For
 // query-aware heads only (others exit): the lower triangle of
 // Z = qbar kbar^T / sqrt(d), z[h][r][c] for c <= r, in the padded triangular
 // layout (row r at h*n(n+1)/2 + r(r+1)/2).  Tiled fp32 product: 64 x 64
@@ -847,12 +851,12 @@ __global__ void __maxnreg__(64)
 // time, double-buffered (the next slice is loaded into registers while the
 // current one is multiplied).
 // ---------------------------------------------------------------------------
-constexpr int kLgTile = 64;
+constexpr int kLgFmaTile = 64;
 constexpr int kLgK = 32;
-constexpr int kLgStride = kLgTile + 4;  // float4-aligned rows
+constexpr int kLgStride = kLgFmaTile + 4;  // float4-aligned rows
 
 __global__ void __launch_bounds__(256)
-    k_qa_logits(const int *__restrict__ pattern, const float *__restrict__ qbar,
+    k_qa_logits_fma(const int *__restrict__ pattern, const float *__restrict__ qbar,
                 const float *__restrict__ kbar, int g, int n, float inv_sqrt_d, float *__restrict__ z) {
   const int h = blockIdx.y;
   if (pattern[h] != 1) return;
@@ -866,7 +870,7 @@ __global__ void __launch_bounds__(256)
   const int tc = x - tr * (tr + 1) / 2;
   const int kvh = h / g;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int row0 = tr * kLgTile, col0 = tc * kLgTile;
+  const int row0 = tr * kLgFmaTile, col0 = tc * kLgFmaTile;
   const float *qh = qbar + (size_t)h * n * 128;
   const float *kh = kbar + (size_t)kvh * n * 128;
   // this thread's share of a k-slice: rows rr0, rr0 + 32 of q-bar and k-bar, 4 consecutive k
@@ -931,6 +935,171 @@ __global__ void __launch_bounds__(256)
       const int c = col0 + tx * 4 + b2;
       if (c <= r) zh[(size_t)r * (r + 1) / 2 + c] = v[b2] * inv_sqrt_d;
     }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// k_split_tf32: one warp per row of 128 fp32 block means (block 256 = 8
+// rows); row r of src becomes row r of dst as 256 floats: x_hi = tf32(x) in
+// columns 0..127 and x_lo = tf32(x - x_hi) in columns 128..255 (nearest,
+// ties away).  With pattern given, rows of heads that are not query-aware
+// (head = row / n) are skipped.  The operands of k_qa_logits.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    k_split_tf32(const float *__restrict__ src, float *__restrict__ dst, int rows, int n,
+                 const int *__restrict__ pattern) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  if (pattern != nullptr && pattern[row / n] != 1) return;
+  const float4 v = *reinterpret_cast<const float4 *>(src + (size_t)row * 128 + lane * 4);
+  const float a[4] = {v.x, v.y, v.z, v.w};
+  uint32_t hi[4], lo[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    hi[e] = tf32_rna(a[e]);
+    lo[e] = tf32_rna(a[e] - __uint_as_float(hi[e]));
+  }
+  *reinterpret_cast<uint4 *>(dst + (size_t)row * 256 + lane * 4) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  *reinterpret_cast<uint4 *>(dst + (size_t)row * 256 + 128 + lane * 4) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+}
+
+// ---------------------------------------------------------------------------
+// k_qa_logits: grid (nt(nt+1)/2, Hq) with nt = ceil(n/128), block 128.  For
+// query-aware heads only (others exit): the lower triangle of
+// Z = qbar kbar^T / sqrt(d), z[h][r][c] for c <= r, in the padded triangular
+// layout (row r at h*n(n+1)/2 + r(r+1)/2), one 128 x 128 tile per CTA on the
+// tensor cores.  The operands come split by k_split_tf32 (x = x_hi + x_lo,
+// both tf32); the tile accumulates hi.hi + hi.lo + lo.hi in fp32 in tensor
+// memory (the dropped lo.lo term and the rounding of x_lo are below 2^-21 of
+// each product, the order of fp32 rounding).  Thread 0 streams d in four
+// slabs of 32 through a two-slot TMA ring (q_hi, q_lo, k_hi, k_lo: 128 rows
+// x 128 bytes each, 128-byte swizzle) and issues 12 MMAs (M = N = 128,
+// K = 8) per slab; a slot is refilled once its MMAs have completed.
+// Epilogue: warp w reads rows 32w.. of the accumulator, scales by 1/sqrt(d)
+// and stages them in shared memory; the CTA then writes each row's c <= r
+// part contiguously.
+// ---------------------------------------------------------------------------
+constexpr int kLgTile = 128;
+// smallest n that takes this kernel.  Below it the 64 x 64 FMA form, with
+// more CTAs and no split pass, is as fast or faster; measured index passes
+// (32 heads, half query-aware), tensor cores vs FMA: 0.144 vs 0.130 ms at
+// n = 256, 0.274 vs 0.260 at 512, 0.333 vs 0.327 at 640, 0.400 vs 0.398 at
+// 768, 0.471 vs 0.470 at 896, 0.529 vs 0.538 at 1024 (0.517 vs 0.529 int8)
+constexpr int kLgTensorMinN = 960;
+constexpr int kLgSlab = 16384;            // 128 rows x 32 tf32
+constexpr int kLgSlot = 4 * kLgSlab;      // q_hi, q_lo, k_hi, k_lo
+constexpr int kLgSmem = 2 * kLgSlot + 1024;
+constexpr int kLgStage = kLgTile + 1;     // staging row stride (floats)
+static_assert(kLgTile * kLgStage * 4 <= 2 * kLgSlot, "k_qa_logits staging exceeds the ring");
+
+__global__ void __launch_bounds__(128, 1)
+    k_qa_logits(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const int *__restrict__ pattern, int g, int n, float inv_sqrt_d, int *__restrict__ err,
+                float *__restrict__ z) {
+  const int h = blockIdx.y;
+  if (pattern[h] != 1) return;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t bar_full[2], bar_empty[2], bar_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  // lower-triangular tile (tr, tc), tc <= tr, from the linear index
+  const int x = blockIdx.x;
+  int tr = (int)((sqrtf(8.f * (float)x + 1.f) - 1.f) * 0.5f);
+  while ((tr + 1) * (tr + 2) / 2 <= x) ++tr;
+  while (tr * (tr + 1) / 2 > x) --tr;
+  const int tc = x - tr * (tr + 1) / 2;
+  const int kvh = h / g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  float *const stage = reinterpret_cast<float *>(smem_raw + (base - smem_u32(smem_raw)));
+  if (tid == 0) {
+    abort_sh = 0;
+    for (int sl = 0; sl < 2; ++sl) {
+      mbar_init(smem_u32(&bar_full[sl]), 1);
+      mbar_init(smem_u32(&bar_empty[sl]), 1);
+    }
+    mbar_init(smem_u32(&bar_done), 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(&tmem_base_sh), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  volatile int *abort_flag = &abort_sh;
+  if (tid == 0) {
+    tma_prefetch_map(&tm_q);
+    tma_prefetch_map(&tm_k);
+    const int qy = h * n + tr * kLgTile, ky = kvh * n + tc * kLgTile;
+    auto load = [&](int sb) {  // slab sb of d into slot sb & 1
+      const uint32_t dst = base + (sb & 1) * kLgSlot, bar = smem_u32(&bar_full[sb & 1]);
+      mbar_expect_tx(bar, kLgSlot);
+      tma_load_2d(dst + 0 * kLgSlab, &tm_q, 32 * sb, qy, bar);
+      tma_load_2d(dst + 1 * kLgSlab, &tm_q, 128 + 32 * sb, qy, bar);
+      tma_load_2d(dst + 2 * kLgSlab, &tm_k, 32 * sb, ky, bar);
+      tma_load_2d(dst + 3 * kLgSlab, &tm_k, 128 + 32 * sb, ky, bar);
+    };
+    const uint32_t idesc = idesc_tf32(128, 128);
+    load(0);
+    load(1);
+    bool ok = true;
+    for (int sb = 0; sb < 4 && ok; ++sb) {
+      const int sl = sb & 1;
+      if (!mbar_wait(smem_u32(&bar_full[sl]), (sb >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t sbase = base + sl * kLgSlot;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t a_hi = umma_desc_sw128(sbase + 0 * kLgSlab + kk * 32, 16, 1024);
+        const uint64_t a_lo = umma_desc_sw128(sbase + 1 * kLgSlab + kk * 32, 16, 1024);
+        const uint64_t b_hi = umma_desc_sw128(sbase + 2 * kLgSlab + kk * 32, 16, 1024);
+        const uint64_t b_lo = umma_desc_sw128(sbase + 3 * kLgSlab + kk * 32, 16, 1024);
+        mma_tf32_ss(tmem, a_hi, b_hi, idesc, (sb > 0 || kk > 0));
+        mma_tf32_ss(tmem, a_hi, b_lo, idesc, 1);
+        mma_tf32_ss(tmem, a_lo, b_hi, idesc, 1);
+      }
+      if (sb + 2 < 4) {
+        tc_commit(smem_u32(&bar_empty[sl]));
+        if (!mbar_wait(smem_u32(&bar_empty[sl]), 0, abort_flag, err)) { ok = false; break; }
+        load(sb + 2);
+      }
+    }
+    tc_commit(smem_u32(&bar_done));  // arrives once every MMA issued above has completed
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(smem_u32(&bar_done), 0, abort_flag, err) && !*abort_flag;
+  if (ok) {
+    tc_fence_after();
+    // accumulator row 32w + lane -> staging row (scaled)
+    const int row = warp * 32 + lane;
+#pragma unroll 1
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t v[32];
+      tmem_ld32(tmem + (((uint32_t)(warp * 32)) << 16) + q4 * 32, v);
+      tmem_ld_wait(v);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) stage[row * kLgStage + q4 * 32 + e] = __uint_as_float(v[e]) * inv_sqrt_d;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (ok) {
+    // row r of the tile: columns tc*128 + c with c <= rq, one contiguous run
+    float *zh = z + (size_t)h * ((size_t)n * (n + 1) / 2);
+#pragma unroll 1
+    for (int r = 0; r < kLgTile; ++r) {
+      const int rq = tr * kLgTile + r;
+      if (rq >= n) break;
+      const int cmax = rq - tc * kLgTile;  // last column of the run, tile-relative
+      if (tid <= cmax) zh[(size_t)rq * (rq + 1) / 2 + tc * kLgTile + tid] = stage[r * kLgStage + tid];
+    }
+  }
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
   }
 }
 

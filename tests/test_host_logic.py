@@ -143,3 +143,14 @@ def test_computed_chunk_tiles():
     # b = 64 with a last tile holding one query block (S = 192: blocks 0..2)
     rp, col = csr([[[0], [0, 1], [2]]])
     assert bench.computed_chunk_tiles(rp, col, 1, 192, 64) == 1 + 1
+
+
+def test_kernels_per_step_counts_the_tensor_core_logits_split():
+    """Six launches per layer step, two more (the tf32 operand splits) where the
+    q-bar . k-bar logits run on the tensor cores (n >= 960 blocks)."""
+    import bench
+    assert bench.kernels_per_step(131072, 128) == 8   # n = 1024
+    assert bench.kernels_per_step(131072, 256) == 6   # n = 512
+    assert bench.kernels_per_step(32768, 128) == 6    # n = 256
+    assert bench.kernels_per_step(122880, 128) == 8   # n = 960, the switch
+    assert bench.kernels_per_step(122752, 128) == 6   # n = 959
