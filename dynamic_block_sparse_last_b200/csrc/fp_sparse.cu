@@ -48,7 +48,7 @@ struct fp_index {
   int *cls;                // [Hq] head-sharing class representatives (fp_index_share)
   int *cover;              // [Hq] blocks covering gamma of vhat (fp_choose_block_size)
   int *gcount;             // [Hkv][n] union sizes of the group lists (fp_index_group_lists)
-  int shared;              // the lists are class unions (fp_index_share ran on this build)
+  int shared;              // the lists are class unions (fp_index_share ran after the last index build)
   int *cols;               // [Hq][n(n+1)/2]
   float *zlog;             // [Hq][n(n+1)/2] q-bar . k-bar logits (query-aware heads)
 };
