@@ -36,8 +36,8 @@ from dynamic_block_sparse_last_b200 import synth  # noqa: E402
 METRIC = "sparse-prefill ms/layer & dense-equiv TFLOPS at S=128K; % of HBM/TC roofline"
 UNIT = "dense-equiv TFLOP/s"
 # the library's switch of the q-bar . k-bar logits to the tensor cores (kLgTensorMinN in
-# index_kernels.cuh): from n = 960 blocks two k_split_tf32 launches precede k_qa_logits
-LOGITS_TENSOR_MIN_N = 960
+# index_kernels.cuh): from n = 640 blocks two k_split_tf32 launches precede k_qa_logits
+LOGITS_TENSOR_MIN_N = 640
 
 
 def kernels_per_step(S: int, b: int) -> int:

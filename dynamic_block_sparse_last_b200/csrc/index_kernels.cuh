@@ -972,34 +972,37 @@ __global__ void __launch_bounds__(256)
 // both tf32); the tile accumulates hi.hi + hi.lo + lo.hi in fp32 in tensor
 // memory (the dropped lo.lo term and the rounding of x_lo are below 2^-21 of
 // each product, the order of fp32 rounding).  Thread 0 streams d in four
-// slabs of 32 through a two-slot TMA ring (q_hi, q_lo, k_hi, k_lo: 128 rows
-// x 128 bytes each, 128-byte swizzle) and issues 12 MMAs (M = N = 128,
-// K = 8) per slab; a slot is refilled once its MMAs have completed.
+// slabs of 32 through one 64 KB shared-memory slot (q_hi, q_lo, k_hi, k_lo:
+// 128 rows x 128 bytes each, TMA with the 128-byte swizzle) and issues 12
+// MMAs (M = N = 128, K = 8) per slab; the slot is refilled once its MMAs
+// have completed.  With one slot three CTAs share an SM and hide each
+// other's load and MMA latencies (a two-slot ring with one CTA per SM
+// measured slower).
 // Epilogue: warp w reads rows 32w.. of the accumulator, scales by 1/sqrt(d)
-// and stages them in shared memory; the CTA then writes each row's c <= r
-// part contiguously.
+// and stages them in the slot (column c of row r at c ^ (r % 32): no bank
+// conflicts either way); the CTA then writes each row's c <= r part
+// contiguously.
 // ---------------------------------------------------------------------------
 constexpr int kLgTile = 128;
 // smallest n that takes this kernel.  Below it the 64 x 64 FMA form, with
 // more CTAs and no split pass, is as fast or faster; measured index passes
-// (32 heads, half query-aware), tensor cores vs FMA: 0.144 vs 0.130 ms at
-// n = 256, 0.274 vs 0.260 at 512, 0.333 vs 0.327 at 640, 0.400 vs 0.398 at
-// 768, 0.471 vs 0.470 at 896, 0.529 vs 0.538 at 1024 (0.517 vs 0.529 int8)
-constexpr int kLgTensorMinN = 960;
+// (32 heads, half query-aware), tensor cores (three CTAs per SM) vs FMA:
+// 0.267 vs 0.261 ms at n = 512, 0.384 vs 0.397 at 768, 0.512 vs 0.529 at
+// 1024 (0.501 vs 0.521 int8)
+constexpr int kLgTensorMinN = 640;
 constexpr int kLgSlab = 16384;            // 128 rows x 32 tf32
 constexpr int kLgSlot = 4 * kLgSlab;      // q_hi, q_lo, k_hi, k_lo
-constexpr int kLgSmem = 2 * kLgSlot + 1024;
-constexpr int kLgStage = kLgTile + 1;     // staging row stride (floats)
-static_assert(kLgTile * kLgStage * 4 <= 2 * kLgSlot, "k_qa_logits staging exceeds the ring");
+constexpr int kLgSmem = kLgSlot + 1024;   // one slot: three CTAs share an SM
+static_assert(kLgTile * kLgTile * 4 <= kLgSlot, "k_qa_logits staging exceeds the slot");
 
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(128, 3)
     k_qa_logits(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const int *__restrict__ pattern, int g, int n, float inv_sqrt_d, int *__restrict__ err,
                 float *__restrict__ z) {
   const int h = blockIdx.y;
   if (pattern[h] != 1) return;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ __align__(8) uint64_t bar_full[2], bar_empty[2], bar_done;
+  __shared__ __align__(8) uint64_t bar_full, bar_empty, bar_done;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
   // lower-triangular tile (tr, tc), tc <= tr, from the linear index
@@ -1014,10 +1017,8 @@ __global__ void __launch_bounds__(128, 1)
   float *const stage = reinterpret_cast<float *>(smem_raw + (base - smem_u32(smem_raw)));
   if (tid == 0) {
     abort_sh = 0;
-    for (int sl = 0; sl < 2; ++sl) {
-      mbar_init(smem_u32(&bar_full[sl]), 1);
-      mbar_init(smem_u32(&bar_empty[sl]), 1);
-    }
+    mbar_init(smem_u32(&bar_full), 1);
+    mbar_init(smem_u32(&bar_empty), 1);
     mbar_init(smem_u32(&bar_done), 1);
     fence_mbar_init();
   }
@@ -1034,37 +1035,34 @@ __global__ void __launch_bounds__(128, 1)
     tma_prefetch_map(&tm_q);
     tma_prefetch_map(&tm_k);
     const int qy = h * n + tr * kLgTile, ky = kvh * n + tc * kLgTile;
-    auto load = [&](int sb) {  // slab sb of d into slot sb & 1
-      const uint32_t dst = base + (sb & 1) * kLgSlot, bar = smem_u32(&bar_full[sb & 1]);
+    auto load = [&](int sb) {  // slab sb of d into the slot
+      const uint32_t bar = smem_u32(&bar_full);
       mbar_expect_tx(bar, kLgSlot);
-      tma_load_2d(dst + 0 * kLgSlab, &tm_q, 32 * sb, qy, bar);
-      tma_load_2d(dst + 1 * kLgSlab, &tm_q, 128 + 32 * sb, qy, bar);
-      tma_load_2d(dst + 2 * kLgSlab, &tm_k, 32 * sb, ky, bar);
-      tma_load_2d(dst + 3 * kLgSlab, &tm_k, 128 + 32 * sb, ky, bar);
+      tma_load_2d(base + 0 * kLgSlab, &tm_q, 32 * sb, qy, bar);
+      tma_load_2d(base + 1 * kLgSlab, &tm_q, 128 + 32 * sb, qy, bar);
+      tma_load_2d(base + 2 * kLgSlab, &tm_k, 32 * sb, ky, bar);
+      tma_load_2d(base + 3 * kLgSlab, &tm_k, 128 + 32 * sb, ky, bar);
     };
     const uint32_t idesc = idesc_tf32(128, 128);
     load(0);
-    load(1);
     bool ok = true;
     for (int sb = 0; sb < 4 && ok; ++sb) {
-      const int sl = sb & 1;
-      if (!mbar_wait(smem_u32(&bar_full[sl]), (sb >> 1) & 1, abort_flag, err)) { ok = false; break; }
+      if (!mbar_wait(smem_u32(&bar_full), sb & 1, abort_flag, err)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t sbase = base + sl * kLgSlot;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t a_hi = umma_desc_sw128(sbase + 0 * kLgSlab + kk * 32, 16, 1024);
-        const uint64_t a_lo = umma_desc_sw128(sbase + 1 * kLgSlab + kk * 32, 16, 1024);
-        const uint64_t b_hi = umma_desc_sw128(sbase + 2 * kLgSlab + kk * 32, 16, 1024);
-        const uint64_t b_lo = umma_desc_sw128(sbase + 3 * kLgSlab + kk * 32, 16, 1024);
+        const uint64_t a_hi = umma_desc_sw128(base + 0 * kLgSlab + kk * 32, 16, 1024);
+        const uint64_t a_lo = umma_desc_sw128(base + 1 * kLgSlab + kk * 32, 16, 1024);
+        const uint64_t b_hi = umma_desc_sw128(base + 2 * kLgSlab + kk * 32, 16, 1024);
+        const uint64_t b_lo = umma_desc_sw128(base + 3 * kLgSlab + kk * 32, 16, 1024);
         mma_tf32_ss(tmem, a_hi, b_hi, idesc, (sb > 0 || kk > 0));
         mma_tf32_ss(tmem, a_hi, b_lo, idesc, 1);
         mma_tf32_ss(tmem, a_lo, b_hi, idesc, 1);
       }
-      if (sb + 2 < 4) {
-        tc_commit(smem_u32(&bar_empty[sl]));
-        if (!mbar_wait(smem_u32(&bar_empty[sl]), 0, abort_flag, err)) { ok = false; break; }
-        load(sb + 2);
+      if (sb + 1 < 4) {
+        tc_commit(smem_u32(&bar_empty));
+        if (!mbar_wait(smem_u32(&bar_empty), sb & 1, abort_flag, err)) { ok = false; break; }
+        load(sb + 1);
       }
     }
     tc_commit(smem_u32(&bar_done));  // arrives once every MMA issued above has completed
@@ -1081,7 +1079,7 @@ __global__ void __launch_bounds__(128, 1)
       tmem_ld32(tmem + (((uint32_t)(warp * 32)) << 16) + q4 * 32, v);
       tmem_ld_wait(v);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) stage[row * kLgStage + q4 * 32 + e] = __uint_as_float(v[e]) * inv_sqrt_d;
+      for (int e = 0; e < 32; ++e) stage[row * kLgTile + ((q4 * 32 + e) ^ lane)] = __uint_as_float(v[e]) * inv_sqrt_d;
     }
   }
   tc_fence_before();
@@ -1094,7 +1092,7 @@ __global__ void __launch_bounds__(128, 1)
       const int rq = tr * kLgTile + r;
       if (rq >= n) break;
       const int cmax = rq - tc * kLgTile;  // last column of the run, tile-relative
-      if (tid <= cmax) zh[(size_t)rq * (rq + 1) / 2 + tc * kLgTile + tid] = stage[r * kLgStage + tid];
+      if (tid <= cmax) zh[(size_t)rq * (rq + 1) / 2 + tc * kLgTile + tid] = stage[r * kLgTile + (tid ^ (r & 31))];
     }
   }
   if (warp == 0) {

@@ -285,12 +285,12 @@ def test_full_size_layers(fp, name, ntiles):
 
 LARGE_N = [synth.Workload("b64_n1024", S=65536, Hq=8, Hkv=2, b=64, n_vertical=64, n_topics=32, seed=31),
            synth.Workload("b256_S131072", S=131072, Hq=8, Hkv=2, b=256, n_vertical=64, n_topics=32, seed=32),
-           # the q-bar . k-bar logits switch from the FMA form to the tensor cores at n = 960:
+           # the q-bar . k-bar logits switch from the FMA form to the tensor cores at n = 640:
            # a ragged n above it (partial last row band of 128 x 128 tiles, partial last block)
            # and n just below
-           synth.Workload("logits_tc_n1000_ragged", S=127960, Hq=8, Hkv=2, b=128, n_vertical=64, n_topics=32,
+           synth.Workload("logits_tc_n700_ragged", S=89550, Hq=8, Hkv=2, b=128, n_vertical=64, n_topics=32,
                           seed=40),
-           synth.Workload("logits_fma_n959", S=122752, Hq=8, Hkv=2, b=128, n_vertical=64, n_topics=32, seed=41)]
+           synth.Workload("logits_fma_n639", S=81792, Hq=8, Hkv=2, b=128, n_vertical=64, n_topics=32, seed=41)]
 
 
 @pytest.mark.parametrize("w", LARGE_N, ids=[w.name for w in LARGE_N])
@@ -298,7 +298,7 @@ def test_largest_block_counts(fp, w):
     """The largest index a block size allows or the longest layer at b = 256:
     n = 1024 blocks of 64 (every key-block bit of the attention bitmaps in
     use) and S = 131072 at b = 256; and the two sides of the logits kernels'
-    switch (n = 1000 ragged on the tensor cores, n = 959 on the FMA pipe);
+    switch (n = 700 ragged on the tensor cores, n = 639 on the FMA pipe);
     full index, 32 sampled tiles."""
     x = synth.make_inputs(w)
     exp, out, idx = run_gpu(fp, x, w)

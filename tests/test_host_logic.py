@@ -147,10 +147,10 @@ def test_computed_chunk_tiles():
 
 def test_kernels_per_step_counts_the_tensor_core_logits_split():
     """Six launches per layer step, two more (the tf32 operand splits) where the
-    q-bar . k-bar logits run on the tensor cores (n >= 960 blocks)."""
+    q-bar . k-bar logits run on the tensor cores (n >= 640 blocks)."""
     import bench
     assert bench.kernels_per_step(131072, 128) == 8   # n = 1024
     assert bench.kernels_per_step(131072, 256) == 6   # n = 512
     assert bench.kernels_per_step(32768, 128) == 6    # n = 256
-    assert bench.kernels_per_step(122880, 128) == 8   # n = 960, the switch
-    assert bench.kernels_per_step(122752, 128) == 6   # n = 959
+    assert bench.kernels_per_step(81920, 128) == 8    # n = 640, the switch
+    assert bench.kernels_per_step(81792, 128) == 6    # n = 639
