@@ -970,8 +970,8 @@ __global__ void __launch_bounds__(256)
 // layout (row r at h*n(n+1)/2 + r(r+1)/2), one 128 x 128 tile per CTA on the
 // tensor cores.  The operands come split by k_split_tf32 (x = x_hi + x_lo,
 // both tf32); the tile accumulates hi.hi + hi.lo + lo.hi in fp32 in tensor
-// memory (the dropped lo.lo term and the rounding of x_lo are below 2^-21 of
-// each product, the order of fp32 rounding).  Thread 0 streams d in four
+// memory (the dropped lo.lo term and the two roundings are each at most 2^-22
+// of a product, together below 2^-20: fp32-class).  Thread 0 streams d in four
 // slabs of 32 through one 64 KB shared-memory slot (q_hi, q_lo, k_hi, k_lo:
 // 128 rows x 128 bytes each, TMA with the 128-byte swizzle) and issues 12
 // MMAs (M = N = 128, K = 8) per slab; the slot is refilled once its MMAs
