@@ -15,7 +15,7 @@ import torch
 
 from dynamic_block_sparse_last_b200 import synth
 from oracle import oracle as orc
-from tests.test_gpu_parity import check_index, check_tiles
+from tests.test_gpu_parity import check_index, check_tiles, sampled_tiles
 
 pytestmark = pytest.mark.gpu
 
@@ -92,4 +92,29 @@ def test_index_on_pooled_means_matches_oracle(fp, w):
     check_index(P, exp, w)
     tiles = [(h, qc) for h in range(w.Hq) for qc in range(-(-w.S // 128))]
     check_tiles(P, exp, out, w, tiles)
+    idx.free()
+
+
+def test_index_on_pooled_means_tensor_core_logits(fp):
+    """n = 672 >= 640: the query-aware logits of the pooled build run on the
+    tensor cores, their operands split from the caller's block means.  Full
+    index against the oracle on its own rotated tensors, 24 sampled tiles."""
+    w = synth.Workload("rp_n672", S=86016, Hq=4, Hkv=2, b=128, seed=93)
+    x = synth.make_prerope_inputs(w)
+    q, k, qbar, kbar = gpu_rope_pool(fp, x, w)
+    v = x["v"].cuda()
+    idx = fp.fp_index_create(w.S, w.Hq, w.Hkv, w.d, w.b)
+    fp.fp_build_index_pooled(q, k, qbar, kbar, w.S, w.Hq, w.Hkv, w.d, w.b, w.gamma, w.tau, idx)
+    out = torch.empty_like(q)
+    fp.fp_sparse_attn(q, k, v, None, None, idx, out)
+    torch.cuda.synchronize()
+    assert fp.fp_get_device_error() == fp.FP_OK
+    exp = fp.fp_index_export(idx)
+    assert 1 in exp["pattern"].tolist(), "the case needs a query-aware head"
+    oq, _ = orc.rope_pool(x["q_in"], x["cos"], x["sin"], w.b)
+    ok, _ = orc.rope_pool(x["k_in"], x["cos"], x["sin"], w.b)
+    P = orc.OracleProblem(torch.from_numpy(oq).to(torch.bfloat16), torch.from_numpy(ok).to(torch.bfloat16),
+                          x["v"], w.b)
+    check_index(P, exp, w)
+    check_tiles(P, exp, out, w, sampled_tiles(w, 24, seed=w.seed))
     idx.free()

@@ -65,7 +65,9 @@ CASES = [("b128", [1000, 2048, 0, 77, 1500], 4, 2, 128, False),
          ("b256", [1300, 512, 2000], 6, 2, 256, False),
          ("int8", [2000, 129, 1024], 4, 2, 128, True),
          ("one_seq", [4096], 8, 2, 128, False),
-         ("b64", [1000, 333, 2048], 4, 2, 64, False)]
+         ("b64", [1000, 333, 2048], 4, 2, 64, False),
+         # a sequence with n = 700 blocks: its query-aware logits run on the tensor cores
+         ("long_tc", [700, 89550, 1000], 4, 2, 128, False)]
 
 
 @pytest.mark.parametrize("name,lens,Hq,Hkv,b,int8", CASES, ids=[c[0] for c in CASES])
