@@ -70,7 +70,9 @@ CASES = [(synth.WORKLOADS["tiny"], 0), (synth.WORKLOADS["tiny"], 1),
          (synth.WORKLOADS["tiny"], 4),
          (synth.Workload("pre_g4_shares", S=4096, Hq=8, Hkv=2, b=128, gamma=0.95, seed=41), 4),
          (synth.Workload("pre_int8_shares", S=2048, Hq=8, Hkv=4, b=128, int8=True, seed=43), 8),
-         (synth.Workload("pre_ragged_shares", S=1300, Hq=6, Hkv=2, b=256, seed=44), 6)]
+         (synth.Workload("pre_ragged_shares", S=1300, Hq=6, Hkv=2, b=256, seed=44), 6),
+         # n = 700 blocks: the groups' query-aware logits run on the tensor cores
+         (synth.Workload("pre_long_tc", S=89550, Hq=4, Hkv=2, b=128, seed=45), 2)]
 
 
 @pytest.mark.parametrize("w,groups", CASES, ids=[f"{w.name}-G{g}" for w, g in CASES])
