@@ -49,13 +49,26 @@ def kernels_per_step(S: int, b: int) -> int:
 ATTN_SRC = os.path.join(ROOT, "dynamic_block_sparse_last_b200", "csrc", "attn_kernel.cuh")
 
 
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
 def load_peaks():
+    """Roofline denominators: the measured copy bandwidth (GB/s) and bf16 GEMM
+    throughput (TFLOP/s, burst and sustained) from MEASURED_PEAKS.json beside
+    this file, else the pool's earlier measurement (source "fallback").  A file
+    without positive numbers under those keys counts as absent."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        d = json.load(open(p))
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
-                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+        try:
+            d = json.load(open(p))
+            hbm, burst = float(d["hbm_gbs"]), float(d["bf16_tflops"])
+            sus = float(d.get("bf16_tflops_sustained", burst))
+            if hbm > 0 and burst > 0 and sus > 0:
+                return {"hbm_gbs": hbm, "bf16_tflops": burst, "bf16_tflops_sustained": sus, "source": "measured"}
+        except (ValueError, TypeError, KeyError, json.JSONDecodeError):
+            pass
+        return dict(FALLBACK_PEAKS, source="fallback (MEASURED_PEAKS.json unreadable)")
+    return dict(FALLBACK_PEAKS, source="fallback")
 
 
 def attn_traffic_record():
@@ -451,8 +464,8 @@ def run_ours(args, w):
 
     peaks = load_peaks()
     bf16_peak = peaks["bf16_tflops_sustained"]
-    src = (f"{peaks['source']} bf16 sustained (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
-           else "fallback 1.4 PFLOP/s sustained")
+    src = ("measured bf16 sustained (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
+           else f"{peaks['source']}: 1.4 PFLOP/s sustained")
     i8 = int8_gemm_peak(dev) if (w.int8 or not args.no_w8a8) else None
     i8_sus = i8.get("sustained_tops") if i8 else None
     if w.int8 and i8_sus:

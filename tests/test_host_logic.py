@@ -154,3 +154,21 @@ def test_kernels_per_step_counts_the_tensor_core_logits_split():
     assert bench.kernels_per_step(32768, 128) == 6    # n = 256
     assert bench.kernels_per_step(81920, 128) == 8    # n = 640, the switch
     assert bench.kernels_per_step(81792, 128) == 6    # n = 639
+
+
+def test_load_peaks_reads_the_measured_file_and_falls_back(tmp_path, monkeypatch):
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    p = bench.load_peaks()
+    assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0 and p["bf16_tflops_sustained"] == 1400.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(
+        json.dumps({"hbm_gbs": 6550, "bf16_tflops": 1644.9, "bf16_tflops_sustained": 1403.3, "other": [1]}))
+    p = bench.load_peaks()
+    assert p["source"] == "measured" and p["hbm_gbs"] == 6550.0 and p["bf16_tflops_sustained"] == 1403.3
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6550, "bf16_tflops": 1644.9}))
+    assert bench.load_peaks()["bf16_tflops_sustained"] == 1644.9   # no sustained figure: the burst one
+    for bad in ('{"hbm_gbs": {"value": 6550}, "bf16_tflops": 1644.9}', '{"bf16_tflops": 1}', 'not json',
+                '{"hbm_gbs": 0, "bf16_tflops": 1644.9}'):
+        (tmp_path / "MEASURED_PEAKS.json").write_text(bad)
+        p = bench.load_peaks()
+        assert p["source"].startswith("fallback") and p["hbm_gbs"] == 6650.0, bad
